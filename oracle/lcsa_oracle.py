@@ -1,0 +1,266 @@
+"""CPU oracle for the hybrid compressed-attention hot path (CSA / HCA).
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, FP64 statement of
+what the library computes.  Only the tests, the smoke check and the bench's
+CPU-baseline leg may import it; the product path never does.  It shares no
+code with the CUDA library.
+
+Sources (web pages about DeepSeek-V4):
+  [p1] "DeepSeek V4的4个技巧", section 1 "技巧1：混合注意力"
+  [p2] "深度解析 DeepSeek-V4：百万级长文本的低成本突破", sections
+       "CSA：Compressed Sparse Attention" (Step 1 Compress, Step 2 Select, the
+       ASCII figure), "HCA：Heavily Compressed Attention",
+       "Sliding Window Branch", "Attention Sink"
+  [p3] untitled classical-Chinese paraphrase page, the sentences headed
+       "Partial RoPE", "Attention sink", "第一步，KV压缩", "第二步，lightning
+       indexer + top-k选择", "第三步，core attention" and the strict-causality,
+       HCA-no-overlap and sliding-window sentences
+  [p4] "DeepSeek V4 技术架构深度解析", section "二、CSA + HCA"
+
+Readings of points the pages leave open:
+  * gate granularity: one softmax over the window's tokens per channel; a
+    per-token gate is the broadcast case;
+  * the CSA window of entry j is the 2m tokens [(j-1)m, (j+1)m) clipped at 0,
+    the HCA window is [j m', (j+1) m'); an entry exists only for complete
+    own-blocks, so there are floor(T/m) of them;
+  * entry j is visible to the query at position t iff j < floor(t/m);
+  * indexer score s[t,j] = sum_h w[t,h] * relu(q_I[t,h] . k_I[j]), no scale;
+  * top-k: the k largest scores among the visible entries, ties to the lower
+    index, indices emitted ascending, -1 padded;
+  * RoPE on the last R dims, adjacent pairs (2i, 2i+1) of that slice,
+    theta_i = base^(-2i/R); compressed entry j sits at position j*m, raw token
+    s at position s; the rotated entry is both key and value; the output's
+    rotary slice is rotated back by -t;
+  * logits scale 1/sqrt(D); window = raw tokens s with t-W < s <= t;
+    sink = one logit per head added as exp(sigma_h) to the denominator.
+
+Parity pins: every function here is checked in tests/test_oracle_pins.py
+against closed forms, a library attention routine, brute force and values the
+pages print.
+"""
+import numpy as np
+
+__all__ = [
+    "compress", "csa_compress", "hca_compress",
+    "n_visible", "indexer_scores", "topk_select", "topk_from_scores", "indexer_topk",
+    "rope_rotate", "attend_one", "csa_sparse_attn", "hca_dense_attn",
+]
+
+
+# ----------------------------------------------------------------------------
+# Step 1: KV compression  ([p2] CSA Step 1: m consecutive tokens are merged into
+# one entry with learned softmax weights; [p3] "第一步，KV压缩" and the sentence on
+# an attention-like pooling with learned weights; [p3] the sentence saying HCA
+# pools every m' tokens without CSA's overlap)
+# ----------------------------------------------------------------------------
+def compress(kv, gate, m, window, rms_weight=None, rms_eps=1e-6):
+    """Pool a [T, D] token sequence into floor(T/m) entries.
+
+    Entry j pools the tokens [(j+1)m - window, (j+1)m) clipped at 0 with
+    softmax weights taken over those tokens, separately for every channel:
+        c[j,d] = sum_i softmax_i(gate[i,d]) * kv[i,d].
+    gate may be [T, D] (per channel) or [T] (one logit per token).
+    With rms_weight, c[j] is RMS-normalised and scaled ([p2] "Attention Sink"
+    section, last paragraph: RMSNorm on the compressed KV entries).
+    """
+    kv = np.asarray(kv, dtype=np.float64)
+    gate = np.asarray(gate, dtype=np.float64)
+    T, D = kv.shape
+    if gate.ndim == 1:
+        gate = np.repeat(gate[:, None], D, axis=1)
+    Nc = T // m
+    out = np.zeros((Nc, D), dtype=np.float64)
+    for j in range(Nc):
+        hi = (j + 1) * m
+        lo = max(0, hi - window)
+        g = gate[lo:hi]
+        e = np.exp(g - g.max(axis=0, keepdims=True))
+        wts = e / e.sum(axis=0, keepdims=True)
+        out[j] = (wts * kv[lo:hi]).sum(axis=0)
+    if rms_weight is not None:
+        rms = np.sqrt(np.mean(out * out, axis=1, keepdims=True) + rms_eps)
+        out = out / rms * np.asarray(rms_weight, dtype=np.float64)[None, :]
+    return out
+
+
+def csa_compress(kv, gate, m=4, rms_weight=None, rms_eps=1e-6):
+    """CSA: overlapping 2m window with stride m."""
+    return compress(kv, gate, m, 2 * m, rms_weight, rms_eps)
+
+
+def hca_compress(kv, gate, m=128, rms_weight=None, rms_eps=1e-6):
+    """HCA: non-overlapping blocks of m tokens."""
+    return compress(kv, gate, m, m, rms_weight, rms_eps)
+
+
+def n_visible(t, m, n_c):
+    """Compressed entries visible to the query at absolute position t:
+    j < floor(t/m) ([p3] strict causality: a query does not see the other
+    tokens of its own compressed block)."""
+    return int(max(0, min(n_c, t // m)))
+
+
+# ----------------------------------------------------------------------------
+# Step 2: Lightning Indexer + top-k  ([p2] CSA Step 2 "Select" and the ASCII
+# figure; [p3] "第二步，lightning indexer + top-k选择" and the sentence on a
+# light indexer scoring every compressed block against each query token)
+# ----------------------------------------------------------------------------
+def indexer_scores(q_idx, w, k_idx, q_pos0, m):
+    """Scores [Tq, Nc] in FP64; entries that are not visible are -inf.
+
+    s[t,j] = sum_h w[t,h] * max(0, q_I[t,h,:] . k_I[j,:]).
+    """
+    q_idx = np.asarray(q_idx, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    k_idx = np.asarray(k_idx, dtype=np.float64)
+    Tq = q_idx.shape[0]
+    Nc = k_idx.shape[0]
+    s = np.full((Tq, Nc), -np.inf, dtype=np.float64)
+    for i in range(Tq):
+        nv = n_visible(q_pos0 + i, m, Nc)
+        if nv == 0:
+            continue
+        dots = q_idx[i] @ k_idx[:nv].T           # [H_I, nv]
+        s[i, :nv] = w[i] @ np.maximum(dots, 0.0)
+    return s
+
+
+def topk_select(row, k):
+    """Indices of the k largest values of `row` (ties to the lower index),
+    returned ascending and padded with -1 to length k."""
+    row = np.asarray(row, dtype=np.float64)
+    assert not np.isnan(row).any(), "NaN score"
+    n = row.shape[0]
+    j = np.arange(n)
+    order = np.lexsort((j, -row))               # primary: score descending; then index ascending
+    chosen = np.sort(order[:min(k, n)])
+    out = np.full(k, -1, dtype=np.int64)
+    out[:chosen.shape[0]] = chosen
+    return out
+
+
+def topk_from_scores(scores, n_valid, k):
+    """Row-wise selection over the first n_valid[r] columns of each row."""
+    scores = np.asarray(scores)
+    out = np.full((scores.shape[0], k), -1, dtype=np.int64)
+    for r in range(scores.shape[0]):
+        nv = int(n_valid[r])
+        if nv > 0:
+            out[r] = topk_select(scores[r, :nv], k)
+    return out
+
+
+def indexer_topk(q_idx, w, k_idx, q_pos0, m, k, score_dtype=np.float32):
+    """Scores in FP64, rounded to the selection precision (FP32, the kernel's),
+    then the top-k of the visible prefix of every row."""
+    s = indexer_scores(q_idx, w, k_idx, q_pos0, m)
+    Tq, Nc = s.shape
+    nv = [n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+    s_sel = s.astype(score_dtype).astype(np.float64)
+    return topk_from_scores(s_sel, nv, k), s
+
+
+# ----------------------------------------------------------------------------
+# Step 3: core attention  ([p3] "第三步，core attention", "Partial RoPE",
+# "Attention sink", the sliding-window sentence; [p2] "Sliding Window Branch",
+# "Attention Sink")
+# ----------------------------------------------------------------------------
+def rope_rotate(x, pos, R, base=10000.0):
+    """Rotate the last R dims of x[..., D] by angle pos*theta_i per adjacent
+    pair (2i, 2i+1) of that slice, theta_i = base^(-2i/R).  pos broadcasts
+    against x's leading dims."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    if R == 0:
+        return x
+    D = x.shape[-1]
+    i = np.arange(R // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / R)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    c, s = np.cos(ang), np.sin(ang)
+    a = x[..., D - R::2].copy()
+    b = x[..., D - R + 1::2].copy()
+    x[..., D - R::2] = a * c - b * s
+    x[..., D - R + 1::2] = a * s + b * c
+    return x
+
+
+def attend_one(q_t, t, entries, ckv, m, kv, kv_pos0, W, sink, R, base=10000.0, scale=None):
+    """One query position t, all heads.
+
+    Keys (= values): the compressed entries `entries` (each rotated at j*m)
+    followed by the raw window tokens s with t-W < s <= t that kv holds
+    (rows kv_pos0 .. kv_pos0+len(kv)-1, each rotated at s).  One softmax over
+    all of them with exp(sink_h) added to the denominator; the output's rotary
+    slice is rotated by -t.  Returns (out [H,D], lse [H]) with
+    lse = log(sum exp(logits) + exp(sink)).
+    """
+    q_t = np.asarray(q_t, dtype=np.float64)
+    H, D = q_t.shape
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    entries = np.asarray(entries, dtype=np.int64)
+    keys = []
+    if entries.size:
+        keys.append(rope_rotate(np.asarray(ckv, dtype=np.float64)[entries], entries * m, R, base))
+    lo = max(t - W + 1, kv_pos0, 0)
+    hi = min(t, kv_pos0 + kv.shape[0] - 1)
+    if hi >= lo:
+        s = np.arange(lo, hi + 1)
+        keys.append(rope_rotate(np.asarray(kv, dtype=np.float64)[s - kv_pos0], s, R, base))
+    qr = rope_rotate(q_t, t, R, base)
+    sink = None if sink is None else np.asarray(sink, dtype=np.float64)
+    if not keys:
+        out = np.zeros((H, D))
+        lse = np.full(H, -np.inf) if sink is None else sink.copy()
+        return out, lse
+    K = np.concatenate(keys, axis=0)                 # [n, D]
+    logits = scale * (qr @ K.T)                      # [H, n]
+    mx = logits.max(axis=1)
+    if sink is not None:
+        mx = np.maximum(mx, sink)
+    e = np.exp(logits - mx[:, None])
+    denom = e.sum(axis=1)
+    if sink is not None:
+        denom = denom + np.exp(sink - mx)
+    out = (e @ K) / denom[:, None]
+    out = rope_rotate(out, -t, R, base)
+    return out, mx + np.log(denom)
+
+
+def _rows(B, Tq, rows):
+    if rows is None:
+        return [(b, i) for b in range(B) for i in range(Tq)]
+    return list(rows)
+
+
+def csa_sparse_attn(q, ckv, idx, kv, q_pos0, kv_pos0, m, W, sink, R, base=10000.0,
+                    scale=None, rows=None):
+    """CSA core attention over the selected entries idx[b,i,:] (>= 0 only).
+
+    q [B,Tq,H,D], ckv [B,Nc,D], idx [B,Tq,k], kv [B,Tkv,D].
+    Returns (out [n,H,D], lse [n,H]) for the (b, i) pairs in `rows`
+    (all rows when None)."""
+    B, Tq = q.shape[0], q.shape[1]
+    outs, lses = [], []
+    for b, i in _rows(B, Tq, rows):
+        sel = np.asarray(idx[b, i])
+        sel = sel[sel >= 0]
+        assert (sel < ckv.shape[1]).all()
+        o, l = attend_one(q[b, i], q_pos0 + i, sel, ckv[b], m, kv[b], kv_pos0, W, sink, R, base, scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+def hca_dense_attn(q, ckv, kv, q_pos0, kv_pos0, m, W, sink, R, base=10000.0,
+                   scale=None, rows=None):
+    """HCA core attention over every visible entry j < floor(t/m)."""
+    B, Tq = q.shape[0], q.shape[1]
+    Nc = ckv.shape[1]
+    outs, lses = [], []
+    for b, i in _rows(B, Tq, rows):
+        t = q_pos0 + i
+        sel = np.arange(n_visible(t, m, Nc))
+        o, l = attend_one(q[b, i], t, sel, ckv[b], m, kv[b], kv_pos0, W, sink, R, base, scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)

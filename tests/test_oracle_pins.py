@@ -1,0 +1,338 @@
+"""Pins for the CPU oracle: closed forms, brute force, a library attention
+routine and values the pages print.  Each test targets a mistake that a
+plausible bug in the oracle would make (dropped term, wrong sign or index,
+transposed operand, off-by-one visibility)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lcsa_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- compress
+@pytest.mark.parametrize("m,window", [(4, 8), (128, 128), (3, 6)])
+def test_compress_equal_gates_is_block_mean(m, window):
+    r = _rng(1)
+    T, D = 10 * m + (m - 1), 7          # ragged tail: last partial block gets no entry
+    kv = r.standard_normal((T, D))
+    gate = np.tile(r.standard_normal((1, D)), (T, 1))  # equal over tokens, per channel
+    out = O.compress(kv, gate, m, window)
+    assert out.shape == (T // m, D)
+    for j in range(T // m):
+        lo, hi = max(0, (j + 1) * m - window), (j + 1) * m
+        np.testing.assert_allclose(out[j], kv[lo:hi].mean(axis=0), rtol=0, atol=1e-13)
+
+
+def test_csa_window_is_previous_plus_own_block():
+    # one-hot gate: the single token with i % 2m == 1 dominates every 2m window
+    m, T, D = 4, 64, 5
+    r = _rng(2)
+    kv = r.standard_normal((T, D))
+    gate = np.where((np.arange(T) % (2 * m)) == 1, 80.0, 0.0)
+    out = O.csa_compress(kv, gate, m)
+    for j in range(T // m):
+        lo, hi = max(0, (j - 1) * m), (j + 1) * m
+        (star,) = [i for i in range(lo, hi) if i % (2 * m) == 1]
+        np.testing.assert_allclose(out[j], kv[star], atol=1e-30 + 1e-12)
+
+
+def test_hca_permutation_within_block_invariant():
+    m, T, D = 16, 64, 6
+    r = _rng(3)
+    kv = r.standard_normal((T, D))
+    gate = r.standard_normal((T, D))
+    perm = np.concatenate([b * m + r.permutation(m) for b in range(T // m)])
+    np.testing.assert_allclose(O.hca_compress(kv, gate, m), O.hca_compress(kv[perm], gate[perm], m),
+                               atol=1e-13)
+
+
+def test_compress_scalar_gate_is_broadcast():
+    r = _rng(4)
+    kv = r.standard_normal((40, 9))
+    g = r.standard_normal(40)
+    np.testing.assert_array_equal(O.csa_compress(kv, g, 4), O.csa_compress(kv, np.repeat(g[:, None], 9, 1), 4))
+
+
+def test_compress_causal_prefix():
+    r = _rng(5)
+    kv = r.standard_normal((48, 4))
+    gate = r.standard_normal((48, 4))
+    base = O.csa_compress(kv, gate, 4)
+    kv2, g2 = kv.copy(), gate.copy()
+    kv2[24:] += 5.0
+    g2[24:] -= 3.0
+    out2 = O.csa_compress(kv2, g2, 4)
+    np.testing.assert_array_equal(base[:6], out2[:6])     # entry 5 pools tokens 16..23
+    assert not np.allclose(base[6], out2[6])              # entry 6 pools 20..27
+
+
+def test_compress_rmsnorm_unit_rms():
+    r = _rng(6)
+    kv = r.standard_normal((32, 16))
+    gate = r.standard_normal((32, 16))
+    out = O.csa_compress(kv, gate, 4, rms_weight=np.full(16, 2.0), rms_eps=0.0)
+    np.testing.assert_allclose(np.sqrt((out ** 2).mean(axis=1)), 2.0, rtol=1e-12)
+
+
+def test_entry_counts_golden():
+    """1M tokens give 250K CSA entries and about 7,800 HCA entries."""
+    g = json.load(open(os.path.join(GOLD, "entry_counts.json")))
+    T = g["T"]
+    z = np.zeros((T, 1))
+    assert O.csa_compress(z, z[:, 0], g["csa_m"]).shape[0] == g["csa_entries"]
+    hca = O.hca_compress(z, z[:, 0], g["hca_m"]).shape[0]
+    assert abs(hca - g["hca_entries_approx"]) / g["hca_entries_approx"] < g["approx_rel_tol"]
+
+
+# ---------------------------------------------------------------- indexer
+def test_indexer_single_head_bruteforce():
+    r = _rng(7)
+    Tq, Nc, D_I, m, q_pos0 = 6, 9, 5, 4, 20
+    q = r.standard_normal((Tq, 1, D_I))
+    k = r.standard_normal((Nc, D_I))
+    w = np.ones((Tq, 1))
+    s = O.indexer_scores(q, w, k, q_pos0, m)
+    for i in range(Tq):
+        t = q_pos0 + i
+        for j in range(Nc):
+            if j < t // m:
+                dot = math.fsum(float(q[i, 0, d]) * float(k[j, d]) for d in range(D_I))
+                assert s[i, j] == pytest.approx(max(0.0, dot), abs=1e-12)
+            else:
+                assert s[i, j] == -np.inf
+
+
+def test_indexer_relu_per_head_then_weighted_sum():
+    r = _rng(8)
+    Tq, H, Nc, D_I = 3, 4, 12, 6
+    q = r.standard_normal((Tq, H, D_I))
+    k = r.standard_normal((Nc, D_I))
+    w1 = r.standard_normal((Tq, H))
+    w2 = r.standard_normal((Tq, H))
+    s1 = O.indexer_scores(q, w1, k, 100, 4)
+    s2 = O.indexer_scores(q, w2, k, 100, 4)
+    s12 = O.indexer_scores(q, w1 + w2, k, 100, 4)
+    np.testing.assert_allclose(s12, s1 + s2, atol=1e-12)       # linear in w => ReLU is per head
+    # a single head with weight -1 gives -relu(dot): never positive
+    s_neg = O.indexer_scores(q[:, :1], -np.ones((Tq, 1)), k, 100, 4)
+    assert (s_neg <= 0).all()
+    # heads are a set: permuting heads of q and w together changes nothing
+    p = r.permutation(H)
+    np.testing.assert_allclose(O.indexer_scores(q[:, p], w1[:, p], k, 100, 4), s1, atol=1e-12)
+
+
+def test_visibility_boundary():
+    # j visible iff j < floor(t/m): m=4 -> t=0..3 see 0, t=4..7 see 1, t=8 sees 2
+    assert [O.n_visible(t, 4, 100) for t in range(10)] == [0, 0, 0, 0, 1, 1, 1, 1, 2, 2]
+    assert O.n_visible(10 ** 6, 4, 250000) == 250000
+    assert O.n_visible(127, 128, 8) == 0 and O.n_visible(128, 128, 8) == 1
+
+
+# ---------------------------------------------------------------- top-k
+def test_topk_golden_toy():
+    g = json.load(open(os.path.join(GOLD, "topk_toy.json")))
+    assert list(O.topk_select(g["scores"], g["k"])) == g["expected_idx"]
+
+
+def test_topk_all_equal_and_short_rows():
+    assert list(O.topk_select(np.full(10, 0.5), 4)) == [0, 1, 2, 3]
+    assert list(O.topk_select(np.array([3.0, 1.0, 2.0]), 5)) == [0, 1, 2, -1, -1]
+    # signed zeros are equal: ties go to the lower index
+    assert list(O.topk_select(np.array([-0.0, 0.0, -1.0, -0.0]), 2)) == [0, 1]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_bruteforce_subsets(seed):
+    r = _rng(100 + seed)
+    n, k = 9, 4
+    row = np.round(r.standard_normal(n) * 2) / 2        # frequent ties
+    def beats(i, j):                                     # i ranks above j
+        return row[i] > row[j] or (row[i] == row[j] and i < j)
+    valid = [S for S in itertools.combinations(range(n), k)
+             if all(beats(i, j) for i in S for j in range(n) if j not in S)]
+    assert len(valid) == 1
+    assert list(O.topk_select(row, k)) == list(valid[0])
+
+
+def test_topk_from_scores_respects_n_valid():
+    s = np.array([[5.0, 4.0, 3.0, 9.0], [1.0, 2.0, 3.0, 4.0]])
+    out = O.topk_from_scores(s, [2, 0], 3)
+    assert out.tolist() == [[0, 1, -1], [-1, -1, -1]]
+
+
+# ---------------------------------------------------------------- rope
+def test_rope_matches_complex_rotation():
+    r = _rng(9)
+    D, R = 12, 8
+    x = r.standard_normal((3, D))
+    pos = np.array([0.0, 5.0, 1234567.0])
+    y = O.rope_rotate(x, pos, R, 10000.0)
+    np.testing.assert_array_equal(y[:, :D - R], x[:, :D - R])
+    z = x[:, D - R::2] + 1j * x[:, D - R + 1::2]
+    theta = 10000.0 ** (-np.arange(R // 2) * 2.0 / R)
+    zr = z * np.exp(1j * pos[:, None] * theta[None, :])
+    np.testing.assert_allclose(y[:, D - R::2], zr.real, atol=1e-9)
+    np.testing.assert_allclose(y[:, D - R + 1::2], zr.imag, atol=1e-9)
+    np.testing.assert_allclose(O.rope_rotate(y, -pos, R), x, atol=1e-9)
+
+
+# ---------------------------------------------------------------- attention
+def _complex_rot(x, pos, R, base=10000.0):
+    """Independent restatement of the rotary map through complex numbers."""
+    x = np.array(x, dtype=np.float64)
+    D = x.shape[-1]
+    if R == 0:
+        return x
+    z = x[..., D - R::2] + 1j * x[..., D - R + 1::2]
+    theta = base ** (-np.arange(R // 2) * 2.0 / R)
+    z = z * np.exp(1j * np.asarray(pos, dtype=np.float64)[..., None] * theta)
+    y = x.copy()
+    y[..., D - R::2] = z.real
+    y[..., D - R + 1::2] = z.imag
+    return y
+
+
+@pytest.mark.parametrize("R", [0, 8])
+def test_m1_window1_reduces_to_causal_sdpa(R):
+    """m=1, W=1, no sink: HCA is ordinary causal single-KV-head attention."""
+    r = _rng(10 + R)
+    T, H, D = 17, 3, 16
+    kv = r.standard_normal((1, T, D))
+    q = r.standard_normal((1, T, H, D))
+    ckv = O.hca_compress(kv[0], r.standard_normal((T, D)), 1)[None]   # m=1: entries are the tokens
+    np.testing.assert_array_equal(ckv[0], kv[0])
+    out, lse = O.hca_dense_attn(q, ckv, kv, 0, 0, 1, 1, None, R)
+    pos = np.arange(T)
+    qr = torch.from_numpy(_complex_rot(q[0], pos[:, None], R)).permute(1, 0, 2)   # [H,T,D]
+    kr = torch.from_numpy(_complex_rot(kv[0], pos, R))[None].expand(H, T, D)
+    ref = torch.nn.functional.scaled_dot_product_attention(qr, kr, kr, is_causal=True)
+    ref = _complex_rot(ref.permute(1, 0, 2).numpy(), -pos[:, None], R)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+    logits = torch.einsum("htd,sd->hts", qr, kr[0]) / math.sqrt(D)
+    mask = torch.triu(torch.ones(T, T, dtype=torch.bool), 1)
+    ref_lse = torch.logsumexp(logits.masked_fill(mask, -float("inf")), dim=-1).T.numpy()
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12)
+
+
+def test_sink_closed_form_zero_query():
+    r = _rng(11)
+    H, D, T = 2, 8, 40
+    kv = r.standard_normal((1, T, D))
+    ckv = r.standard_normal((1, T // 4, D))
+    sink = np.array([0.7, -1.3])
+    q = np.zeros((1, 1, H, D))
+    t = 25
+    n_keys = O.n_visible(t, 4, T // 4) + 8            # entries 0..5 plus window of 8 raw tokens
+    out, lse = O.hca_dense_attn(q, ckv, kv, t, 0, 4, 8, sink, R=0, rows=[(0, 0)])
+    expect = (ckv[0, :6].sum(0) + kv[0, t - 7:t + 1].sum(0))[None, :] / (n_keys + np.exp(sink))[:, None]
+    np.testing.assert_allclose(out[0], expect, atol=1e-13)
+    np.testing.assert_allclose(lse[0], np.log(n_keys + np.exp(sink)), atol=1e-13)
+
+
+def test_sink_weights_sum_below_one():
+    r = _rng(12)
+    H, D = 3, 8
+    u = r.standard_normal(D)
+    kv = np.tile(u, (1, 20, 1))
+    ckv = np.tile(u, (1, 5, 1))
+    q = r.standard_normal((1, 1, H, D))
+    for sink, lo, hi in [(np.zeros(H), 0.0, 1.0), (np.full(H, -1e3), 1 - 1e-12, 1 + 1e-12)]:
+        out, _ = O.hca_dense_attn(q, ckv, kv, 19, 0, 4, 4, sink, R=0, rows=[(0, 0)])
+        ratio = out[0] / u[None, :]
+        assert (ratio > lo).all() and (ratio < hi).all()
+    out, _ = O.hca_dense_attn(q, ckv, kv, 19, 0, 4, 4, None, R=0, rows=[(0, 0)])
+    np.testing.assert_allclose(out[0] / u[None, :], 1.0, atol=1e-12)
+
+
+def test_single_window_key_closed_form():
+    """No visible entry and W=1: out = kv_t * sigmoid(l - sigma) with the
+    relative-position logit l = q.kv_t/sqrt(D) (the -t rotation cancels)."""
+    r = _rng(13)
+    H, D, R = 2, 16, 8
+    kv = r.standard_normal((1, 3, D))
+    q = r.standard_normal((1, 1, H, D))
+    sink = np.array([0.3, -0.4])
+    t = 2                                      # t < m: no entry visible
+    out, _ = O.hca_dense_attn(q, np.zeros((1, 0, D)), kv, t, 0, 4, 1, sink, R, rows=[(0, 0)])
+    lg = q[0, 0] @ kv[0, t] / math.sqrt(D)
+    expect = kv[0, t][None, :] / (1.0 + np.exp(sink - lg))[:, None]
+    np.testing.assert_allclose(out[0], expect, atol=1e-12)
+
+
+def test_csa_translation_invariance():
+    """Shift every position by delta (a multiple of m): entries move by delta/m,
+    the window rows and the query by delta; the output does not change."""
+    r = _rng(14)
+    H, D, R, m, W = 2, 16, 8, 4, 6
+    Nc, Tkv, k = 30, 130, 8
+    ckv = r.standard_normal((1, Nc, D))
+    kv = r.standard_normal((1, Tkv, D))
+    q = r.standard_normal((1, 3, H, D))
+    sink = r.standard_normal(H)
+    idx = np.stack([np.sort(r.choice(n, k, replace=False)) for n in (25, 26, 27)])[None]
+    out0, lse0 = O.csa_sparse_attn(q, ckv, idx, kv, 101, 0, m, W, sink, R)
+    dshift = 12
+    ckv2 = np.concatenate([r.standard_normal((1, dshift // m, D)), ckv], axis=1)
+    out1, lse1 = O.csa_sparse_attn(q, ckv2, idx + dshift // m, kv, 101 + dshift, dshift, m, W, sink, R)
+    np.testing.assert_allclose(out1, out0, atol=1e-9)
+    np.testing.assert_allclose(lse1, lse0, atol=1e-9)
+
+
+def test_csa_with_all_visible_selected_equals_dense():
+    r = _rng(15)
+    H, D, R, m, W = 2, 16, 8, 4, 5
+    T = 64
+    ckv = r.standard_normal((1, T // m, D))
+    kv = r.standard_normal((1, T, D))
+    q = r.standard_normal((1, T, H, D))
+    sink = r.standard_normal(H)
+    k = T // m
+    idx = np.full((1, T, k), -1)
+    for t in range(T):
+        nv = O.n_visible(t, m, T // m)
+        idx[0, t, :nv] = np.arange(nv)
+    a, la = O.csa_sparse_attn(q, ckv, idx, kv, 0, 0, m, W, sink, R)
+    b, lb = O.hca_dense_attn(q, ckv, kv, 0, 0, m, W, sink, R)
+    np.testing.assert_allclose(a, b, atol=1e-13)
+    np.testing.assert_allclose(la, lb, atol=1e-13)
+
+
+def test_decode_ring_equals_full_kv():
+    r = _rng(16)
+    H, D, R, W, T = 2, 16, 8, 8, 50
+    kv = r.standard_normal((1, T, D))
+    ckv = r.standard_normal((1, T // 4, D))
+    q = r.standard_normal((1, 1, H, D))
+    t = T - 1
+    full, _ = O.hca_dense_attn(q, ckv, kv, t, 0, 4, W, None, R)
+    ring, _ = O.hca_dense_attn(q, ckv, kv[:, t - W + 1:], t, t - W + 1, 4, W, None, R)
+    np.testing.assert_array_equal(full, ring)
+
+
+def test_hca_pipeline_strictly_causal():
+    r = _rng(17)
+    H, D, R, m, W, T = 2, 8, 4, 8, 4, 64
+    kv = r.standard_normal((1, T, D))
+    gate = r.standard_normal((1, T, D))
+    q = r.standard_normal((1, T, H, D))
+    def run(kv_, gate_):
+        ckv = O.hca_compress(kv_[0], gate_[0], m)[None]
+        return O.hca_dense_attn(q, ckv, kv_, 0, 0, m, W, None, R)[0]
+    base = run(kv, gate)
+    kv2, g2 = kv.copy(), gate.copy()
+    kv2[0, 30:] += 1.0
+    g2[0, 30:] += 2.0
+    out2 = run(kv2, g2)
+    np.testing.assert_array_equal(base[:30], out2[:30])
+    assert not np.allclose(base[30], out2[30])
