@@ -1,0 +1,201 @@
+/*
+ * lcsa.h - C ABI of liblcsa, the B200 (sm_100a) hot path of the DeepSeek-V4
+ * hybrid compressed attention: CSA (compressed sparse attention) and HCA
+ * (heavily compressed attention).
+ *
+ * Sources, cited below by tag (web pages about DeepSeek-V4):
+ *   [p1] "DeepSeek V4的4个技巧", section 1 "技巧1：混合注意力"
+ *   [p2] "深度解析 DeepSeek-V4：百万级长文本的低成本突破", sections
+ *        "CSA：Compressed Sparse Attention" (Step 1 Compress, Step 2 Select,
+ *        ASCII figure), "HCA：Heavily Compressed Attention",
+ *        "Sliding Window Branch", "Attention Sink"
+ *   [p3] untitled classical-Chinese paraphrase page: the "Partial RoPE",
+ *        "Attention sink", "第一步/第二步/第三步" step sentences, and the
+ *        strict-causality, HCA-no-overlap and sliding-window sentences
+ *   [p4] "DeepSeek V4 技术架构深度解析", section "二、CSA + HCA"
+ *
+ * Conventions shared by every call
+ *   - Every tensor argument is a DEVICE pointer, allocated and owned by the
+ *     caller; the library never allocates device memory.  Tensors are dense
+ *     row-major with the last dimension contiguous.  Every tensor pointer and
+ *     every row must be 16-byte aligned (rows of D elements: D*elem % 16 == 0).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and stream-ordered.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     returned synchronously (LCSA_ERR_INVALID_ARG / LCSA_ERR_UNSUPPORTED /
+ *     LCSA_ERR_WORKSPACE); a failed launch returns LCSA_ERR_CUDA.  Problems a
+ *     kernel detects while running (a bounded wait that gave up, an index out
+ *     of range) are written to a per-device status word that
+ *     lcsa_get_device_status() reads; the kernel skips the bad access.
+ *   - Positions are absolute token positions (int64).  Compressed entry j of a
+ *     stride-m cache sits at position j*m and is visible to the query at
+ *     position t iff j < floor(t/m) ([p3] strict causality: a query never sees
+ *     the tokens of its own compressed block).
+ *   - Storage dtypes: LCSA_BF16 (BF16 storage, FP32 arithmetic) or LCSA_FP32.
+ *     BF16 with the layer's shapes (H=64, D=512, R=64; indexer H_I=64,
+ *     D_I=128) runs on tcgen05 tensor cores; other shapes and FP32 run on
+ *     FP32 CUDA-core kernels.  There is no CPU path: without a CUDA device every
+ *     compute call returns LCSA_ERR_CUDA.
+ */
+#ifndef LCSA_H
+#define LCSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LCSA_OK = 0,
+  LCSA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size           */
+  LCSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented combination         */
+  LCSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required    */
+  LCSA_ERR_CUDA = 4,          /* launch failure / no device                    */
+  LCSA_ERR_DEVICE = 5         /* device status word holds an error             */
+} lcsa_status;
+
+typedef enum { LCSA_FP32 = 0, LCSA_BF16 = 1 } lcsa_dtype;
+
+/* Device status codes (lcsa_get_device_status). */
+#define LCSA_DEV_OK 0
+#define LCSA_DEV_TIMEOUT 1        /* a bounded mbarrier / flag wait gave up     */
+#define LCSA_DEV_BAD_INDEX 2      /* a selected index was >= Nc (skipped)       */
+
+const char* lcsa_version(void);
+const char* lcsa_status_string(lcsa_status s);
+
+/* Synchronises `stream`, returns the current device's status word in *code
+ * (LCSA_DEV_*) and clears it.  Returns LCSA_ERR_DEVICE when *code != 0. */
+lcsa_status lcsa_get_device_status(void* stream, int* code);
+
+/* ------------------------------------------------------------------------
+ * KV compression ([p2] CSA Step 1: m consecutive tokens merged into one entry
+ * with learned softmax weights; [p2] HCA: m' = 128 tokens per entry; [p3]
+ * "第一步，KV压缩" and the sentence that HCA pools every m' tokens without
+ * CSA's overlap).
+ *
+ *   c[b,j,d] = sum_{i in S_j} softmax_{i in S_j}(gate[b,i,d]) * kv[b,i,d]
+ *   CSA: S_j = [(j-1)m, (j+1)m) clipped at 0 (window 2m, stride m)
+ *   HCA: S_j = [j m, (j+1) m)              (non-overlapping)
+ * for j < floor(T/m) (entries exist only for complete own-blocks).  With
+ * rms_weight != NULL the entry is RMS-normalised, c / sqrt(mean(c^2)+eps) * w
+ * ([p2] "Attention Sink" section: RMSNorm on the compressed KV entries).
+ *
+ *   kv   [B,T,D] dtype          gate [B,T,D] dtype (gate_per_channel=1) or
+ *                               [B,T] dtype (one logit per token, =0)
+ *   out  [B,floor(T/m),D] out_dtype
+ * Constraints: D*elem % 16 == 0, m >= 1, T >= 0.
+ * ------------------------------------------------------------------------ */
+lcsa_status lcsa_csa_compress(const void* kv, const void* gate, int gate_per_channel,
+                              int B, int T, int D, int m, lcsa_dtype dtype,
+                              const float* rms_weight, float rms_eps,
+                              void* out, lcsa_dtype out_dtype, void* stream);
+lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_channel,
+                              int B, int T, int D, int m, lcsa_dtype dtype,
+                              const float* rms_weight, float rms_eps,
+                              void* out, lcsa_dtype out_dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Top-k selection ([p2] CSA Step 2 and its ASCII figure: keep only the top-k
+ * scored entries; [p1] section 1: the top 2048 blocks).
+ *
+ * For every row r: the k column indices of the largest scores among columns
+ * [0, n_valid[r]), ties broken to the lower index, written ascending to
+ * idx_out[r, 0:k] and padded with -1 when n_valid[r] < k.  -0.0 equals +0.0.
+ * Scores must not be NaN.  The selection is exact (radix select on the
+ * order-preserving 32-bit key), so two calls on identical scores agree bit
+ * for bit with any other exact implementation.
+ *
+ *   scores  [rows, ld] fp32 (row stride ld >= n_cols)
+ *   n_valid [rows] int32 device, or NULL (= n_cols for every row)
+ *   idx_out [rows, k] int32
+ * ------------------------------------------------------------------------ */
+size_t lcsa_topk_workspace(int rows, int n_cols, int k);
+lcsa_status lcsa_topk_from_scores(const float* scores, int rows, int n_cols, int64_t ld,
+                                  const int32_t* n_valid, int k, int32_t* idx_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Lightning Indexer + top-k ([p2] CSA Step 2; [p3] "第二步，lightning indexer
+ * + top-k选择" and the sentence on scoring every compressed block against
+ * each query token; [p4] "二、CSA + HCA": the indexer QK path and its scores).
+ *
+ *   s[b,t,j] = sum_h w[b,t,h] * relu(q_I[b,t,h,:] . k_I[b,j,:]),  j < N_vis(t)
+ *   N_vis(t) = min(Nc, floor(t/m)),  t = q_pos0 + row
+ * then the top-k of every row as lcsa_topk_from_scores does, on the FP32
+ * scores.  BF16 inputs are multiplied exactly and accumulated in FP32.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* q_idx;     /* [B,Tq,H_I,D_I] dtype                                 */
+  const float* w;        /* [B,Tq,H_I] fp32 head weights                          */
+  const void* k_idx;     /* [B,Nc,D_I] dtype, one indexer key per entry            */
+  int B, Tq, Nc, H_I, D_I;
+  lcsa_dtype dtype;
+  int64_t q_pos0;        /* absolute position of query row 0 (every sequence)    */
+  int m;                 /* entry stride, for the visibility rule                */
+  int k;                 /* entries kept per query                               */
+  int32_t* idx_out;      /* [B,Tq,k] int32, ascending, -1 padded                 */
+  float* scores_out;     /* optional [B,Tq,Nc] fp32; columns >= N_vis(t) undefined */
+} lcsa_indexer_args;
+
+size_t lcsa_indexer_topk_workspace(const lcsa_indexer_args* a);
+lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace,
+                              size_t workspace_bytes, void* stream);
+int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a);
+
+/* ------------------------------------------------------------------------
+ * Core attention ([p3] "第三步，core attention"; [p3] the sentence on running
+ * multi-query attention over the selected blocks (CSA) and the HCA sentence on
+ * dense attention over all compressed KV; [p2] "Sliding Window Branch": the
+ * 128 most recent raw tokens; [p2] "Attention Sink" and [p3] "Attention
+ * sink": a learnable logit per head added to the softmax denominator;
+ * [p3] "Partial RoPE": rotary on the last 64 dims of queries and KV entries,
+ * and the output rotated at position -i because each entry is both key and
+ * value).
+ *
+ * For query row i of sequence b at position t = q_pos0 + i and head h:
+ *   keys  = { entry j rotated at position j*m : j in sel(t) }
+ *         U { raw row kv[b, s - kv_pos0] rotated at s : t-W < s <= t,
+ *             kv_pos0 <= s < kv_pos0 + Tkv }
+ *   sel(t) = idx[b,i,:] minus the -1 padding          (CSA, sparse)
+ *          = { j : j < min(Nc, floor(t/m)) }           (HCA, dense)
+ *   l_hj  = softmax_scale * rot_t(q[b,i,h]) . key_j
+ *   out   = rot_{-t}( sum_j e^{l_hj} key_j / (sum_j e^{l_hj} + e^{sink_h}) )
+ *   lse   = log(sum_j e^{l_hj} + e^{sink_h})
+ * rot_p rotates dims [D-R, D) pairwise (2i, 2i+1) by p*base^(-2i/R); one
+ * softmax covers compressed entries, window rows and the sink (shared
+ * log-sum-exp).  The rotated entry is both key and value.  The CSA call trusts
+ * idx for visibility (the indexer emits only visible entries); an index
+ * >= Nc is skipped and flagged LCSA_DEV_BAD_INDEX.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* q;         /* [B,Tq,H,D] dtype                                     */
+  const void* ckv;       /* [B,Nc,D] dtype compressed entries (shared K=V)       */
+  const int32_t* idx;    /* CSA: [B,Tq,k] int32 ascending, -1 padded; HCA: unused */
+  const void* kv;        /* [B,Tkv,D] dtype raw rows at kv_pos0 .. kv_pos0+Tkv-1  */
+  const float* sink;     /* [H] fp32 or NULL (no sink)                           */
+  int B, Tq, H, D, R, Nc, k, Tkv;
+  int64_t q_pos0, kv_pos0;
+  int m;                 /* entry stride (position j*m, visibility floor(t/m))   */
+  int W;                 /* sliding window (raw tokens), W >= 0                  */
+  float softmax_scale;   /* 0 -> 1/sqrt(D)                                       */
+  float rope_base;       /* 0 -> 10000                                           */
+  lcsa_dtype dtype;
+  void* out;             /* [B,Tq,H,D] out_dtype                                 */
+  lcsa_dtype out_dtype;
+  float* lse;            /* optional [B,Tq,H] fp32 (natural log)                 */
+} lcsa_attn_args;
+
+size_t lcsa_attn_workspace(const lcsa_attn_args* a, int sparse);
+lcsa_status lcsa_csa_sparse_attn(const lcsa_attn_args* a, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+lcsa_status lcsa_hca_dense_attn(const lcsa_attn_args* a, void* workspace,
+                                size_t workspace_bytes, void* stream);
+int lcsa_attn_uses_tensor_cores(const lcsa_attn_args* a);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LCSA_H */

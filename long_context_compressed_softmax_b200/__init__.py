@@ -1,0 +1,255 @@
+"""Python binding of liblcsa (argument marshalling only).
+
+Every call forwards raw device pointers, sizes and the current CUDA stream to
+the C ABI declared in include/lcsa.h; all computation runs in the library's
+sm_100a kernels.  PyTorch is used for device memory and streams.  There is no
+fallback: if liblcsa.so is missing, importing this package fails.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblcsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"liblcsa.so not found at {LIB_PATH}; build it with "
+        "`python -m long_context_compressed_softmax_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LCSA_FP32, LCSA_BF16 = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported combination", 3: "workspace missing or too small",
+           4: "CUDA error", 5: "device reported an error"}
+
+EXPORTED = [
+    "lcsa_version", "lcsa_status_string", "lcsa_get_device_status",
+    "lcsa_csa_compress", "lcsa_hca_compress",
+    "lcsa_topk_workspace", "lcsa_topk_from_scores",
+    "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
+    "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
+]
+
+
+class LcsaError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = int(status)
+        super().__init__(f"{what}: {_STATUS.get(self.status, self.status)} ({self.status})")
+
+
+class IndexerArgs(ctypes.Structure):
+    _fields_ = [
+        ("q_idx", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k_idx", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Tq", ctypes.c_int), ("Nc", ctypes.c_int), ("H_I", ctypes.c_int),
+        ("D_I", ctypes.c_int), ("dtype", ctypes.c_int), ("q_pos0", ctypes.c_int64), ("m", ctypes.c_int),
+        ("k", ctypes.c_int), ("idx_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
+    ]
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("ckv", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("kv", ctypes.c_void_p),
+        ("sink", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Tq", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int), ("R", ctypes.c_int),
+        ("Nc", ctypes.c_int), ("k", ctypes.c_int), ("Tkv", ctypes.c_int),
+        ("q_pos0", ctypes.c_int64), ("kv_pos0", ctypes.c_int64),
+        ("m", ctypes.c_int), ("W", ctypes.c_int), ("softmax_scale", ctypes.c_float), ("rope_base", ctypes.c_float),
+        ("dtype", ctypes.c_int), ("out", ctypes.c_void_p), ("out_dtype", ctypes.c_int), ("lse", ctypes.c_void_p),
+    ]
+
+
+_vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_sig = {
+    "lcsa_version": (ctypes.c_char_p, []),
+    "lcsa_status_string": (ctypes.c_char_p, [_i]),
+    "lcsa_get_device_status": (_i, [_vp, ctypes.POINTER(_i)]),
+    "lcsa_csa_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
+    "lcsa_hca_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
+    "lcsa_topk_workspace": (_sz, [_i, _i, _i]),
+    "lcsa_topk_from_scores": (_i, [_vp, _i, _i, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
+    "lcsa_indexer_topk_workspace": (_sz, [ctypes.POINTER(IndexerArgs)]),
+    "lcsa_indexer_topk": (_i, [ctypes.POINTER(IndexerArgs), _vp, _sz, _vp]),
+    "lcsa_indexer_uses_tensor_cores": (_i, [ctypes.POINTER(IndexerArgs)]),
+    "lcsa_attn_workspace": (_sz, [ctypes.POINTER(AttnArgs), _i]),
+    "lcsa_csa_sparse_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
+    "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
+    "lcsa_attn_uses_tensor_cores": (_i, [ctypes.POINTER(AttnArgs)]),
+}
+for _name, (_res, _args) in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+lib = _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LCSA_BF16
+    if t.dtype == torch.float32:
+        return LCSA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _tdt(code: int) -> torch.dtype:
+    return torch.bfloat16 if code == LCSA_BF16 else torch.float32
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(status, what):
+    if status != 0:
+        raise LcsaError(status, what)
+
+
+def _need_contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def version() -> str:
+    return _lib.lcsa_version().decode()
+
+
+def get_device_status() -> int:
+    code = ctypes.c_int(0)
+    st = _lib.lcsa_get_device_status(_stream(), ctypes.byref(code))
+    if st not in (0, 5):
+        raise LcsaError(st, "lcsa_get_device_status")
+    return code.value
+
+
+# ----------------------------------------------------------------- compress
+def _compress(fn, name, kv, gate, m, out_dtype, rms_weight, rms_eps, out):
+    _need_contig(kv, gate, rms_weight)
+    B, T, D = kv.shape
+    per_channel = 1 if gate.dim() == 3 else 0
+    odt = _dt(kv) if out_dtype is None else (LCSA_BF16 if out_dtype == torch.bfloat16 else LCSA_FP32)
+    if out is None:
+        out = torch.empty((B, T // m, D), dtype=_tdt(odt), device=kv.device)
+    st = fn(_p(kv), _p(gate), per_channel, B, T, D, m, _dt(kv), _p(rms_weight), float(rms_eps), _p(out), odt,
+            _stream(kv.device))
+    _check(st, name)
+    return out
+
+
+def csa_compress(kv, gate, m=4, out_dtype=None, rms_weight=None, rms_eps=1e-6, out=None):
+    """kv [B,T,D], gate [B,T,D] or [B,T] -> [B,T//m,D] (window 2m, stride m)."""
+    return _compress(_lib.lcsa_csa_compress, "csa_compress", kv, gate, m, out_dtype, rms_weight, rms_eps, out)
+
+
+def hca_compress(kv, gate, m=128, out_dtype=None, rms_weight=None, rms_eps=1e-6, out=None):
+    """kv [B,T,D], gate [B,T,D] or [B,T] -> [B,T//m,D] (non-overlapping blocks)."""
+    return _compress(_lib.lcsa_hca_compress, "hca_compress", kv, gate, m, out_dtype, rms_weight, rms_eps, out)
+
+
+# ----------------------------------------------------------------- top-k
+def topk_from_scores(scores, k, n_valid=None, out=None):
+    """scores [rows, n_cols] fp32 (row stride may exceed n_cols) -> idx [rows, k] int32."""
+    rows, n_cols = scores.shape
+    if scores.stride(1) != 1:
+        raise ValueError("scores rows must be contiguous")
+    if out is None:
+        out = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    st = _lib.lcsa_topk_from_scores(_p(scores), rows, n_cols, scores.stride(0), _p(n_valid), k, _p(out), None, 0,
+                                    _stream(scores.device))
+    _check(st, "topk_from_scores")
+    return out
+
+
+# ----------------------------------------------------------------- indexer
+def _indexer_args(q_idx, w, k_idx, q_pos0, m, k, idx_out, scores_out):
+    B, Tq, H_I, D_I = q_idx.shape
+    return IndexerArgs(_p(q_idx), _p(w), _p(k_idx), B, Tq, k_idx.shape[1], H_I, D_I, _dt(q_idx), int(q_pos0), m, k,
+                       _p(idx_out), _p(scores_out))
+
+
+def indexer_workspace_bytes(q_idx, k_idx, k):
+    B, Tq, H_I, D_I = q_idx.shape
+    a = IndexerArgs(None, None, None, B, Tq, k_idx.shape[1], H_I, D_I, _dt(q_idx), 0, 1, k, None, None)
+    return int(_lib.lcsa_indexer_topk_workspace(ctypes.byref(a)))
+
+
+def indexer_uses_tensor_cores(q_idx, k_idx, k):
+    B, Tq, H_I, D_I = q_idx.shape
+    a = IndexerArgs(None, None, None, B, Tq, k_idx.shape[1], H_I, D_I, _dt(q_idx), 0, 1, k, None, None)
+    return bool(_lib.lcsa_indexer_uses_tensor_cores(ctypes.byref(a)))
+
+
+def indexer_topk(q_idx, w, k_idx, q_pos0, m, k, return_scores=False, workspace=None, idx_out=None):
+    """q_idx [B,Tq,H_I,D_I], w [B,Tq,H_I] fp32, k_idx [B,Nc,D_I] -> idx [B,Tq,k] int32
+    (and scores [B,Tq,Nc] fp32 when return_scores)."""
+    _need_contig(q_idx, w, k_idx)
+    B, Tq = q_idx.shape[:2]
+    Nc = k_idx.shape[1]
+    dev = q_idx.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Tq, k), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, Tq, Nc), dtype=torch.float32, device=dev) if return_scores else None
+    a = _indexer_args(q_idx, w, k_idx, q_pos0, m, k, idx_out, scores)
+    need = int(_lib.lcsa_indexer_topk_workspace(ctypes.byref(a)))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = _lib.lcsa_indexer_topk(ctypes.byref(a), _p(workspace), workspace.numel(), _stream(dev))
+    _check(st, "indexer_topk")
+    return (idx_out, scores) if return_scores else idx_out
+
+
+# ----------------------------------------------------------------- attention
+def _attn_args(q, ckv, idx, kv, sink, q_pos0, kv_pos0, m, W, R, softmax_scale, rope_base, out, lse):
+    B, Tq, H, D = q.shape
+    k = idx.shape[2] if idx is not None else 0
+    return AttnArgs(_p(q), _p(ckv), _p(idx), _p(kv), _p(sink), B, Tq, H, D, R, ckv.shape[1], k, kv.shape[1],
+                    int(q_pos0), int(kv_pos0), m, W, float(softmax_scale), float(rope_base), _dt(q), _p(out),
+                    _dt(out), _p(lse))
+
+
+def attn_workspace_bytes(q, ckv, idx, kv, m, W, R=64, sparse=True):
+    a = _attn_args(q, ckv, idx, kv, None, 0, 0, m, W, R, 0.0, 0.0, q, None)
+    return int(_lib.lcsa_attn_workspace(ctypes.byref(a), 1 if sparse else 0))
+
+
+def attn_uses_tensor_cores(q, ckv, kv, R=64):
+    a = _attn_args(q, ckv, None, kv, None, 0, 0, 1, 0, R, 0.0, 0.0, q, None)
+    return bool(_lib.lcsa_attn_uses_tensor_cores(ctypes.byref(a)))
+
+
+def _attn(fn, name, sparse, q, ckv, idx, kv, sink, q_pos0, kv_pos0, m, W, R, softmax_scale, rope_base, out_dtype,
+          return_lse, workspace, out):
+    _need_contig(q, ckv, idx, kv, sink)
+    B, Tq, H, D = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Tq, H, D), dtype=out_dtype, device=dev)
+    lse = torch.empty((B, Tq, H), dtype=torch.float32, device=dev) if return_lse else None
+    a = _attn_args(q, ckv, idx, kv, sink, q_pos0, kv_pos0, m, W, R, softmax_scale, rope_base, out, lse)
+    need = int(_lib.lcsa_attn_workspace(ctypes.byref(a), sparse))
+    if need > 0 and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_n = 0 if workspace is None else workspace.numel()
+    st = fn(ctypes.byref(a), _p(workspace), ws_n, _stream(dev))
+    _check(st, name)
+    return (out, lse) if return_lse else out
+
+
+def csa_sparse_attn(q, ckv, idx, kv, sink, q_pos0, kv_pos0, m=4, W=128, R=64, softmax_scale=0.0,
+                    rope_base=10000.0, out_dtype=torch.float32, return_lse=False, workspace=None, out=None):
+    """CSA core attention over the selected entries idx [B,Tq,k] plus the window and sink."""
+    return _attn(_lib.lcsa_csa_sparse_attn, "csa_sparse_attn", 1, q, ckv, idx, kv, sink, q_pos0, kv_pos0, m, W, R,
+                 softmax_scale, rope_base, out_dtype, return_lse, workspace, out)
+
+
+def hca_dense_attn(q, ckv, kv, sink, q_pos0, kv_pos0, m=128, W=128, R=64, softmax_scale=0.0, rope_base=10000.0,
+                   out_dtype=torch.float32, return_lse=False, workspace=None, out=None):
+    """HCA core attention over every visible entry plus the window and sink."""
+    return _attn(_lib.lcsa_hca_dense_attn, "hca_dense_attn", 0, q, ckv, None, kv, sink, q_pos0, kv_pos0, m, W, R,
+                 softmax_scale, rope_base, out_dtype, return_lse, workspace, out)

@@ -1,0 +1,276 @@
+// liblcsa: C ABI entry points (declared in include/lcsa.h), argument
+// validation and kernel dispatch.  This is the library's only translation
+// unit; the kernels live in the included headers.
+#include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "lcsa.h"
+#include "common.cuh"
+#include "compress.cuh"
+#include "topk.cuh"
+#include "generic.cuh"
+#include "rope.cuh"
+#include "indexer_tc.cuh"
+#include "attn_tc.cuh"
+
+using namespace lcsa;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t esize(lcsa_dtype d) { return d == LCSA_BF16 ? 2 : 4; }
+inline bool valid_dtype(lcsa_dtype d) { return d == LCSA_BF16 || d == LCSA_FP32; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline lcsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LCSA_OK : LCSA_ERR_CUDA; }
+
+// A device must exist for any compute call (there is no CPU path).
+inline bool have_device() {
+  int n = 0;
+  return cudaGetDeviceCount(&n) == cudaSuccess && n > 0;
+}
+
+lcsa_status compress_common(const void* kv, const void* gate, int per_channel, int B, int T, int D, int m,
+                            int window, lcsa_dtype dt, const float* rms_w, float rms_eps, void* out,
+                            lcsa_dtype odt, void* stream) {
+  if (!valid_dtype(dt) || !valid_dtype(odt)) return LCSA_ERR_INVALID_ARG;
+  if (B < 0 || T < 0 || D <= 0 || m <= 0) return LCSA_ERR_INVALID_ARG;
+  const int vec = dt == LCSA_BF16 ? 8 : 4;
+  if (D % vec != 0 || D / vec > 1024) return LCSA_ERR_INVALID_ARG;
+  if (odt == LCSA_BF16 && D % 8 != 0 && dt == LCSA_BF16) return LCSA_ERR_INVALID_ARG;
+  const int Nc = T / m;
+  if ((long long)B * Nc == 0) return LCSA_OK;
+  if (!kv || !gate || !out) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(kv) || !aligned16(out) || (per_channel && !aligned16(gate))) return LCSA_ERR_INVALID_ARG;
+  if (rms_w && (reinterpret_cast<uintptr_t>(rms_w) & 3u)) return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  return from_cuda(launch_compress(kv, gate, per_channel, B, T, D, m, window, dt, rms_w, rms_eps, out, odt,
+                                   (cudaStream_t)stream));
+}
+
+lcsa_status check_indexer(const lcsa_indexer_args* a) {
+  if (!a) return LCSA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->dtype)) return LCSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->Tq < 0 || a->Nc < 0 || a->H_I <= 0 || a->D_I <= 0 || a->m <= 0 || a->k <= 0)
+    return LCSA_ERR_INVALID_ARG;
+  if (a->q_pos0 < 0) return LCSA_ERR_INVALID_ARG;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if (!a->q_idx || !a->w || !a->idx_out || (a->Nc > 0 && !a->k_idx)) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(a->q_idx) || !aligned16(a->w) || !aligned16(a->idx_out) ||
+      (a->k_idx && !aligned16(a->k_idx)) || (a->scores_out && !aligned16(a->scores_out)))
+    return LCSA_ERR_INVALID_ARG;
+  if ((a->D_I * esize(a->dtype)) % 16 != 0) return LCSA_ERR_INVALID_ARG;
+  if (!indexer_tc_supported(a) && (size_t)(a->H_I * (a->D_I + 1) + 64 * (a->D_I + 1) + a->H_I) * 4 > 200 * 1024)
+    return LCSA_ERR_UNSUPPORTED;
+  return LCSA_OK;
+}
+
+lcsa_status check_attn(const lcsa_attn_args* a, int sparse) {
+  if (!a) return LCSA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->dtype) || !valid_dtype(a->out_dtype)) return LCSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->Tq < 0 || a->H <= 0 || a->D <= 0 || a->R < 0 || a->R > a->D || (a->R & 1) ||
+      a->Nc < 0 || a->Tkv < 0 || a->m <= 0 || a->W < 0)
+    return LCSA_ERR_INVALID_ARG;
+  if (sparse && a->k <= 0) return LCSA_ERR_INVALID_ARG;
+  if (a->q_pos0 < 0) return LCSA_ERR_INVALID_ARG;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if ((a->D * esize(a->dtype)) % 16 != 0) return LCSA_ERR_INVALID_ARG;
+  if (!a->q || !a->out) return LCSA_ERR_INVALID_ARG;
+  if (a->Nc > 0 && !a->ckv) return LCSA_ERR_INVALID_ARG;
+  if (a->Tkv > 0 && !a->kv) return LCSA_ERR_INVALID_ARG;
+  if (sparse && !a->idx) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->out) || (a->ckv && !aligned16(a->ckv)) ||
+      (a->kv && !aligned16(a->kv)) || (sparse && !aligned16(a->idx)) || (a->lse && !aligned16(a->lse)) ||
+      (a->sink && (reinterpret_cast<uintptr_t>(a->sink) & 3u)))
+    return LCSA_ERR_INVALID_ARG;
+  if (!attn_tc_supported(a) && (size_t)(2 + kGenKT) * a->D * 4 > 200 * 1024) return LCSA_ERR_UNSUPPORTED;
+  return LCSA_OK;
+}
+
+template <typename T, typename To>
+cudaError_t launch_attn_generic_t(const lcsa_attn_args* a, int sparse, cudaStream_t st) {
+  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / sqrtf((float)a->D);
+  const double log_base = log(a->rope_base > 0.f ? (double)a->rope_base : 10000.0);
+  const size_t smem = (size_t)(2 + kGenKT) * a->D * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(attn_generic<T, To>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long blocks = (long long)a->B * a->Tq * a->H;
+  attn_generic<T, To><<<(unsigned)blocks, 128, smem, st>>>(
+      (const T*)a->q, (const T*)a->ckv, a->idx, (const T*)a->kv, a->sink, (To*)a->out, a->lse, a->Tq, a->H,
+      a->D, a->R, a->Nc, a->k, a->Tkv, a->q_pos0, a->kv_pos0, a->m, a->W, scale, log_base, sparse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_generic(const lcsa_attn_args* a, int sparse, cudaStream_t st) {
+  if (a->dtype == LCSA_BF16)
+    return a->out_dtype == LCSA_BF16 ? launch_attn_generic_t<__nv_bfloat16, __nv_bfloat16>(a, sparse, st)
+                                     : launch_attn_generic_t<__nv_bfloat16, float>(a, sparse, st);
+  return a->out_dtype == LCSA_BF16 ? launch_attn_generic_t<float, __nv_bfloat16>(a, sparse, st)
+                                   : launch_attn_generic_t<float, float>(a, sparse, st);
+}
+
+template <typename T>
+cudaError_t launch_indexer_generic_t(const lcsa_indexer_args* a, float* scores, int row0, int rows,
+                                     cudaStream_t st) {
+  const size_t smem = (size_t)(a->H_I * (a->D_I + 1) + 64 * (a->D_I + 1) + a->H_I) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(indexer_scores_generic<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a->Nc + 63) / 64, rows);
+  indexer_scores_generic<T><<<grid, 256, smem, st>>>((const T*)a->q_idx, a->w, (const T*)a->k_idx, scores, a->Tq,
+                                                     a->Nc, a->H_I, a->D_I, a->q_pos0, a->m, row0);
+  return cudaGetLastError();
+}
+
+// n_valid per row of a chunk: min(Nc, floor(t/m)) -- computed on the device.
+__global__ void nvalid_kernel(int32_t* nv, int rows, int row0, int Tq, long long q_pos0, int m, int Nc) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  const int i = (row0 + r) % Tq;
+  long long v = (q_pos0 + i) / m;
+  nv[r] = (int32_t)(v < Nc ? v : Nc);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lcsa_version(void) { return "lcsa 0.1 (sm_100a)"; }
+
+const char* lcsa_status_string(lcsa_status s) {
+  switch (s) {
+    case LCSA_OK: return "ok";
+    case LCSA_ERR_INVALID_ARG: return "invalid argument";
+    case LCSA_ERR_UNSUPPORTED: return "unsupported combination";
+    case LCSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LCSA_ERR_CUDA: return "CUDA error";
+    case LCSA_ERR_DEVICE: return "device reported an error";
+  }
+  return "unknown status";
+}
+
+lcsa_status lcsa_get_device_status(void* stream, int* code) {
+  if (!code) return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  int v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LCSA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return LCSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return LCSA_ERR_CUDA;
+  *code = v;
+  return v == 0 ? LCSA_OK : LCSA_ERR_DEVICE;
+}
+
+lcsa_status lcsa_csa_compress(const void* kv, const void* gate, int gate_per_channel, int B, int T, int D, int m,
+                              lcsa_dtype dtype, const float* rms_weight, float rms_eps, void* out,
+                              lcsa_dtype out_dtype, void* stream) {
+  return compress_common(kv, gate, gate_per_channel, B, T, D, m, 2 * m, dtype, rms_weight, rms_eps, out,
+                         out_dtype, stream);
+}
+
+lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_channel, int B, int T, int D, int m,
+                              lcsa_dtype dtype, const float* rms_weight, float rms_eps, void* out,
+                              lcsa_dtype out_dtype, void* stream) {
+  return compress_common(kv, gate, gate_per_channel, B, T, D, m, m, dtype, rms_weight, rms_eps, out, out_dtype,
+                         stream);
+}
+
+size_t lcsa_topk_workspace(int rows, int n_cols, int k) {
+  (void)rows; (void)n_cols; (void)k;
+  return 0;
+}
+
+lcsa_status lcsa_topk_from_scores(const float* scores, int rows, int n_cols, int64_t ld, const int32_t* n_valid,
+                                  int k, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (rows < 0 || n_cols < 0 || k <= 0 || ld < n_cols) return LCSA_ERR_INVALID_ARG;
+  if (rows == 0) return LCSA_OK;
+  if (!idx_out || (n_cols > 0 && !scores)) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(idx_out) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)) ||
+      (n_valid && (reinterpret_cast<uintptr_t>(n_valid) & 3u)))
+    return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  return from_cuda(launch_topk(scores, rows, n_cols, (long long)ld, n_valid, k, idx_out, (cudaStream_t)stream));
+}
+
+int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a) { return a && indexer_tc_supported(a) ? 1 : 0; }
+
+size_t lcsa_indexer_topk_workspace(const lcsa_indexer_args* a) {
+  if (!a || a->B <= 0 || a->Tq <= 0) return 0;
+  const long long rows = (long long)a->B * a->Tq;
+  const long long chunk = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
+  // score chunk + per-row visible counts
+  return align256((size_t)chunk * (size_t)(a->Nc > 0 ? a->Nc : 1) * 4) + align256((size_t)chunk * 4);
+}
+
+lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_t workspace_bytes, void* stream) {
+  lcsa_status s = check_indexer(a);
+  if (s != LCSA_OK) return s;
+  const long long rows = (long long)a->B * a->Tq;
+  if (rows == 0) return LCSA_OK;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int Nc = a->Nc > 0 ? a->Nc : 1;
+  // Chunk size: as many rows as the workspace holds (score rows + counts).
+  long long chunk = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
+  const size_t per_row = (size_t)Nc * 4;
+  while (chunk > 1 && align256((size_t)chunk * per_row) + align256((size_t)chunk * 4) > workspace_bytes) chunk >>= 1;
+  if (!workspace || align256((size_t)chunk * per_row) + align256((size_t)chunk * 4) > workspace_bytes)
+    return LCSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
+  float* sc_ws = (float*)workspace;
+  int32_t* nv = (int32_t*)((char*)workspace + align256((size_t)chunk * per_row));
+  const bool tc = indexer_tc_supported(a);
+  for (long long r0 = 0; r0 < rows; r0 += chunk) {
+    const int nr = (int)(rows - r0 < chunk ? rows - r0 : chunk);
+    // scores go straight to scores_out when the caller wants them
+    float* sc = a->scores_out ? a->scores_out + r0 * (long long)a->Nc : sc_ws;
+    cudaError_t e;
+    if (a->Nc > 0) {
+      if (tc) e = launch_indexer_tc(a, sc, (int)r0, nr, st);
+      else if (a->dtype == LCSA_BF16) e = launch_indexer_generic_t<__nv_bfloat16>(a, sc, (int)r0, nr, st);
+      else e = launch_indexer_generic_t<float>(a, sc, (int)r0, nr, st);
+      if (e != cudaSuccess) return LCSA_ERR_CUDA;
+    }
+    nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, (int)r0, a->Tq, a->q_pos0, a->m, a->Nc);
+    e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + r0 * a->k, st);
+    if (e != cudaSuccess) return LCSA_ERR_CUDA;
+  }
+  return LCSA_OK;
+}
+
+int lcsa_attn_uses_tensor_cores(const lcsa_attn_args* a) { return a && attn_tc_supported(a) ? 1 : 0; }
+
+size_t lcsa_attn_workspace(const lcsa_attn_args* a, int sparse) {
+  if (!a || a->B <= 0 || a->Tq <= 0 || !attn_tc_supported(a)) return 0;
+  return attn_tc_workspace(a, sparse);
+}
+
+static lcsa_status attn_common(const lcsa_attn_args* a, int sparse, void* ws, size_t ws_bytes, void* stream) {
+  lcsa_status s = check_attn(a, sparse);
+  if (s != LCSA_OK) return s;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (attn_tc_supported(a)) {
+    const size_t need = attn_tc_workspace(a, sparse);
+    if (need > 0 && (!ws || ws_bytes < need)) return LCSA_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return LCSA_ERR_INVALID_ARG;
+    return from_cuda(launch_attn_tc(a, sparse, ws, st));
+  }
+  return from_cuda(launch_attn_generic(a, sparse, st));
+}
+
+lcsa_status lcsa_csa_sparse_attn(const lcsa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return attn_common(a, 1, ws, ws_bytes, stream);
+}
+
+lcsa_status lcsa_hca_dense_attn(const lcsa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return attn_common(a, 0, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/lcsa.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lcsa():
+    from long_context_compressed_softmax_b200 import build
+    build.build()
+    import long_context_compressed_softmax_b200 as m
+    return m
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lcsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lcsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ["lcsa_csa_compress", "lcsa_hca_compress", "lcsa_indexer_topk", "lcsa_topk_from_scores",
+              "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_get_device_status"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lcsa):
+    for n in _declared():
+        assert hasattr(lcsa.lib, n), n
+    assert sorted(lcsa.EXPORTED) == sorted(_declared())
+
+
+def test_version_and_status_strings(lcsa):
+    assert "sm_100a" in lcsa.version()
+    for s in range(6):
+        assert lcsa.lib.lcsa_status_string(s)
+
+
+def test_struct_layouts_match_header(lcsa, tmp_path):
+    """The ctypes mirrors have the C structs' size and field offsets (gcc)."""
+    import subprocess
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "lcsa.h"', 'int main(void){']
+    for cname, py in (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs)):
+        lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0;}")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines())
+    for cname, py in (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs)):
+        assert int(got[cname]) == ctypes.sizeof(py)
+        for f, _ in py._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
+
+
+def test_invalid_arguments_rejected_without_launch(lcsa):
+    L = lcsa.lib
+    # null pointers with non-empty sizes
+    assert L.lcsa_csa_compress(None, None, 1, 1, 64, 512, 4, lcsa.LCSA_BF16, None, 0.0, None, lcsa.LCSA_BF16,
+                               None) == 1
+    # misaligned pointer (odd address) is refused before touching it
+    assert L.lcsa_hca_compress(ctypes.c_void_p(0x1001), ctypes.c_void_p(0x2000), 1, 1, 256, 512, 128,
+                               lcsa.LCSA_BF16, None, 0.0, ctypes.c_void_p(0x3000), lcsa.LCSA_BF16, None) == 1
+    # D not a multiple of the 16-byte vector
+    assert L.lcsa_csa_compress(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, 1, 64, 12, 4,
+                               lcsa.LCSA_BF16, None, 0.0, ctypes.c_void_p(0x3000), lcsa.LCSA_BF16, None) == 1
+    # bad k
+    assert L.lcsa_topk_from_scores(ctypes.c_void_p(0x1000), 4, 16, 16, None, 0, ctypes.c_void_p(0x2000), None, 0,
+                                   None) == 1
+    # ld < n_cols
+    assert L.lcsa_topk_from_scores(ctypes.c_void_p(0x1000), 4, 16, 8, None, 4, ctypes.c_void_p(0x2000), None, 0,
+                                   None) == 1
+    a = lcsa.AttnArgs()
+    a.B, a.Tq, a.H, a.D, a.R, a.Nc, a.k, a.Tkv, a.m, a.W = 1, 1, 64, 512, 63, 8, 8, 8, 4, 8
+    a.dtype = a.out_dtype = lcsa.LCSA_BF16
+    assert L.lcsa_csa_sparse_attn(ctypes.byref(a), None, 0, None) == 1      # odd R
+    a.R = 64
+    assert L.lcsa_csa_sparse_attn(ctypes.byref(a), None, 0, None) == 1      # null q/out
+    ia = lcsa.IndexerArgs()
+    ia.B, ia.Tq, ia.Nc, ia.H_I, ia.D_I, ia.m, ia.k = 1, 4, 8, 64, 128, 0, 8
+    assert L.lcsa_indexer_topk(ctypes.byref(ia), None, 0, None) == 1         # m = 0
+
+
+def test_empty_problems_are_noops(lcsa):
+    L = lcsa.lib
+    # T < m: no entries, nothing to do, no device needed
+    assert L.lcsa_csa_compress(None, None, 1, 1, 3, 512, 4, lcsa.LCSA_BF16, None, 0.0, None, lcsa.LCSA_BF16,
+                               None) == 0
+    assert L.lcsa_topk_from_scores(None, 0, 16, 16, None, 4, None, None, 0, None) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device behaviour")
+def test_no_cpu_fallback(lcsa):
+    """Without a CUDA device a valid compute call fails loudly (no CPU path)."""
+    L = lcsa.lib
+    st = L.lcsa_csa_compress(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, 1, 64, 512, 4,
+                             lcsa.LCSA_BF16, None, 0.0, ctypes.c_void_p(0x3000), lcsa.LCSA_BF16, None)
+    assert st == 4
+
+
+def test_workspace_queries(lcsa):
+    q = torch.empty((1, 4096, 64, 128), dtype=torch.bfloat16)
+    k = torch.empty((1, 1024, 128), dtype=torch.bfloat16)
+    assert lcsa.indexer_workspace_bytes(q, k, 2048) >= 4096 * 1024 * 4

@@ -1,0 +1,214 @@
+"""Parity of every library call with the CPU oracle on the same seeded inputs
+(sizes that span several tiles plus ragged tails, and the edge cases)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import lcsa_oracle as O
+from workloads import gen
+
+pytestmark = pytest.mark.gpu
+
+ATT_MAX, ATT_MEAN = 1e-2, 1e-3        # attention tolerance (BF16 in, FP32 accumulate, unit scale)
+
+
+@pytest.fixture(scope="module")
+def lcsa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_compressed_softmax_b200 import build
+    build.build()
+    import long_context_compressed_softmax_b200 as m
+    return m
+
+
+DEV = "cuda"
+
+
+def np64(t):
+    return t.detach().double().cpu().numpy()
+
+
+def assert_attn_close(got, ref, max_abs=ATT_MAX, mean_abs=ATT_MEAN):
+    err = np.abs(np.asarray(got, dtype=np.float64) - ref)
+    assert err.max() <= max_abs, f"max abs err {err.max():.3e}"
+    assert err.mean() <= mean_abs, f"mean abs err {err.mean():.3e}"
+
+
+# ------------------------------------------------------------------ compress
+@pytest.mark.parametrize("dtype,D", [("fp32", 64), ("bf16", 512), ("bf16", 64)])
+@pytest.mark.parametrize("kind,m", [("csa", 4), ("hca", 128), ("csa", 3), ("hca", 16)])
+@pytest.mark.parametrize("per_channel", [True, False])
+def test_compress_parity(lcsa, dtype, D, kind, m, per_channel):
+    B, T = 2, 1037                                   # ragged: T % m != 0
+    x = gen.make_compress_inputs(B, T, D, dtype, seed=21, device=DEV, gate_per_channel=per_channel)
+    fn = lcsa.csa_compress if kind == "csa" else lcsa.hca_compress
+    ofn = O.csa_compress if kind == "csa" else O.hca_compress
+    out = fn(x["kv"], x["gate"], m, out_dtype=torch.float32)
+    assert out.shape == (B, T // m, D)
+    for b in range(B):
+        ref = ofn(np64(x["kv"][b]), np64(x["gate"][b]), m)
+        np.testing.assert_allclose(np64(out[b]), ref, rtol=0, atol=2e-6)
+
+
+def test_compress_bf16_out_and_rmsnorm(lcsa):
+    B, T, D = 1, 512, 512
+    x = gen.make_compress_inputs(B, T, D, "bf16", seed=22, device=DEV)
+    w = torch.randn(D, device=DEV, generator=torch.Generator(device=DEV).manual_seed(5))
+    out = lcsa.csa_compress(x["kv"], x["gate"], 4, rms_weight=w, rms_eps=1e-6)
+    assert out.dtype == torch.bfloat16
+    ref = O.csa_compress(np64(x["kv"][0]), np64(x["gate"][0]), 4, rms_weight=np64(w), rms_eps=1e-6)
+    np.testing.assert_allclose(np64(out[0]), ref, rtol=1e-2, atol=1e-2)
+
+
+def test_compress_short_sequence(lcsa):
+    x = gen.make_compress_inputs(1, 3, 512, "bf16", seed=23, device=DEV)
+    assert lcsa.csa_compress(x["kv"], x["gate"], 4).shape == (1, 0, 512)
+
+
+# ------------------------------------------------------------------ top-k
+@pytest.mark.parametrize("n_cols,k,ties", [(64, 8, 0), (1000, 64, 4), (8191, 2048, 0), (8191, 2048, 16),
+                                          (40000, 2048, 0), (5000, 1, 3), (300, 2048, 0)])
+def test_topk_bitexact(lcsa, n_cols, k, ties):
+    rows = 37
+    s = gen.make_scores(rows, n_cols, seed=31 + n_cols, device=DEV, tie_levels=ties)
+    g = torch.Generator(device="cpu").manual_seed(7)
+    nv = torch.randint(0, n_cols + 1, (rows,), generator=g, dtype=torch.int32)
+    nv[0], nv[1] = n_cols, min(k, n_cols)
+    idx = lcsa.topk_from_scores(s, k, n_valid=nv.to(DEV))
+    ref = O.topk_from_scores(s.cpu().double().numpy(), nv.numpy(), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_adversarial_rows(lcsa):
+    k = 16
+    rows = [np.zeros(100), np.full(100, -3.5), np.r_[np.full(50, 1.0), np.full(50, -0.0)],
+            np.r_[np.full(30, -0.0), np.full(70, 0.0)], np.linspace(-1, 1, 100)[::-1].copy(),
+            np.r_[np.full(99, -np.inf), [0.0]], np.r_[[np.inf], np.zeros(99)]]
+    s = torch.tensor(np.stack(rows), dtype=torch.float32, device=DEV)
+    idx = lcsa.topk_from_scores(s, k)
+    ref = O.topk_from_scores(s.cpu().double().numpy(), [100] * len(rows), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_toy_from_pages(lcsa):
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "topk_toy.json")))
+    s = torch.tensor([g["scores"]], dtype=torch.float32, device=DEV)
+    assert lcsa.topk_from_scores(s, g["k"]).cpu().tolist() == [g["expected_idx"]]
+
+
+# ------------------------------------------------------------------ indexer
+def _score_err_ok(got, ref, nv):
+    for i in range(ref.shape[0]):
+        n = nv[i]
+        if n == 0:
+            continue
+        r, g_ = ref[i, :n], got[i, :n]
+        scale = np.maximum(np.abs(r), np.sqrt(np.mean(r * r)))
+        bad = np.abs(g_ - r) > 1e-3 * scale
+        assert not bad.any(), f"row {i}: {int(bad.sum())} scores off, worst {np.max(np.abs(g_ - r) / scale):.2e}"
+
+
+@pytest.mark.parametrize("dtype,H_I,D_I,Tq,Nc,m,k,q_pos0", [
+    ("fp32", 2, 32, 300, 256, 4, 64, 724),          # tiny-layer shapes, tail rows
+    ("bf16", 64, 128, 260, 1030, 4, 256, 3900),     # layer shapes, several tiles + ragged tail
+    ("bf16", 64, 128, 37, 700, 4, 2048, 0),         # N_vis < k everywhere
+    ("bf16", 16, 64, 50, 333, 4, 32, 1200),         # other shape on the CUDA-core kernel
+])
+def test_indexer_scores_and_recall(lcsa, dtype, H_I, D_I, Tq, Nc, m, k, q_pos0):
+    B = 2
+    x = gen.make_indexer_inputs(B, Tq, Nc, H_I, D_I, dtype, seed=41, device=DEV)
+    idx, sc = lcsa.indexer_topk(x["q_idx"], x["w"], x["k_idx"], q_pos0, m, k, return_scores=True)
+    hits = tot = 0
+    for b in range(B):
+        ref_idx, ref_s = O.indexer_topk(np64(x["q_idx"][b]), np64(x["w"][b]), np64(x["k_idx"][b]), q_pos0, m, k)
+        nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+        _score_err_ok(np64(sc[b]), ref_s, nv)
+        got = idx[b].cpu().numpy()
+        # structure: ascending valid prefix, -1 padding, all visible
+        for i in range(Tq):
+            v = got[i][got[i] >= 0]
+            assert (np.diff(v) > 0).all() and (v < max(nv[i], 1)).all()
+            assert len(v) == min(k, nv[i]) and (got[i][len(v):] == -1).all()
+            hits += len(set(v) & set(ref_idx[i][ref_idx[i] >= 0]))
+            tot += int((ref_idx[i] >= 0).sum())
+        # same scores -> identical selection
+        sel = O.topk_from_scores(np64(sc[b]), nv, k)
+        np.testing.assert_array_equal(got, sel)
+    assert hits >= 0.999 * tot, f"recall {hits / tot:.5f}"
+
+
+# ------------------------------------------------------------------ attention
+def _attn_case(B, Tq, H, D, Nc, Tkv, dtype, seed, unit=True, sink=True):
+    return gen.make_attn_inputs(B, Tq, H, D, Nc, Tkv, dtype, seed=seed, device=DEV, unit_scale=unit,
+                                with_sink=sink)
+
+
+def _sink(x):
+    return None if x["sink"] is None else np64(x["sink"])
+
+
+@pytest.mark.parametrize("dtype,H,D,R,m,W,k,Tq,Nc,q_pos0,unit", [
+    ("fp32", 4, 64, 32, 4, 64, 64, 200, 256, 824, True),       # tiny layer: rows near the end of T=1024
+    ("fp32", 4, 64, 32, 4, 64, 64, 64, 256, 0, True),          # first rows: no entries / short window
+    ("bf16", 64, 512, 64, 4, 128, 256, 40, 700, 2700, True),   # layer shapes
+    ("bf16", 64, 512, 64, 4, 128, 256, 40, 700, 2700, False),  # spec scale
+    ("bf16", 64, 512, 64, 4, 128, 2048, 9, 3000, 9000, True),  # full k
+    ("bf16", 64, 512, 64, 4, 100, 100, 20, 900, 3000, True),   # odd W and k
+])
+def test_csa_sparse_attn_parity(lcsa, dtype, H, D, R, m, W, k, Tq, Nc, q_pos0, unit):
+    B = 2
+    Tkv = q_pos0 + Tq
+    x = _attn_case(B, Tq, H, D, Nc, Tkv, dtype, seed=51, unit=unit)
+    nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+    idx = gen.make_topk_idx(B, Tq, k, nv, seed=52, device=DEV)
+    out, lse = lcsa.csa_sparse_attn(x["q"], x["ckv"], idx, x["kv"], x["sink"], q_pos0, 0, m, W, R, return_lse=True)
+    ref, ref_lse = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), q_pos0, 0, m,
+                                     W, _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+    np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
+
+
+@pytest.mark.parametrize("dtype,H,D,R,m,W,Tq,Nc,q_pos0,unit,sink", [
+    ("fp32", 4, 64, 32, 128, 64, 300, 8, 724, True, True),
+    ("bf16", 64, 512, 64, 128, 128, 130, 40, 2000, True, True),    # crosses a 128-block boundary
+    ("bf16", 64, 512, 64, 128, 128, 130, 40, 2000, False, True),
+    ("bf16", 64, 512, 64, 128, 128, 70, 40, 0, True, False),       # t < m: window only, no sink
+    ("bf16", 64, 512, 64, 16, 128, 50, 400, 5000, True, True),     # many entries (> several tiles)
+])
+def test_hca_dense_attn_parity(lcsa, dtype, H, D, R, m, W, Tq, Nc, q_pos0, unit, sink):
+    B = 2
+    Tkv = q_pos0 + Tq
+    x = _attn_case(B, Tq, H, D, Nc, Tkv, dtype, seed=61, unit=unit, sink=sink)
+    out, lse = lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q_pos0, 0, m, W, R, return_lse=True)
+    ref, ref_lse = O.hca_dense_attn(np64(x["q"]), np64(x["ckv"]), np64(x["kv"]), q_pos0, 0, m, W, _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+    np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
+
+
+def test_decode_window_ring(lcsa):
+    """Decode layout: kv holds only the last W raw rows (kv_pos0 = t-W+1)."""
+    B, H, D, R, m, W, k, Nc = 3, 64, 512, 64, 4, 128, 512, 4000
+    t = 4 * Nc
+    x = _attn_case(B, 1, H, D, Nc, W, "bf16", seed=71)
+    idx = gen.make_topk_idx(B, 1, k, [Nc], seed=72, device=DEV)
+    out = lcsa.csa_sparse_attn(x["q"], x["ckv"], idx, x["kv"], x["sink"], t, t - W + 1, m, W, R)
+    ref, _ = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), t, t - W + 1, m, W,
+                               _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+
+
+def test_attn_bf16_output(lcsa):
+    B, H, D, R, m, W, k, Tq, Nc, q0 = 1, 64, 512, 64, 4, 128, 128, 16, 600, 2400
+    x = _attn_case(B, Tq, H, D, Nc, q0 + Tq, "bf16", seed=81)
+    idx = gen.make_topk_idx(B, Tq, k, [O.n_visible(q0 + i, m, Nc) for i in range(Tq)], seed=82, device=DEV)
+    out = lcsa.csa_sparse_attn(x["q"], x["ckv"], idx, x["kv"], x["sink"], q0, 0, m, W, R, out_dtype=torch.bfloat16)
+    ref, _ = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), q0, 0, m, W,
+                               _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref, max_abs=2e-2, mean_abs=3e-3)
+
+
+def test_device_status_clean(lcsa):
+    torch.cuda.synchronize()
+    assert lcsa.get_device_status() == 0
