@@ -124,11 +124,12 @@ cudaError_t launch_indexer_generic_t(const lcsa_indexer_args* a, float* scores, 
   return cudaGetLastError();
 }
 
-// n_valid per row of a chunk: min(Nc, floor(t/m)) -- computed on the device.
-__global__ void nvalid_kernel(int32_t* nv, int rows, int row0, int Tq, long long q_pos0, int m, int Nc) {
+// n_valid per row of a chunk rectangle (rows ordered [b][i0..i0+ni)):
+// min(Nc, floor(t/m)) with t = q_pos0 + i.
+__global__ void nvalid_kernel(int32_t* nv, int rows, int i0, int ni, long long q_pos0, int m, int Nc) {
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= rows) return;
-  const int i = (row0 + r) % Tq;
+  const int i = i0 + r % ni;
   long long v = (q_pos0 + i) / m;
   nv[r] = (int32_t)(v < Nc ? v : Nc);
 }
@@ -215,30 +216,39 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_
   if (!have_device()) return LCSA_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
   const int Nc = a->Nc > 0 ? a->Nc : 1;
-  // Chunk size: as many rows as the workspace holds (score rows + counts).
-  long long chunk = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
+  // Rows per chunk: as many score rows as the workspace holds (scores + counts).
   const size_t per_row = (size_t)Nc * 4;
-  while (chunk > 1 && align256((size_t)chunk * per_row) + align256((size_t)chunk * 4) > workspace_bytes) chunk >>= 1;
-  if (!workspace || align256((size_t)chunk * per_row) + align256((size_t)chunk * 4) > workspace_bytes)
-    return LCSA_ERR_WORKSPACE;
+  auto need = [&](long long r) { return align256((size_t)r * per_row) + align256((size_t)r * 4); };
+  long long budget = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
+  while (budget > 1 && need(budget) > workspace_bytes) budget >>= 1;
+  if (!workspace || need(budget) > workspace_bytes) return LCSA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
   float* sc_ws = (float*)workspace;
-  int32_t* nv = (int32_t*)((char*)workspace + align256((size_t)chunk * per_row));
+  int32_t* nv = (int32_t*)((char*)workspace + align256((size_t)budget * per_row));
   const bool tc = indexer_tc_supported(a);
-  for (long long r0 = 0; r0 < rows; r0 += chunk) {
-    const int nr = (int)(rows - r0 < chunk ? rows - r0 : chunk);
-    // scores go straight to scores_out when the caller wants them
-    float* sc = a->scores_out ? a->scores_out + r0 * (long long)a->Nc : sc_ws;
-    cudaError_t e;
-    if (a->Nc > 0) {
-      if (tc) e = launch_indexer_tc(a, sc, (int)r0, nr, st);
-      else if (a->dtype == LCSA_BF16) e = launch_indexer_generic_t<__nv_bfloat16>(a, sc, (int)r0, nr, st);
-      else e = launch_indexer_generic_t<float>(a, sc, (int)r0, nr, st);
+  // Chunk rectangles: whole sequences when a sequence fits, else row ranges of
+  // one sequence (a multiple of the 4-row query group).
+  int nb_step, ni_step;
+  if (a->Tq <= budget) { nb_step = (int)(budget / a->Tq); ni_step = a->Tq; }
+  else { nb_step = 1; ni_step = budget >= 4 ? (int)(budget & ~3LL) : (int)budget; }
+  for (int b0 = 0; b0 < a->B; b0 += nb_step) {
+    const int nb = a->B - b0 < nb_step ? a->B - b0 : nb_step;
+    for (int i0 = 0; i0 < a->Tq; i0 += ni_step) {
+      const int ni = a->Tq - i0 < ni_step ? a->Tq - i0 : ni_step;
+      const long long row0 = (long long)b0 * a->Tq + i0;      // rectangle rows are contiguous
+      const int nr = nb * ni;
+      float* sc = a->scores_out ? a->scores_out + row0 * (long long)a->Nc : sc_ws;
+      cudaError_t e = cudaSuccess;
+      if (a->Nc > 0) {
+        if (tc) e = launch_indexer_tc_rect(a, sc, b0, nb, i0, ni, st);
+        else if (a->dtype == LCSA_BF16) e = launch_indexer_generic_t<__nv_bfloat16>(a, sc, (int)row0, nr, st);
+        else e = launch_indexer_generic_t<float>(a, sc, (int)row0, nr, st);
+        if (e != cudaSuccess) return LCSA_ERR_CUDA;
+      }
+      nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, a->q_pos0, a->m, a->Nc);
+      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st);
       if (e != cudaSuccess) return LCSA_ERR_CUDA;
     }
-    nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, (int)r0, a->Tq, a->q_pos0, a->m, a->Nc);
-    e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + r0 * a->k, st);
-    if (e != cudaSuccess) return LCSA_ERR_CUDA;
   }
   return LCSA_OK;
 }

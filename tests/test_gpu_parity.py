@@ -156,6 +156,7 @@ def _sink(x):
     ("bf16", 64, 512, 64, 4, 128, 256, 40, 700, 2700, False),  # spec scale
     ("bf16", 64, 512, 64, 4, 128, 2048, 9, 3000, 9000, True),  # full k
     ("bf16", 64, 512, 64, 4, 100, 100, 20, 900, 3000, True),   # odd W and k
+    ("bf16", 64, 512, 64, 4, 128, 256, 160, 700, 2700, True),  # >= 296 rows: no key-range split
 ])
 def test_csa_sparse_attn_parity(lcsa, dtype, H, D, R, m, W, k, Tq, Nc, q_pos0, unit):
     B = 2
@@ -176,6 +177,7 @@ def test_csa_sparse_attn_parity(lcsa, dtype, H, D, R, m, W, k, Tq, Nc, q_pos0, u
     ("bf16", 64, 512, 64, 128, 128, 130, 40, 2000, False, True),
     ("bf16", 64, 512, 64, 128, 128, 70, 40, 0, True, False),       # t < m: window only, no sink
     ("bf16", 64, 512, 64, 16, 128, 50, 400, 5000, True, True),     # many entries (> several tiles)
+    ("bf16", 64, 512, 64, 128, 128, 160, 40, 4000, True, True),    # >= 296 rows: no key-range split
 ])
 def test_hca_dense_attn_parity(lcsa, dtype, H, D, R, m, W, Tq, Nc, q_pos0, unit, sink):
     B = 2
@@ -207,6 +209,15 @@ def test_attn_bf16_output(lcsa):
     ref, _ = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), q0, 0, m, W,
                                _sink(x), R)
     assert_attn_close(np64(out).reshape(ref.shape), ref, max_abs=2e-2, mean_abs=3e-3)
+
+
+def test_layer_shapes_use_tensor_cores(lcsa):
+    x = _attn_case(1, 4, 64, 512, 100, 100, "bf16", seed=91)
+    assert lcsa.attn_uses_tensor_cores(x["q"], x["ckv"], x["kv"], R=64)
+    y = _attn_case(1, 4, 4, 64, 100, 100, "fp32", seed=92)
+    assert not lcsa.attn_uses_tensor_cores(y["q"], y["ckv"], y["kv"], R=32)
+    ix = gen.make_indexer_inputs(1, 4, 100, 64, 128, "bf16", seed=93, device=DEV)
+    assert lcsa.indexer_uses_tensor_cores(ix["q_idx"], ix["k_idx"], 2048)
 
 
 def test_device_status_clean(lcsa):
