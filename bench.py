@@ -1,0 +1,585 @@
+"""Benchmark of the hybrid compressed-attention hot path on B200.
+
+Default workload (one step = the whole hot path): the alternating four-layer
+stack CSA -> HCA -> CSA -> HCA, prefill of B=2 sequences of T=131072 tokens,
+64 heads x 512 dims (last 64 rotary), indexer 64 x 128, m=4 / m'=128,
+top-k 2048, window 128, per-head sink, independent seeded inputs per layer.
+CSA layer = csa_compress -> indexer_topk -> csa_sparse_attn; HCA layer =
+hca_compress -> hca_dense_attn.  Metric: prefill tokens/s through the stack.
+A second object reports the CSA decode workload at 1M context (64 sequences,
+one query each, queries/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lcsa|reference]
+                    [--workload stack_4layer_128k|csa_prefill_32k|hca_prefill_128k|csa_decode_1m]
+
+N > 1 runs under torchrun, one rank per GPU; every rank runs the same
+per-GPU workload on its own seeds (weak scaling, no data-path collective) and
+the job time is the maximum over ranks.  `--impl reference` times the CPU
+oracle on a bounded sample of the same workload on the host cores.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import get_config  # noqa: E402
+from workloads import gen  # noqa: E402
+from workloads.scaling import max_over_ranks, rank_seed, weak_scaling_throughput  # noqa: E402
+
+METRIC = "CSA/HCA prefill tokens/s and 1M-ctx decode queries/s; % of roofline"
+
+# DRAM traffic per launch of the dominant kernels from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
+# kernel source it was taken on; a changed source reports null.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = bus_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.bus_id:
+                cmd += ["-i", self.bus_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, _, flags in rows for n, f in zip(names, flags) if f.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workloads
+def _nvis(T, m, Nc):
+    t = np.arange(T, dtype=np.int64)
+    return np.minimum(t // m, Nc)
+
+
+def attn_flops(T, m, Nc, W, k=None, H=64, D=512):
+    """Algorithmic MMA FLOPs of one sequence's attention: QK^T and PV over the
+    visible (HCA) or selected (CSA, capped at k) entries plus the window rows."""
+    nv = _nvis(T, m, Nc)
+    n_c = np.minimum(nv, k) if k is not None else nv
+    n_w = np.minimum(W, np.arange(T) + 1)
+    return float(((n_c + n_w).astype(np.float64)).sum() * H * D * 4)
+
+
+def indexer_flops(T, m, Nc, H_I=64, D_I=128):
+    return float(_nvis(T, m, Nc).astype(np.float64).sum() * H_I * D_I * 2)
+
+
+class Layer:
+    """Device tensors of one layer (inputs seeded per layer and rank)."""
+
+    def __init__(self, kind, cfg, seed, dev):
+        B, T, D = cfg.B, cfg.T, cfg.D
+        self.kind = kind
+        m = cfg.m if kind == "csa" else cfg.m_hca
+        self.m = m
+        self.Nc = T // m
+        g = gen._gen(seed, dev)
+        self.kv = gen._randn((B, T, D), g, dev, 1.0 / math.sqrt(D), torch.bfloat16)
+        self.gate = gen._randn((B, T, D), g, dev, 1.0, torch.bfloat16)
+        self.q = gen._randn((B, T, cfg.H, D), g, dev, 1.0 / math.sqrt(D), torch.bfloat16)
+        self.sink = gen._randn((cfg.H,), g, dev)
+        self.ckv = torch.empty((B, self.Nc, D), dtype=torch.bfloat16, device=dev)
+        if kind == "csa":
+            self.q_idx = gen._randn((B, T, cfg.H_I, cfg.D_I), g, dev, 1.0 / math.sqrt(cfg.D_I), torch.bfloat16)
+            self.w = gen._randn((B, T, cfg.H_I), g, dev, 1.0 / math.sqrt(cfg.H_I))
+            self.k_idx = gen._randn((B, self.Nc, cfg.D_I), g, dev, 1.0 / math.sqrt(cfg.D_I), torch.bfloat16)
+
+    def inputs(self):
+        names = ["kv", "gate", "q"] + (["q_idx", "w", "k_idx"] if self.kind == "csa" else [])
+        return {n: getattr(self, n) for n in names}
+
+
+class StackRunner:
+    """Runs the layers through the library with per-call CUDA events."""
+
+    def __init__(self, lcsa, cfg, layers, dev):
+        self.lcsa, self.cfg, self.layers = lcsa, cfg, layers
+        B, T = cfg.B, cfg.T
+        self.out = torch.empty((B, T, cfg.H, cfg.D), dtype=torch.bfloat16, device=dev)
+        self.idx = torch.empty((B, T, cfg.k), dtype=torch.int32, device=dev) if any(
+            L.kind == "csa" for L in layers) else None
+        ws = 256
+        for L in layers:
+            if L.kind == "csa":
+                ws = max(ws, lcsa.indexer_workspace_bytes(L.q_idx, L.k_idx, cfg.k))
+                ws = max(ws, lcsa.attn_workspace_bytes(L.q, L.ckv, self.idx, L.kv, L.m, cfg.W, cfg.R, True))
+            else:
+                ws = max(ws, lcsa.attn_workspace_bytes(L.q, L.ckv, None, L.kv, L.m, cfg.W, cfg.R, False))
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.events = []      # (layer index, call name, start, end)
+        self.record = False
+
+    def _ev(self):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    def _call(self, li, name, fn):
+        if self.record:
+            a = self._ev()
+            fn()
+            self.events.append((li, name, a, self._ev()))
+        else:
+            fn()
+
+    def layer(self, li):
+        L, c, lc = self.layers[li], self.cfg, self.lcsa
+        if L.kind == "csa":
+            self._call(li, "csa_compress", lambda: lc.csa_compress(L.kv, L.gate, L.m, out=L.ckv))
+            self._call(li, "indexer_topk", lambda: lc.indexer_topk(L.q_idx, L.w, L.k_idx, 0, L.m, c.k,
+                                                                   workspace=self.ws, idx_out=self.idx))
+            self._call(li, "csa_sparse_attn", lambda: lc.csa_sparse_attn(
+                L.q, L.ckv, self.idx, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
+        else:
+            self._call(li, "hca_compress", lambda: lc.hca_compress(L.kv, L.gate, L.m, out=L.ckv))
+            self._call(li, "hca_dense_attn", lambda: lc.hca_dense_attn(
+                L.q, L.ckv, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
+
+    def step(self):
+        for li in range(len(self.layers)):
+            self.layer(li)
+
+
+def _gpu_selector(dev):
+    """nvidia-smi -i selector (UUID) of this rank's GPU, or None."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def _barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def timed(fn, steps, warmup, bus_id, sample_clocks=True):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    _barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(bus_id) if sample_clocks else None
+    if clk:
+        clk.start()
+        time.sleep(0.4)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    _barrier()
+    torch.cuda.synchronize()
+    clocks = clk.stop() if clk else None
+    return a.elapsed_time(b) / steps, clocks
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample(cfg, n_rows, seed):
+    """Run the oracle on a bounded sample of the workload: sequence 0 of every
+    layer, the full compression plus `n_rows` stratified query rows through
+    indexer, top-k and attention.  Returns (seconds, extrapolated seconds of
+    the full step, description)."""
+    from oracle import lcsa_oracle as O
+    B, T, D, H = cfg.B, cfg.T, cfg.D, cfg.H
+    layers = cfg.layers or ("csa",)
+    rows = np.unique(np.linspace(0, T - 1, n_rows).astype(np.int64))
+    g = torch.Generator().manual_seed(seed)
+    t_sample = 0.0
+    t_full = 0.0
+    for li, kind in enumerate(layers):
+        m = cfg.m if kind == "csa" else cfg.m_hca
+        Nc = T // m
+        kv = (torch.randn(T, D, generator=g) / math.sqrt(D)).to(torch.bfloat16).double().numpy()
+        gate = torch.randn(T, D, generator=g).to(torch.bfloat16).double().numpy()
+        q = (torch.randn(len(rows), H, D, generator=g) / math.sqrt(D)).to(torch.bfloat16).double().numpy()
+        sink = torch.randn(H, generator=g).double().numpy()
+        t0 = time.perf_counter()
+        ckv = (O.csa_compress(kv, gate, m) if kind == "csa" else O.hca_compress(kv, gate, m))
+        t_comp = time.perf_counter() - t0
+        t_rows = 0.0
+        if kind == "csa":
+            qi = (torch.randn(len(rows), cfg.H_I, cfg.D_I, generator=g) / math.sqrt(cfg.D_I)).to(
+                torch.bfloat16).double().numpy()
+            w = (torch.randn(len(rows), cfg.H_I, generator=g) / math.sqrt(cfg.H_I)).double().numpy()
+            ki = (torch.randn(Nc, cfg.D_I, generator=g) / math.sqrt(cfg.D_I)).to(torch.bfloat16).double().numpy()
+        for r_i, t in enumerate(rows):
+            t0 = time.perf_counter()
+            if kind == "csa":
+                idx, _ = O.indexer_topk(qi[r_i:r_i + 1], w[r_i:r_i + 1], ki, int(t), m, cfg.k)
+                O.csa_sparse_attn(q[None, r_i:r_i + 1], ckv[None], idx[None], kv[None], int(t), 0, m, cfg.W, sink,
+                                  cfg.R)
+            else:
+                O.hca_dense_attn(q[None, r_i:r_i + 1], ckv[None], kv[None], int(t), 0, m, cfg.W, sink, cfg.R)
+            t_rows += time.perf_counter() - t0
+        t_sample += t_comp + t_rows
+        t_full += B * (t_comp + t_rows / len(rows) * T)
+    desc = (f"oracle on sequence 0 of {len(layers)} layer(s): full compression + {len(rows)} stratified query rows "
+            f"per layer through indexer/top-k/attention; extrapolated to B={B} x T={T} by per-row cost")
+    return t_sample, t_full, desc
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    units = cfg.B * cfg.T if not cfg.decode else cfg.B
+    n_rows = 4
+    times, fulls = [], []
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        t_sample, t_full, desc = oracle_sample(cfg, n_rows, seed=100 + s)
+        if s >= args.warmup:
+            times.append(t_sample)
+            fulls.append(t_full)
+    full = statistics.mean(fulls)
+    value = units / full
+    unit = "queries/s" if cfg.decode else "tokens/s"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * full,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1)-scaled, BF16-rounded)",
+            "config": {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.T,
+                       "parallelism": f"dp{world}"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": _blas_threads(), "kind": "oracle",
+                             "sample": desc + f"; {statistics.mean(times):.1f} s of CPU work per step"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
+    layers = [Layer(kind, cfg, rank_seed(cfg.seed * 10 + li, rank), dev) for li, kind in enumerate(cfg.layers)]
+    runner = StackRunner(lcsa, cfg, layers, dev)
+    n0 = lcsa.kernel_launches()
+    runner.step()
+    torch.cuda.synchronize()
+    launches_per_step = lcsa.kernel_launches() - n0
+
+    # device-resident timing (per-call events recorded inside the timed steps)
+    def step_recorded():
+        runner.step()
+    for _ in range(args.warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    runner.record = True
+    runner.events.clear()
+    ms, clocks = timed(step_recorded, args.steps, 0, bus_id)
+    runner.record = False
+    ms = max_over_ranks(ms)
+    per_call = {}
+    for li, name, a, b in runner.events:
+        per_call.setdefault((li, name), []).append(a.elapsed_time(b))
+    units = cfg.B * cfg.T
+    value = weak_scaling_throughput(units, ms / 1e3, world)
+
+    # algorithmic work
+    Nc4, Nc128 = cfg.T // cfg.m, cfg.T // cfg.m_hca
+    f_csa = cfg.B * attn_flops(cfg.T, cfg.m, Nc4, cfg.W, cfg.k)
+    f_hca = cfg.B * attn_flops(cfg.T, cfg.m_hca, Nc128, cfg.W)
+    f_idx = cfg.B * indexer_flops(cfg.T, cfg.m, Nc4)
+    kern = {}
+    for (li, name), v in sorted(per_call.items()):
+        avg = statistics.mean(v)
+        d = kern.setdefault(name, {"ms": [], "layers": []})
+        d["ms"].append(avg)
+        d["layers"].append(li)
+    summary = {}
+    for name, d in kern.items():
+        avg = statistics.mean(d["ms"])
+        e = {"ms_avg": round(avg, 4), "calls_per_step": len(d["ms"])}
+        if name == "csa_sparse_attn":
+            e["tflops"] = round(f_csa / avg / 1e9, 1)
+        elif name == "hca_dense_attn":
+            e["tflops"] = round(f_hca / avg / 1e9, 1)
+        elif name == "indexer_topk":
+            e["tflops"] = round(f_idx / avg / 1e9, 1)
+        elif name.endswith("compress"):
+            m = cfg.m if name.startswith("csa") else cfg.m_hca
+            byts = cfg.B * (2 * cfg.T * cfg.D * 2 + (cfg.T // m) * cfg.D * 2)
+            e["gbs"] = round(byts / avg / 1e6, 1)
+        summary[name] = e
+    per_layer = {}
+    for (li, name), v in per_call.items():
+        per_layer[li] = per_layer.get(li, 0.0) + statistics.mean(v)
+    layer_ms = [round(per_layer[li], 3) for li in sorted(per_layer)]
+
+    # roofline of the dominant kernel (largest share of the step)
+    dom = max(summary, key=lambda n: summary[n]["ms_avg"] * summary[n]["calls_per_step"])
+    dom_flops = {"csa_sparse_attn": f_csa, "hca_dense_attn": f_hca, "indexer_topk": f_idx}.get(dom)
+    avg_ms = summary[dom]["ms_avg"]
+    peak = peaks["bf16_tflops_sustained"]
+    achieved = dom_flops / avg_ms / 1e9 if dom_flops else None
+    tr = NCU_TRAFFIC.get(dom)
+    traffic = tr["bytes_per_launch"] if tr and tr.get("src") == _src_hash(tr["file"]) else None
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"bf16_tflops_sustained of {peaks['source']}",
+                "flops_per_launch": dom_flops,
+                "note": "launch = one library call (rotary pre-pass + attention kernel); "
+                        "FLOPs = QK^T + PV over selected/visible entries plus window rows"}
+
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cfg, runner, layers, units, world)
+
+    # cpu baseline (oracle on a bounded sample) on rank 0 at N=1
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        t_sample, t_full, desc = oracle_sample(cfg, 16, seed=7)
+        cpu = {"value": units / t_full, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {t_sample:.1f} s of CPU work"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1)-scaled BF16 inputs, independent per layer and rank)",
+            "config": {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.T,
+                       "parallelism": f"dp{world}", "layers": list(cfg.layers), "heads": cfg.H, "head_dim": cfg.D,
+                       "rope_dims": cfg.R, "indexer": f"{cfg.H_I}x{cfg.D_I}", "m": cfg.m, "m_hca": cfg.m_hca,
+                       "topk": cfg.k, "window": cfg.W, "out_dtype": "bf16",
+                       "l2": "inputs larger than L2 (GBs per layer); no flush"},
+            "layer_ms": layer_ms, "kernels": summary, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
+    return line
+
+
+def run_e2e(args, cfg, runner, layers, units, world):
+    """Same stack through the public API with inputs copied from pinned host
+    memory every step and the final output read back."""
+    try:
+        hosts = {}
+        for kind in ("csa", "hca"):
+            L = next(L for L in layers if L.kind == kind)
+            hosts[kind] = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t, non_blocking=False)
+                           for n, t in L.inputs().items()}
+        out_host = torch.empty(runner.out.shape, dtype=runner.out.dtype, pin_memory=True)
+    except Exception as ex:  # host memory for pinned buffers unavailable
+        return {"value": None, "unit": "tokens/s", "error": f"pinned host buffers: {type(ex).__name__}"}
+    h2d = sum(t.numel() * t.element_size() for L in layers for t in hosts[L.kind].values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for li, L in enumerate(layers):
+            for n, t in hosts[L.kind].items():
+                getattr(L, n).copy_(t, non_blocking=True)
+            runner.layer(li)
+        out_host.copy_(runner.out, non_blocking=True)
+
+    steps = max(1, min(args.steps, 2))
+    ms, _ = timed(step, steps, 1, None, sample_clocks=False)
+    ms = max_over_ranks(ms)
+    del hosts, out_host
+    return {"value": weak_scaling_throughput(units, ms / 1e3, world), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
+    """CSA decode at 1M context: indexer top-k over 262144 entries per
+    sequence, then sparse attention over the 2048 selected entries plus the
+    128-row window ring."""
+    B, T, Nc = cfg.B, cfg.T, cfg.T // cfg.m
+    seed = rank_seed(cfg.seed, rank)
+    ix = gen.make_indexer_inputs(B, 1, Nc, cfg.H_I, cfg.D_I, "bf16", seed=seed, device=dev,
+                                 boost_frac=cfg.boost_frac)
+    g = gen._gen(seed + 1, dev)
+    ckv = gen._randn((B, Nc, cfg.D), g, dev, 1.0 / math.sqrt(cfg.D), torch.bfloat16)
+    q = gen._randn((B, 1, cfg.H, cfg.D), g, dev, 1.0 / math.sqrt(cfg.D), torch.bfloat16)
+    kvw = gen._randn((B, cfg.W, cfg.D), g, dev, 1.0 / math.sqrt(cfg.D), torch.bfloat16)
+    sink = gen._randn((cfg.H,), g, dev)
+    idx = torch.empty((B, 1, cfg.k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, 1, cfg.H, cfg.D), dtype=torch.bfloat16, device=dev)
+    ws_ix = torch.empty(lcsa.indexer_workspace_bytes(ix["q_idx"], ix["k_idx"], cfg.k), dtype=torch.uint8,
+                        device=dev)
+    ws_at = torch.empty(max(256, lcsa.attn_workspace_bytes(q, ckv, idx, kvw, cfg.m, cfg.W, cfg.R, True, T, T - cfg.W + 1)),
+                        dtype=torch.uint8, device=dev)
+    t = T                                 # query position: all 262144 entries visible
+    ev = []
+
+    def step(record=False):
+        a = torch.cuda.Event(enable_timing=True) if record else None
+        if a:
+            a.record()
+        lcsa.indexer_topk(ix["q_idx"], ix["w"], ix["k_idx"], t, cfg.m, cfg.k, workspace=ws_ix, idx_out=idx)
+        b = torch.cuda.Event(enable_timing=True) if record else None
+        if b:
+            b.record()
+        lcsa.csa_sparse_attn(q, ckv, idx, kvw, sink, t, t - cfg.W + 1, cfg.m, cfg.W, cfg.R, out=out,
+                             workspace=ws_at)
+        if record:
+            c = torch.cuda.Event(enable_timing=True)
+            c.record()
+            ev.append((a, b, c))
+
+    n0 = lcsa.kernel_launches()
+    step()
+    torch.cuda.synchronize()
+    launches = lcsa.kernel_launches() - n0
+    ms, clocks = timed(lambda: step(True), args.steps * 4, args.warmup, bus_id)
+    ms = max_over_ranks(ms)
+    ix_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    at_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    byts = B * (Nc * cfg.D_I * 2 + cfg.k * cfg.D * 2 + cfg.W * cfg.D * 2 + cfg.H * cfg.D * 2 * 2
+                + cfg.H_I * cfg.D_I * 2 + cfg.k * 4)
+    gbs = byts / (ms / 1e3) / 1e9
+    res = {"workload": cfg.name, "value": weak_scaling_throughput(B, ms / 1e3, world), "unit": "queries/s",
+           "ms_per_step": ms, "indexer_topk_ms": ix_ms, "csa_sparse_attn_ms": at_ms,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                        "bytes_per_step": byts, "peak_source": f"hbm_gbs of {peaks['source']}",
+                        "note": "whole decode step (indexer keys + gathered rows + window + q/out)"},
+           "gpu_launches": int(launches), "clocks": clocks}
+    del ix, ckv, q, kvw, idx, out, ws_ix, ws_at
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_single(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
+    """One layer workload (csa_prefill_32k or hca_prefill_128k)."""
+    kind = "csa" if cfg.name.startswith("csa") else "hca"
+    cfg1 = cfg.__class__(**{**cfg.__dict__, "layers": (kind,)})
+    line = run_stack(args, cfg1, lcsa, dev, world, rank, bus_id, peaks)
+    line["config"]["workload"] = cfg.name
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
+    ap.add_argument("--workload", default="stack_4layer_128k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = get_config(args.workload)
+
+    if args.impl == "reference":
+        run_reference(args, cfg, world, rank)
+        return
+
+    import datetime
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=dev)
+    try:
+        from __graft_entry__ import _build_module
+        if rank == 0:
+            _build_module().build()
+        _barrier()
+        import long_context_compressed_softmax_b200 as lcsa
+        bus_id = _gpu_selector(dev)
+        peaks = _peaks()
+        if cfg.decode:
+            line = run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world)
+            line = {"metric": METRIC, **line, "n_gpus": world, "steps": args.steps * 4, "warmup": args.warmup,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                    "data": "synthetic", "config": {"workload": cfg.name, "global_batch": cfg.B * world,
+                                                    "seq_len": cfg.T, "parallelism": f"dp{world}"}}
+        elif cfg.layers:
+            line = run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks)
+            if not args.no_decode:
+                torch.cuda.empty_cache()
+                line["decode_1m"] = run_decode(args, get_config("csa_decode_1m"), lcsa, dev, rank, bus_id, peaks,
+                                               world)
+        else:
+            line = run_single(args, cfg, lcsa, dev, world, rank, bus_id, peaks)
+        st = lcsa.get_device_status()
+        if st != 0:
+            line["device_status"] = st
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -66,6 +66,11 @@ typedef enum { LCSA_FP32 = 0, LCSA_BF16 = 1 } lcsa_dtype;
 const char* lcsa_version(void);
 const char* lcsa_status_string(lcsa_status s);
 
+/* Number of kernels this library has launched in the calling process (all
+ * devices, all streams).  Benchmarks read it before and after a timed region
+ * to report how many of the library's kernels ran inside it. */
+uint64_t lcsa_kernel_launches(void);
+
 /* Synchronises `stream`, returns the current device's status word in *code
  * (LCSA_DEV_*) and clears it.  Returns LCSA_ERR_DEVICE when *code != 0. */
 lcsa_status lcsa_get_device_status(void* stream, int* code);

@@ -25,7 +25,7 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported combination", 3: "wor
            4: "CUDA error", 5: "device reported an error"}
 
 EXPORTED = [
-    "lcsa_version", "lcsa_status_string", "lcsa_get_device_status",
+    "lcsa_version", "lcsa_status_string", "lcsa_get_device_status", "lcsa_kernel_launches",
     "lcsa_csa_compress", "lcsa_hca_compress",
     "lcsa_topk_workspace", "lcsa_topk_from_scores",
     "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
@@ -64,6 +64,7 @@ _vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c
 _sig = {
     "lcsa_version": (ctypes.c_char_p, []),
     "lcsa_status_string": (ctypes.c_char_p, [_i]),
+    "lcsa_kernel_launches": (ctypes.c_uint64, []),
     "lcsa_get_device_status": (_i, [_vp, ctypes.POINTER(_i)]),
     "lcsa_csa_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
     "lcsa_hca_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
@@ -118,6 +119,11 @@ def _need_contig(*ts):
 
 def version() -> str:
     return _lib.lcsa_version().decode()
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(_lib.lcsa_kernel_launches())
 
 
 def get_device_status() -> int:
@@ -213,8 +219,8 @@ def _attn_args(q, ckv, idx, kv, sink, q_pos0, kv_pos0, m, W, R, softmax_scale, r
                     _dt(out), _p(lse))
 
 
-def attn_workspace_bytes(q, ckv, idx, kv, m, W, R=64, sparse=True):
-    a = _attn_args(q, ckv, idx, kv, None, 0, 0, m, W, R, 0.0, 0.0, q, None)
+def attn_workspace_bytes(q, ckv, idx, kv, m, W, R=64, sparse=True, q_pos0=0, kv_pos0=0):
+    a = _attn_args(q, ckv, idx, kv, None, q_pos0, kv_pos0, m, W, R, 0.0, 0.0, q, None)
     return int(_lib.lcsa_attn_workspace(ctypes.byref(a), 1 if sparse else 0))
 
 

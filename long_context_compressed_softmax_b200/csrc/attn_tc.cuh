@@ -616,8 +616,10 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)rows, pl.splits);
   attn_tc_kernel<<<grid, kAtThreads, kAtSmem, st>>>(P, g);
+  count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
+  count_launch();
   attn_combine_kernel<<<(unsigned)(rows * 64), 128, 0, st>>>(P.o_part, P.ml_part, a->sink, a->out, a->lse,
                                                               pl.splits, rows, a->Tq, a->q_pos0, log_base,
                                                               g.out_bf16);

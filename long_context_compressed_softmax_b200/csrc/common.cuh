@@ -18,6 +18,13 @@ __device__ int g_status;
 
 __device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
 
+// Host-side count of kernel launches issued by the library.
+inline unsigned long long& launch_counter() {
+  static unsigned long long n = 0;
+  return n;
+}
+inline void count_launch(int n = 1) { __atomic_fetch_add(&launch_counter(), (unsigned long long)n, __ATOMIC_RELAXED); }
+
 // ---------------------------------------------------------------------------
 // Element load / store helpers (BF16 storage, FP32 arithmetic).
 // ---------------------------------------------------------------------------

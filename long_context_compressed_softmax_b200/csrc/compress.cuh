@@ -110,6 +110,7 @@ static cudaError_t launch_compress_t(const void* kv, const void* gate, int per_c
   const int threads = epb * tpe <= 1024 ? (epb * tpe < 32 ? 32 : epb * tpe) : 1024;
   dim3 grid((Nc + epb - 1) / epb, B);
   const size_t smem = rms_w ? (size_t)epb * sizeof(float) : 0;
+  count_launch();
   if (per_channel)
     compress_kernel<Tin, Tout, true><<<grid, threads, smem, st>>>(
         (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, window, Nc, epb, rms_w, rms_eps);

@@ -224,6 +224,7 @@ static cudaError_t launch_indexer_tc_rect(const lcsa_indexer_args* a, float* sco
   if (e != cudaSuccess) return e;
   dim3 grid(n_groups, splits);
   indexer_tc_kernel<<<grid, kIxThreads, kIxSmem, st>>>(qm, km, a->w, scores, g);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -97,6 +97,7 @@ cudaError_t launch_attn_generic_t(const lcsa_attn_args* a, int sparse, cudaStrea
                                        (int)smem);
   if (e != cudaSuccess) return e;
   const long long blocks = (long long)a->B * a->Tq * a->H;
+  count_launch();
   attn_generic<T, To><<<(unsigned)blocks, 128, smem, st>>>(
       (const T*)a->q, (const T*)a->ckv, a->idx, (const T*)a->kv, a->sink, (To*)a->out, a->lse, a->Tq, a->H,
       a->D, a->R, a->Nc, a->k, a->Tkv, a->q_pos0, a->kv_pos0, a->m, a->W, scale, log_base, sparse);
@@ -119,6 +120,7 @@ cudaError_t launch_indexer_generic_t(const lcsa_indexer_args* a, float* scores, 
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a->Nc + 63) / 64, rows);
+  count_launch();
   indexer_scores_generic<T><<<grid, 256, smem, st>>>((const T*)a->q_idx, a->w, (const T*)a->k_idx, scores, a->Tq,
                                                      a->Nc, a->H_I, a->D_I, a->q_pos0, a->m, row0);
   return cudaGetLastError();
@@ -139,6 +141,8 @@ __global__ void nvalid_kernel(int32_t* nv, int rows, int i0, int ni, long long q
 extern "C" {
 
 const char* lcsa_version(void) { return "lcsa 0.1 (sm_100a)"; }
+
+uint64_t lcsa_kernel_launches(void) { return __atomic_load_n(&launch_counter(), __ATOMIC_RELAXED); }
 
 const char* lcsa_status_string(lcsa_status s) {
   switch (s) {
@@ -245,6 +249,7 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_
         else e = launch_indexer_generic_t<float>(a, sc, (int)row0, nr, st);
         if (e != cudaSuccess) return LCSA_ERR_CUDA;
       }
+      count_launch();
       nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, a->q_pos0, a->m, a->Nc);
       e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st);
       if (e != cudaSuccess) return LCSA_ERR_CUDA;

@@ -52,6 +52,7 @@ static cudaError_t launch_rope_rows(const void* src, void* dst, long long n_rows
                                     const int32_t* idx, long long slots_per_seq, int Nc, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
   const long long blocks = (n_rows + 7) / 8;
+  count_launch();
   rope_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>((const __nv_bfloat16*)src, (__nv_bfloat16*)dst, n_rows, D,
                                                      rows_per_seq, pos0, pos_step, log_base, mode, idx,
                                                      slots_per_seq, Nc);

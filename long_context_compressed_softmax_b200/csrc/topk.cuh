@@ -164,6 +164,7 @@ static cudaError_t launch_topk(const float* scores, int rows, int n_cols, long l
   cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel<kTopkThreads>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCachedKeys * 4);
   if (e != cudaSuccess) return e;
+  count_launch();
   topk_rows_kernel<kTopkThreads><<<rows, kTopkThreads, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out,
                                                                    cache_cap);
   return cudaGetLastError();

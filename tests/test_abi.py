@@ -12,10 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lcsa():
-    from long_context_compressed_softmax_b200 import build
-    build.build()
-    import long_context_compressed_softmax_b200 as m
-    return m
+    from conftest import build_library
+    return build_library()
 
 
 def _declared():

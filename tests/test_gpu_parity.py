@@ -16,10 +16,8 @@ ATT_MAX, ATT_MEAN = 1e-2, 1e-3        # attention tolerance (BF16 in, FP32 accum
 def lcsa():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from long_context_compressed_softmax_b200 import build
-    build.build()
-    import long_context_compressed_softmax_b200 as m
-    return m
+    from conftest import build_library
+    return build_library()
 
 
 DEV = "cuda"

@@ -26,11 +26,25 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
-def _randn(shape, g, device, scale=1.0):
-    x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
-    if scale != 1.0:
-        x.mul_(scale)
-    return x
+_CHUNK = 1 << 24     # elements drawn per generator call (fixes the stream for any size)
+
+
+def randn_into(out: torch.Tensor, g: torch.Generator, scale=1.0):
+    """Fill `out` (any float dtype) with N(0,1)*scale drawn in FP32 chunk by
+    chunk and rounded once to out.dtype; no full-size FP32 temporary."""
+    flat = out.view(-1)
+    n = flat.numel()
+    for i in range(0, n, _CHUNK):
+        j = min(n, i + _CHUNK)
+        x = torch.randn(j - i, generator=g, device=out.device, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        flat[i:j].copy_(x)
+    return out
+
+
+def _randn(shape, g, device, scale=1.0, dtype=torch.float32):
+    return randn_into(torch.empty(shape, dtype=dtype, device=device), g, scale)
 
 
 def storage_dtype(dtype: str) -> torch.dtype:
@@ -42,9 +56,9 @@ def make_compress_inputs(B, T, D, dtype="bf16", seed=0, device="cpu",
     """kv [B,T,D] and gate logits [B,T,D] (or [B,T] for a per-token gate)."""
     g = _gen(seed, device)
     kv_scale = 1.0 / math.sqrt(D) if kv_scale is None else kv_scale
-    kv = _randn((B, T, D), g, device, kv_scale).to(_DT[dtype])
+    kv = _randn((B, T, D), g, device, kv_scale, _DT[dtype])
     gshape = (B, T, D) if gate_per_channel else (B, T)
-    gate = _randn(gshape, g, device, gate_scale).to(_DT[dtype])
+    gate = _randn(gshape, g, device, gate_scale, _DT[dtype])
     return {"kv": kv, "gate": gate}
 
 
@@ -59,10 +73,9 @@ def make_indexer_inputs(B, Tq, Nc, H_I=64, D_I=128, dtype="bf16", seed=0, device
     heavy-tailed (the +3 sigma boosted-affinity workload).
     """
     g = _gen(seed, device)
-    q = _randn((B, Tq, H_I, D_I), g, device, 1.0 / math.sqrt(D_I))
+    q = _randn((B, Tq, H_I, D_I), g, device, 1.0 / math.sqrt(D_I), _DT[dtype])
     w = _randn((B, Tq, H_I), g, device, 1.0 / math.sqrt(H_I))
     k = _randn((B, Nc, D_I), g, device, 1.0 / math.sqrt(D_I))
-    q = q.to(_DT[dtype])
     if boost_frac > 0.0:
         n_boost = max(1, int(round(boost_frac * Nc)))
         qf = q.float()
@@ -80,9 +93,9 @@ def make_attn_inputs(B, Tq, H, D, Nc, Tkv, dtype="bf16", seed=0, device="cpu",
     kv [B,Tkv,D] and per-head sink logits [H] (FP32)."""
     g = _gen(seed, device)
     s = 1.0 if unit_scale else 1.0 / math.sqrt(D)
-    q = _randn((B, Tq, H, D), g, device, s).to(_DT[dtype])
-    ckv = _randn((B, Nc, D), g, device, s).to(_DT[dtype])
-    kv = _randn((B, Tkv, D), g, device, s).to(_DT[dtype])
+    q = _randn((B, Tq, H, D), g, device, s, _DT[dtype])
+    ckv = _randn((B, Nc, D), g, device, s, _DT[dtype])
+    kv = _randn((B, Tkv, D), g, device, s, _DT[dtype])
     sink = _randn((H,), g, device) if with_sink else None
     return {"q": q, "ckv": ckv, "kv": kv, "sink": sink}
 
