@@ -32,7 +32,10 @@ constexpr uint32_t kAtQBytes = 64 * 512 * 2;   // 64 KB
 constexpr uint32_t kAtKBytes = kAtKT * 512 * 2;  // 64 KB
 constexpr uint32_t kAtPBytes = 64 * kAtKT * 2;   // 8 KB
 constexpr uint32_t kAtRegion = 64 * 128;       // one 64-dim column block of a 64-row tile
-constexpr size_t kAtSmem = 1024 + kAtQBytes + 2 * kAtKBytes + 2 * kAtPBytes + 2 * kAtKT * 16 + 64 * 8 + 256;
+constexpr int kAtMaxIdx = 2048;                 // selected entries staged in shared memory per CTA
+constexpr int kAtStages = 3;                    // K=V tile stages
+constexpr size_t kAtSmem = 1024 + kAtStages * kAtKBytes + 2 * kAtPBytes + kAtStages * kAtKT * 2 * 8 +
+                           kAtMaxIdx * 4 + 32 * 8 + 16 * 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AtGeom {
@@ -72,6 +75,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Arrive on `bar` (counted as one of its expected arrivals) once every
+// cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Key-set geometry of one query.
 struct KeySet {
@@ -108,21 +117,19 @@ __device__ __forceinline__ KeySet key_set(const AtGeom& g, const int32_t* idx_ro
 __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_q = smem;
-  uint8_t* s_k = s_q + kAtQBytes;                  // 2 stages
-  uint8_t* s_p = s_k + 2 * kAtKBytes;              // 2 buffers
-  const uint8_t** s_rowmain = reinterpret_cast<const uint8_t**>(s_p + 2 * kAtPBytes);   // [2][64]
-  const uint8_t** s_rowrope = s_rowmain + 2 * kAtKT;                                    // [2][64]
-  float2* s_cs = reinterpret_cast<float2*>(s_rowrope + 2 * kAtKT);                       // [32] (cos, sin) at t
+  uint8_t* s_k = smem;                                                  // kAtStages K=V tiles
+  uint8_t* s_p = s_k + kAtStages * kAtKBytes;                           // 2 P buffers
+  const uint8_t** s_tab = reinterpret_cast<const uint8_t**>(s_p + 2 * kAtPBytes);   // [stage][64][2] row pointers
+  int32_t* s_idx = reinterpret_cast<int32_t*>(s_tab + kAtStages * kAtKT * 2);       // selected entries of this range
+  float2* s_cs = reinterpret_cast<float2*>(s_idx + kAtMaxIdx);                      // [32] (cos, sin) at t
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_cs + 32);
-  uint64_t* q_full = bars + 0;       // producers (128)
-  uint64_t* q_ready = bars + 1;      // softmax warps (4)
-  uint64_t* kv_full = bars + 2;      // [2] producers (128)
-  uint64_t* kv_empty = bars + 4;     // [2] MMA commit
-  uint64_t* s_full = bars + 6;       // [2] MMA commit
-  uint64_t* s_free = bars + 8;       // [2] softmax warps (4)
-  uint64_t* p_full = bars + 10;      // [2] softmax warps (4)
-  uint64_t* pv_done = bars + 12;     // [2] MMA commit
+  uint64_t* q_ready = bars + 0;                 // softmax warps (4): Q is in TMEM
+  uint64_t* kv_full = bars + 1;                 // [kAtStages] producers (128, async arrivals)
+  uint64_t* kv_empty = kv_full + kAtStages;     // [kAtStages] MMA commit
+  uint64_t* s_full = kv_empty + kAtStages;      // [2] MMA commit
+  uint64_t* s_free = s_full + 2;                // [2] softmax warps (4)
+  uint64_t* p_full = s_free + 2;                // [2] softmax warps (4)
+  uint64_t* pv_done = p_full + 2;               // [2] MMA commit
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -140,7 +147,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
 
   // ---------------------------------------------------------------- no keys
   if (n_tiles == 0) {
-    // zero output (or neutral partial); lse = sink (or -inf)
     for (int e = threadIdx.x; e < 64 * 512; e += kAtThreads) {
       const long long o = row * 64 * 512 + e;
       if (g.splits > 1) P.o_part[(long long)split * gridDim.x * 64 * 512 + o] = 0.f;
@@ -160,11 +166,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
   }
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(q_full, 128);
     tc::mbar_init(q_ready, 4);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kAtStages; ++s) {
       tc::mbar_init(kv_full + s, 128);
       tc::mbar_init(kv_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(s_full + s, 1);
       tc::mbar_init(s_free + s, 4);
       tc::mbar_init(p_full + s, 4);
@@ -179,6 +186,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
   tc::tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
+  // TMEM map: lanes 0-15 of each sub-partition hold S[0] (cols 0-63), S[1]
+  // (64-127) and Q (128-383, the A operand of S = Q K^T); lanes 16-31 hold O
+  // (cols 0-511).
+  constexpr uint32_t kTmQ = 128;
+  constexpr uint32_t kTmO = 16u << 16;
 
   if (warp < 4) {
     // ============================================================ producers
@@ -186,27 +198,19 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
     const int piece = tid & 63;                     // 16-byte piece of a 1 KB row
     const int region = piece >> 3, c16 = piece & 7;
     const int kk0 = tid >> 6;                       // keys kk0, kk0+2, ..., kk0+62
-    // Q: 64 head rows
-    {
-      const uint8_t* qrow0 = reinterpret_cast<const uint8_t*>(P.q + row * 64 * 512);
-      const uint32_t qb = tc::smem_u32(s_q);
-#pragma unroll 4
-      for (int u = 0; u < 32; ++u) {
-        const int h = kk0 + 2 * u;
-        const uint32_t dst = qb + region * kAtRegion + h * 128 + ((c16 ^ (h & 7)) << 4);
-        cp_async16(dst, qrow0 + (long long)h * 1024 + piece * 16, 16);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(q_full);
+    const int slot0 = t0 * kAtKT;
+    if (g.sparse) {
+      const int n_sel = (ks.n_c < t1 * kAtKT ? ks.n_c : t1 * kAtKT) - slot0;
+      for (int e = tid; e < n_sel; e += 128) s_idx[e] = idx_row[slot0 + e];
+      named_bar(1, 128);
     }
+    const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.q);
     for (int n = 0; n < n_tiles; ++n) {
-      const int s = n & 1;
-      if (n >= 2 && !tc::mbar_wait(kv_empty + s, ((n - 2) >> 1) & 1)) { *abort_flag = 1; }
+      const int s = n % kAtStages;
+      if (n >= kAtStages && !tc::mbar_wait_backoff(kv_empty + s, ((n - kAtStages) / kAtStages) & 1)) *abort_flag = 1;
       if (*abort_flag) break;
       const int gt = t0 + n;                        // tile index in the query's key list
-      // row table for this tile (64 threads)
+      const uint8_t** tab = s_tab + s * kAtKT * 2;
       if (tid < kAtKT) {
         const int kk = tid;
         const uint8_t* rm = nullptr;
@@ -214,12 +218,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
         if (gt < ks.tiles_c) {
           const int slot = gt * kAtKT + kk;
           if (slot < ks.n_c) {
-            int j = g.sparse ? idx_row[slot] : slot;
-            if (j < 0 || j >= g.Nc) { report(LCSA_DEV_BAD_INDEX); j = -1; }
-            if (j >= 0) {
+            const int j = g.sparse ? s_idx[slot - slot0] : slot;
+            if (j >= 0 && j < g.Nc) {
               rm = reinterpret_cast<const uint8_t*>(P.ckv + ((long long)b * g.Nc + j) * 512);
               rr = reinterpret_cast<const uint8_t*>(
                   P.rot_c + (g.rot_slot ? (row * g.k + slot) : ((long long)b * g.Nc + j)) * 64);
+            } else {
+              report(LCSA_DEV_BAD_INDEX);
             }
           }
         } else {
@@ -230,87 +235,88 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
             rr = reinterpret_cast<const uint8_t*>(P.rot_w + ((long long)b * g.Tkv + r) * 64);
           }
         }
-        s_rowmain[s * kAtKT + kk] = rm;
-        s_rowrope[s * kAtKT + kk] = rr;
+        tab[2 * kk] = rm;
+        tab[2 * kk + 1] = rr;
       }
       named_bar(1, 128);
-      const uint32_t kb = tc::smem_u32(s_k + s * kAtKBytes);
-      const void* dummy = P.q;
-#pragma unroll 4
+      const uint32_t kb = tc::smem_u32(s_k + s * kAtKBytes) + region * kAtRegion + (c16 << 4);
+      const int off = region == 7 ? c16 * 16 : piece * 16;
+#pragma unroll 8
       for (int u = 0; u < 32; ++u) {
         const int kk = kk0 + 2 * u;
-        const uint8_t* rm = s_rowmain[s * kAtKT + kk];
-        const uint8_t* src;
-        uint32_t nbytes = 16;
-        if (rm == nullptr) { src = reinterpret_cast<const uint8_t*>(dummy); nbytes = 0; }
-        else if (region == 7) src = s_rowrope[s * kAtKT + kk] + c16 * 16;
-        else src = rm + piece * 16;
-        const uint32_t dst = kb + region * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4);
-        cp_async16(dst, src, nbytes);
+        const uint8_t* base = tab[2 * kk + (region == 7 ? 1 : 0)];
+        const uint32_t dst = (kb + kk * 128) ^ ((uint32_t)(kk & 7) << 4);
+        cp_async16(dst, base ? base + off : dummy, base ? 16u : 0u);
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(kv_full + s);
+      cp_async_arrive_noinc(kv_full + s);
     }
+    cp_async_wait_all();                            // nothing may land after the CTA exits
   } else if (warp == 4) {
     // ============================================================ MMA issuer
+    // S(n+1) and PV(n) are independent: whichever is ready is issued first.
     if (tc::elect_one()) {
-      const uint32_t idesc_s = tc::idesc_bf16(64, kAtKT, 0, 0);    // A K-major, B K-major
+      const uint32_t idesc_s = tc::idesc_bf16(64, kAtKT, 0, 0);    // A (TMEM) K-major, B K-major
       const uint32_t idesc_o = tc::idesc_bf16(64, 256, 0, 1);      // A K-major, B MN-major
-      const uint32_t qb = tc::smem_u32(s_q);
-      const uint32_t tm_s = tmem + (16u << 16);                     // S: lanes 16-31 of each sub-partition
       bool ok = tc::mbar_wait(q_ready, 0);
-      auto issue_s = [&](int n) {
-        const int s = n & 1;
-        const uint32_t kb = tc::smem_u32(s_k + s * kAtKBytes);
+      int next_s = 0, next_pv = 0;
+      uint64_t t_idle = 0;
+      while (ok && next_pv < n_tiles) {
+        bool did = false;
+        if (next_s < n_tiles && next_s <= next_pv + 1) {
+          const int st = next_s % kAtStages, sb = next_s & 1;
+          if (tc::mbar_try_wait(kv_full + st, (next_s / kAtStages) & 1) &&
+              (next_s < 2 || tc::mbar_try_wait(s_free + sb, ((next_s >> 1) - 1) & 1))) {
+            tc::tc_fence_after();
+            const uint32_t kb = tc::smem_u32(s_k + st * kAtKBytes);
 #pragma unroll
-        for (int kstep = 0; kstep < 32; ++kstep) {
-          const uint32_t off = (uint32_t)((kstep >> 2) * kAtRegion + (kstep & 3) * 32);
-          tc::mma_bf16_ss(tm_s + s * kAtKT, tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024),
-                          idesc_s, kstep > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(s_full + s);
-      };
-      if (ok && tc::mbar_wait(kv_full, 0)) {
-        tc::tc_fence_after();
-        issue_s(0);
-      } else {
-        ok = false;
-      }
-      for (int n = 0; ok && n < n_tiles; ++n) {
-        if (*abort_flag) { ok = false; break; }
-        if (n + 1 < n_tiles) {
-          const int s1 = (n + 1) & 1;
-          if (!tc::mbar_wait(kv_full + s1, ((n + 1) >> 1) & 1)) { ok = false; break; }
-          if (n + 1 >= 2 && !tc::mbar_wait(s_free + s1, (((n + 1) >> 1) - 1) & 1)) { ok = false; break; }
-          tc::tc_fence_after();
-          issue_s(n + 1);
-        }
-        const int s = n & 1;
-        if (!tc::mbar_wait(p_full + s, (n >> 1) & 1)) { ok = false; break; }
-        tc::tc_fence_after();
-        const uint32_t pb = tc::smem_u32(s_p + s * kAtPBytes);
-        const uint32_t kb = tc::smem_u32(s_k + s * kAtKBytes);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int kstep = 0; kstep < kAtKT / 16; ++kstep) {
-            const uint64_t ad = tc::sdesc_sw128(pb + kstep * 32, 16, 1024);
-            const uint64_t bd = tc::sdesc_sw128(kb + half * 4 * kAtRegion + kstep * 2048, kAtRegion, 1024);
-            tc::mma_bf16_ss(tmem + half * 256, ad, bd, idesc_o, (n > 0 || kstep > 0) ? 1u : 0u);
+            for (int kstep = 0; kstep < 32; ++kstep) {
+              const uint32_t off = (uint32_t)((kstep >> 2) * kAtRegion + (kstep & 3) * 32);
+              tc::mma_bf16_ts(tmem + sb * kAtKT, tmem + kTmQ + kstep * 8, tc::sdesc_sw128(kb + off, 16, 1024),
+                              idesc_s, kstep > 0 ? 1u : 0u);
+            }
+            tc::mma_commit(s_full + sb);
+            ++next_s;
+            did = true;
           }
         }
-        tc::mma_commit(kv_empty + s);
-        tc::mma_commit(pv_done + s);
+        if (next_pv < next_s) {
+          const int st = next_pv % kAtStages, sb = next_pv & 1;
+          if (tc::mbar_try_wait(p_full + sb, (next_pv >> 1) & 1)) {
+            tc::tc_fence_after();
+            const uint32_t pb = tc::smem_u32(s_p + sb * kAtPBytes);
+            const uint32_t kb = tc::smem_u32(s_k + st * kAtKBytes);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+              for (int kstep = 0; kstep < kAtKT / 16; ++kstep) {
+                const uint64_t ad = tc::sdesc_sw128(pb + kstep * 32, 16, 1024);
+                const uint64_t bd = tc::sdesc_sw128(kb + half * 4 * kAtRegion + kstep * 2048, kAtRegion, 1024);
+                tc::mma_bf16_ss(tmem + kTmO + half * 256, ad, bd, idesc_o, (next_pv > 0 || kstep > 0) ? 1u : 0u);
+              }
+            }
+            tc::mma_commit(kv_empty + st);
+            tc::mma_commit(pv_done + sb);
+            ++next_pv;
+            did = true;
+          }
+        }
+        if (did) {
+          t_idle = 0;
+        } else if (*abort_flag) {
+          ok = false;
+        } else {
+          const uint64_t now = tc::globaltimer();
+          if (t_idle == 0) t_idle = now;
+          else if (now - t_idle > tc::kWaitLimitNs) { report(LCSA_DEV_TIMEOUT); ok = false; }
+        }
       }
       if (!ok) *abort_flag = 1;
     }
   } else {
     // ============================================================ softmax / epilogue
     const int quarter = warp & 3;
-    const bool s_owner = lane >= 16;
-    const int h = quarter * 16 + (lane & 15);         // head row this thread owns (S or O)
+    const bool s_owner = lane < 16;                   // lanes 0-15: S rows; lanes 16-31: O rows
+    const int h = quarter * 16 + (lane & 15);         // head row this thread owns
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int stid = threadIdx.x - 5 * 32;            // 0..127
     // rotary table at position t (shared by the Q rotation and the -t output rotation)
@@ -319,38 +325,55 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
       rope_cs(t, stid, kRopeR, g.log_base, &c, &sn);
       s_cs[stid] = make_float2(c, sn);
     }
-    bool ok = tc::mbar_wait(q_full, 0);
     named_bar(2, 128);
-    if (ok) {
-      // rotate Q's rotary block (region 7) in place: 64 rows x 32 pairs
-      for (int e = stid; e < 64 * 32; e += 128) {
-        const int hr = e >> 5, p = e & 31;
-        const int byte = p * 4;                               // pair p -> bytes [4p, 4p+4)
-        uint8_t* addr = s_q + 7 * kAtRegion + hr * 128 + ((((byte >> 4) ^ (hr & 7))) << 4) + (byte & 15);
-        __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(addr);
-        const float2 f = __bfloat1622float2(*x);
-        const float2 cs = s_cs[p];
-        *x = __floats2bfloat162_rn(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
+    // Q -> TMEM (A operand): lane h holds head h's 512 dims, two per column; the
+    // rotary block (dims 448..511) is rotated at t on the way.
+    {
+      const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row * 64 + h) * 512);
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {                  // 32 dims = 16 columns per step
+        uint32_t r[16];
+        if (s_owner) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = __ldg(qrow + 4 * c + v);
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          if (c >= 14) {
+#pragma unroll
+            for (int q2 = 0; q2 < 16; ++q2) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r[q2]));
+              const float2 cs = s_cs[(c - 14) * 16 + q2];
+              const __nv_bfloat162 o = __floats2bfloat162_rn(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
+              r[q2] = *reinterpret_cast<const uint32_t*>(&o);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q2 = 0; q2 < 16; ++q2) r[q2] = 0u;   // O lanes: overwritten by the first PV
+        }
+        tc::tmem_st16(tmem + lane_base + kTmQ + c * 16, r);
       }
-      tc::fence_proxy_async_smem();
+      tc::tmem_wait_st();
     }
+    tc::tc_fence_before();
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(q_ready);
 
+    bool ok = true;
     float m_run = -INFINITY, l_run = 0.f;
     for (int n = 0; ok && n < n_tiles; ++n) {
-      const int s = n & 1;
+      const int sb = n & 1;
       if (*abort_flag) { ok = false; break; }
-      if (!tc::mbar_wait(s_full + s, (n >> 1) & 1)) { ok = false; break; }
+      if (!tc::mbar_wait(s_full + sb, (n >> 1) & 1)) { ok = false; break; }
       tc::tc_fence_after();
       uint32_t v[64];
-      tc::tmem_ld32(tmem + lane_base + s * kAtKT, v);
-      tc::tmem_ld32(tmem + lane_base + s * kAtKT + 32, v + 32);
+      tc::tmem_ld32(tmem + lane_base + sb * kAtKT, v);
+      tc::tmem_ld32(tmem + lane_base + sb * kAtKT + 32, v + 32);
       tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(s_free + s);
-      // valid keys in this tile
+      if (lane == 0) tc::mbar_arrive(s_free + sb);
       const int gt = t0 + n;
       int nvalid = gt < ks.tiles_c ? ks.n_c - gt * kAtKT : ks.n_w - (gt - ks.tiles_c) * kAtKT;
       nvalid = nvalid < kAtKT ? nvalid : kAtKT;
@@ -372,15 +395,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
           rescale = true;
         }
       }
-      // the O-owner (lane - 16) rescales the O row when its S-owner asks
-      const float alpha_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-      const bool any_rescale = __any_sync(0xffffffffu, rescale);
-      if (any_rescale) {
-        // PV(n-1) must have finished before O is touched, and the 32-lane
-        // read-modify-write below also rewrites the S lanes: S(n+1), the only
-        // S that can be in flight now, must have landed first.
-        if (!tc::mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1)) { ok = false; }
-        if (n + 1 < n_tiles && !tc::mbar_wait(s_full + ((n + 1) & 1), ((n + 1) >> 1) & 1)) { ok = false; }
+      // the O-owner (lane + 16) rescales the O row when its S-owner asks
+      const float alpha_o = __shfl_sync(0xffffffffu, alpha, lane & 15);
+      if (__any_sync(0xffffffffu, rescale)) {
+        // The 32-lane read-modify-write below also rewrites lanes 0-15 (S, Q):
+        // it runs only once PV(n-1) and S(n+1) have finished, when no MMA can
+        // be in flight (S(n+2) and PV(n) both wait for this tile's P).
+        if (!tc::mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1)) ok = false;
+        if (n + 1 < n_tiles && !tc::mbar_wait(s_full + ((n + 1) & 1), ((n + 1) >> 1) & 1)) ok = false;
         tc::tc_fence_after();
         for (int c = 0; c < 512; c += 16) {
           uint32_t r[16];
@@ -388,28 +410,28 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
           tc::tmem_wait_ld();
           if (!s_owner) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha_o);
+            for (int q2 = 0; q2 < 16; ++q2) r[q2] = __float_as_uint(__uint_as_float(r[q2]) * alpha_o);
           }
-          tc::tmem_st16(tmem + lane_base + c, r);      // S-owner lanes (16-31) write back what they read
+          tc::tmem_st16(tmem + lane_base + c, r);
         }
         tc::tmem_wait_st();
       }
       if (s_owner) l_run *= alpha;
-      // P buffer s is free once PV(n-2) is done
-      if (n >= 2 && !tc::mbar_wait(pv_done + s, ((n - 2) >> 1) & 1)) { ok = false; }
+      // P buffer sb is free once PV(n-2) is done
+      if (n >= 2 && !tc::mbar_wait(pv_done + sb, ((n - 2) >> 1) & 1)) ok = false;
       if (s_owner) {
         float psum = 0.f;
-        uint8_t* prow = s_p + s * kAtPBytes + h * 128;
+        uint8_t* prow = s_p + sb * kAtPBytes + h * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t pk[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float p0 = exp2f(x[8 * c + 2 * q] - m_run);
-            const float p1 = exp2f(x[8 * c + 2 * q + 1] - m_run);
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float p0 = exp2f(x[8 * c + 2 * q2] - m_run);
+            const float p1 = exp2f(x[8 * c + 2 * q2 + 1] - m_run);
             psum += p0 + p1;
             __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
-            pk[q] = *reinterpret_cast<uint32_t*>(&bp);
+            pk[q2] = *reinterpret_cast<uint32_t*>(&bp);
           }
           *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
@@ -418,14 +440,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(p_full + s);
+      if (lane == 0) tc::mbar_arrive(p_full + sb);
     }
     // ---------------------------------------------------------- epilogue
     if (ok && !tc::mbar_wait(pv_done + ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1)) ok = false;
     tc::tc_fence_after();
-    // the O-owner (lane < 16) takes m, l from its S-owner (lane + 16)
-    const float m_o = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
-    const float l_o = __shfl_sync(0xffffffffu, l_run, (lane & 15) + 16);
+    // the O-owner (lane >= 16) takes m, l from its S-owner (lane - 16)
+    const float m_o = __shfl_sync(0xffffffffu, m_run, lane & 15);
+    const float l_o = __shfl_sync(0xffffffffu, l_run, lane & 15);
     if (ok) {
       const long long orow = row * 64 + h;
       float scale_out;
@@ -452,19 +474,19 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
       }
       for (int c = 0; c < 512; c += 32) {
         uint32_t r[32];
-        tc::tmem_ld32(tmem + lane_base + c, r);
+        tc::tmem_ld32(tmem + lane_base + c, r);         // lanes 16-31: O rows
         tc::tmem_wait_ld();
         if (!s_owner) {
           float o[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(r[q]) * scale_out;
+          for (int q2 = 0; q2 < 32; ++q2) o[q2] = __uint_as_float(r[q2]) * scale_out;
           if (g.splits == 1 && c >= 448) {
 #pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              const float2 cs = s_cs[(c - 448 + q) >> 1];          // rotate by -t: (cos, -sin)
-              const float a0 = o[q], a1 = o[q + 1];
-              o[q] = a0 * cs.x + a1 * cs.y;
-              o[q + 1] = -a0 * cs.y + a1 * cs.x;
+            for (int q2 = 0; q2 < 32; q2 += 2) {
+              const float2 cs = s_cs[(c - 448 + q2) >> 1];          // rotate by -t: (cos, -sin)
+              const float a0 = o[q2], a1 = o[q2 + 1];
+              o[q2] = a0 * cs.x + a1 * cs.y;
+              o[q2 + 1] = -a0 * cs.y + a1 * cs.x;
             }
           }
           if (g.splits > 1) {
@@ -550,6 +572,11 @@ static AtPlan attn_tc_plan(const lcsa_attn_args* a, int sparse) {
     splits = (int)((2 * 148 + rows - 1) / rows);
     const int cap = max_tiles / 4 > 1 ? max_tiles / 4 : 1;        // >= 4 tiles per split
     splits = splits < cap ? splits : cap;
+  }
+  // A CTA stages at most kAtMaxIdx selected entries: larger k needs more key-range splits.
+  if (sparse && a->k > kAtMaxIdx) {
+    const int need = (max_tiles + kAtMaxIdx / kAtKT - 1) / (kAtMaxIdx / kAtKT);
+    splits = splits > need ? splits : need;
   }
   p.splits = splits;
   p.rot_slot = sparse && ((long long)a->Tq * a->k < (long long)a->Nc) ? 1 : 0;

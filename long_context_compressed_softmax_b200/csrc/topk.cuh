@@ -3,9 +3,12 @@
 // index; indices emitted ascending, -1 padded.)
 //
 // One CTA per row.  Scores map to 32-bit keys whose unsigned order is the
-// float order (-0 folded onto +0).  Four 8-bit MSB-first histogram passes in
-// shared memory find the k-th largest key K and how many of its ties to keep;
-// a last pass in index order writes every key > K plus the first r ties, with
+// float order (-0 folded onto +0).  Three MSB-first histogram passes over
+// 12, 12 and 8 key bits (4096-bin shared-memory histograms: a score's sign,
+// exponent and top mantissa bits land in distinct bins, which keeps
+// same-address atomics rare) find the k-th largest key K and how many of its
+// ties to keep; a pass stops early once the threshold bucket is taken whole.
+// A last pass in index order writes every key > K plus the first r ties, with
 // output slots from a block-wide prefix count, so the list comes out
 // ascending.  Rows up to kMaxCachedKeys are staged in shared memory once;
 // longer rows are re-read from L2 on every pass.
@@ -16,6 +19,7 @@ namespace lcsa {
 
 constexpr int kTopkThreads = 512;
 constexpr int kMaxCachedKeys = 32768;   // 128 KiB of dynamic shared memory
+constexpr int kTopkBins = 4096;
 
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -23,7 +27,7 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan of one packed value (two 16-bit counters).
+// Exclusive block scan (NT threads); also returns the block total.
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -47,8 +51,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
     if (lane == 31) *total = z;
   }
   __syncthreads();
-  const uint32_t r = s_warp[warp] + x - v;
-  return r;
+  return s_warp[warp] + x - v;
 }
 
 template <int NT>
@@ -56,8 +59,9 @@ __global__ void __launch_bounds__(NT)
 topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
                  const int32_t* __restrict__ n_valid, int k, int32_t* __restrict__ idx_out,
                  int cache_cap) {
+  static_assert(kTopkBins == 8 * NT, "each thread owns 8 bins");
   extern __shared__ uint32_t s_keys[];
-  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_hist[kTopkBins];
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_total;
   __shared__ uint32_t s_prefix, s_mask, s_kr;
@@ -80,49 +84,39 @@ topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
   if (cached)
     for (int i = threadIdx.x; i < n; i += NT) s_keys[i] = score_key(__ldg(src + i));
   if (threadIdx.x == 0) { s_prefix = 0u; s_mask = 0u; s_kr = (uint32_t)k; s_done = 0; }
-  __syncthreads();
 
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += NT) s_hist[i] = 0u;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const uint32_t dmask = pass == 2 ? 0xFFu : 0xFFFu;
+    for (int i = threadIdx.x; i < kTopkBins; i += NT) s_hist[i] = 0u;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
     for (int i = threadIdx.x; i < n; i += NT) {
       const uint32_t key = cached ? s_keys[i] : score_key(__ldg(src + i));
-      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & dmask], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-      // Lane l owns bins [248-8l, 255-8l]; find the bin (scanning from the top)
-      // where the running count first reaches the remaining rank kr.
-      const int lane = threadIdx.x;
-      const uint32_t kr = s_kr;
-      uint32_t cnt[8], sum = 0;
+    // Thread t owns bins [4095-8t-7, 4095-8t] (descending); a block scan of the
+    // per-thread sums locates the bin where the count from the top reaches kr.
+    const uint32_t kr = s_kr;
+    uint32_t cnt[8], sum = 0;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) { cnt[q] = s_hist[255 - 8 * lane - q]; sum += cnt[q]; }
-      uint32_t incl = sum;
+    for (int q = 0; q < 8; ++q) { cnt[q] = s_hist[kTopkBins - 1 - 8 * threadIdx.x - q]; sum += cnt[q]; }
+    const uint32_t excl = block_excl_scan<NT>(sum, s_warp, &s_total);
+    if (excl < kr && excl + sum >= kr) {             // exactly one thread
+      uint32_t c = excl;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t excl = incl - sum;
-      const unsigned ballot = __ballot_sync(0xffffffffu, incl >= kr);
-      const int owner = __ffs(ballot) - 1;            // first lane whose range reaches kr
-      if (lane == owner) {
-        uint32_t c = excl;
-        int bin = 0;
-        uint32_t before = 0, inbin = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (c + cnt[q] >= kr) { bin = 255 - 8 * lane - q; before = c; inbin = cnt[q]; break; }
-          c += cnt[q];
+      for (int q = 0; q < 8; ++q) {
+        if (c + cnt[q] >= kr) {
+          const uint32_t bin = (uint32_t)(kTopkBins - 1 - 8 * threadIdx.x - q);
+          const uint32_t krem = kr - c;
+          s_prefix = prefix | (bin << shift);
+          s_mask = mask | (dmask << shift);
+          s_kr = krem;
+          s_done = (krem == cnt[q]) ? 1 : 0;       // whole bucket taken: no need to refine
+          break;
         }
-        const uint32_t krem = kr - before;
-        s_prefix = prefix | ((uint32_t)bin << shift);
-        s_mask = mask | (255u << shift);
-        s_kr = krem;
-        s_done = (krem == inbin) ? 1 : 0;           // whole bucket taken: no need to refine
+        c += cnt[q];
       }
     }
     __syncthreads();

@@ -155,6 +155,7 @@ def _sink(x):
     ("bf16", 64, 512, 64, 4, 128, 2048, 9, 3000, 9000, True),  # full k
     ("bf16", 64, 512, 64, 4, 100, 100, 20, 900, 3000, True),   # odd W and k
     ("bf16", 64, 512, 64, 4, 128, 256, 160, 700, 2700, True),  # >= 296 rows: no key-range split
+    ("bf16", 64, 512, 64, 4, 128, 3000, 4, 5000, 19000, True), # k > 2048: forced key-range splits
 ])
 def test_csa_sparse_attn_parity(lcsa, dtype, H, D, R, m, W, k, Tq, Nc, q_pos0, unit):
     B = 2

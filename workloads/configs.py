@@ -45,6 +45,8 @@ CONFIGS = {
     "tiny": WorkloadConfig(name="tiny", dtype="fp32", B=1, T=1024, H=4, D=64, R=32,
                            H_I=2, D_I=32, m=4, m_hca=128, k=64, W=64, seed=0,
                            gate_scale_by_dim=True),
+    # Small CSA layer (profiling-sized case of the prefill kernels).
+    "csa_prefill_8k": WorkloadConfig(name="csa_prefill_8k", dtype="bf16", B=1, T=8192, seed=6),
     # CSA layer prefill, T=32768.
     "csa_prefill_32k": WorkloadConfig(name="csa_prefill_32k", dtype="bf16", B=1, T=32768, seed=1),
     # HCA layer prefill, T=131072 (1024 entries).
