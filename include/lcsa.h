@@ -151,6 +151,30 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace,
 int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a);
 
 /* ------------------------------------------------------------------------
+ * Indexer + top-k without a caller workspace.  The pages have no counterpart
+ * to this call: it exists for callers that cannot allocate device memory when
+ * they call the library (an allocator or arena they do not own, a runtime
+ * that forbids allocation after start-up, a thread that must not let
+ * cudaMalloc/cudaFree synchronise the device).
+ *
+ * Same arguments and results as lcsa_indexer_topk, minus the workspace.  The
+ * score workspace is a fixed 32 MiB array inside the library's device image,
+ * held by every GPU that loads the library until the process exits; large
+ * problems are processed in row chunks that fit it.  Nothing is allocated and
+ * nothing needs clearing (each chunk writes the scratch it reads).
+ *   - Returns LCSA_ERR_WORKSPACE when a single score row does not fit, i.e.
+ *     when Nc * 4 bytes (rounded up to 256) + 256 exceeds 32 MiB
+ *     (Nc > 8,388,544).
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before capturing any stream into a CUDA graph.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (different streams, or concurrent host threads without ordering)
+ *     race on it.  Order them on one stream.
+ * ------------------------------------------------------------------------ */
+lcsa_status lcsa_indexer_topk_noalloc(const lcsa_indexer_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
  * Core attention ([p3] "第三步，core attention"; [p3] the sentence on running
  * multi-query attention over the selected blocks (CSA) and the HCA sentence on
  * dense attention over all compressed KV; [p2] "Sliding Window Branch": the

@@ -29,6 +29,7 @@ EXPORTED = [
     "lcsa_csa_compress", "lcsa_hca_compress",
     "lcsa_topk_workspace", "lcsa_topk_from_scores",
     "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
+    "lcsa_indexer_topk_noalloc",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
 ]
 
@@ -73,6 +74,7 @@ _sig = {
     "lcsa_indexer_topk_workspace": (_sz, [ctypes.POINTER(IndexerArgs)]),
     "lcsa_indexer_topk": (_i, [ctypes.POINTER(IndexerArgs), _vp, _sz, _vp]),
     "lcsa_indexer_uses_tensor_cores": (_i, [ctypes.POINTER(IndexerArgs)]),
+    "lcsa_indexer_topk_noalloc": (_i, [ctypes.POINTER(IndexerArgs), _vp]),
     "lcsa_attn_workspace": (_sz, [ctypes.POINTER(AttnArgs), _i]),
     "lcsa_csa_sparse_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),

@@ -2,8 +2,8 @@
 
     python -m long_context_compressed_softmax_b200.build [--verbose]
 
-Compiles csrc/lcsa.cu (the single translation unit that includes every
-kernel) with nvcc for sm_100a and writes liblcsa.so next to this file.
+Compiles csrc/lcsa.cu (the translation unit that includes every kernel) and
+csrc/noalloc.cu with nvcc for sm_100a and writes liblcsa.so next to this file.
 """
 import os
 import shutil
@@ -41,7 +41,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return OUT
     nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
     tmp = OUT + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, os.path.join(SRC, "lcsa.cu")]
+    units = [os.path.join(SRC, "lcsa.cu"), os.path.join(SRC, "noalloc.cu")]
+    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, *units]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
