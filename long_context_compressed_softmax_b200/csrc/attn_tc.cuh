@@ -27,7 +27,11 @@
 namespace lcsa {
 
 constexpr int kAtKT = 64;                      // keys per tile
-constexpr int kAtThreads = 288;
+constexpr int kAtProdWarps = 8;                 // gather / TMA producers
+constexpr int kAtProdThreads = kAtProdWarps * 32;
+constexpr int kAtMmaWarp = kAtProdWarps;        // TMEM allocator and MMA issuer
+constexpr int kAtSmWarp0 = kAtProdWarps + 1;    // first of the 4 softmax / epilogue warps
+constexpr int kAtThreads = (kAtProdWarps + 5) * 32;
 constexpr uint32_t kAtQBytes = 64 * 512 * 2;   // 64 KB
 constexpr uint32_t kAtKBytes = kAtKT * 512 * 2;  // 64 KB
 constexpr uint32_t kAtPBytes = 64 * kAtKT * 2;   // 8 KB
@@ -35,7 +39,7 @@ constexpr uint32_t kAtRegion = 64 * 128;       // one 64-dim column block of a 6
 constexpr int kAtMaxIdx = 2048;                 // selected entries staged in shared memory per CTA
 constexpr int kAtStages = 3;                    // K=V tile stages
 constexpr size_t kAtSmem = 1024 + kAtStages * kAtKBytes + 2 * kAtPBytes + kAtStages * kAtKT * 2 * 8 +
-                           kAtMaxIdx * 4 + 32 * 8 + 16 * 8;
+                           kAtMaxIdx * 4 + 32 * 8 + 17 * 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AtGeom {
@@ -114,7 +118,9 @@ __device__ __forceinline__ KeySet key_set(const AtGeom& g, const int32_t* idx_ro
   return s;
 }
 
-__global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom g) {
+__global__ void __launch_bounds__(kAtThreads, 1)
+attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, const __grid_constant__ CUtensorMap tm_kv,
+               const __grid_constant__ CUtensorMap tm_rotc, const __grid_constant__ CUtensorMap tm_rotw) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_k = smem;                                                  // kAtStages K=V tiles
@@ -124,7 +130,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
   float2* s_cs = reinterpret_cast<float2*>(s_idx + kAtMaxIdx);                      // [32] (cos, sin) at t
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_cs + 32);
   uint64_t* q_ready = bars + 0;                 // softmax warps (4): Q is in TMEM
-  uint64_t* kv_full = bars + 1;                 // [kAtStages] producers (128, async arrivals)
+  uint64_t* q_full = bars + 15;                 // producers (async arrivals): Q staged in the last stage
+  uint64_t* kv_full = bars + 1;                 // [kAtStages] producers (one arrival each; TMA bytes)
   uint64_t* kv_empty = kv_full + kAtStages;     // [kAtStages] MMA commit
   uint64_t* s_full = kv_empty + kAtStages;      // [2] MMA commit
   uint64_t* s_free = s_full + 2;                // [2] softmax warps (4)
@@ -167,8 +174,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_ready, 4);
+    tc::mbar_init(q_full, kAtProdThreads);
     for (int s = 0; s < kAtStages; ++s) {
-      tc::mbar_init(kv_full + s, 128);
+      tc::mbar_init(kv_full + s, kAtProdThreads);
       tc::mbar_init(kv_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -180,7 +188,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
     tc::fence_barrier_init();
     s_abort = 0;
   }
-  if (warp == 4) { tc::tmem_alloc(&s_tmem, 512); tc::tmem_relinquish(); }
+  if (warp == kAtMmaWarp) { tc::tmem_alloc(&s_tmem, 512); tc::tmem_relinquish(); }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -192,58 +200,96 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
   constexpr uint32_t kTmQ = 128;
   constexpr uint32_t kTmO = 16u << 16;
 
-  if (warp < 4) {
+  if (warp < kAtProdWarps) {
     // ============================================================ producers
-    const int tid = threadIdx.x;                    // 0..127
+    // Contiguous tiles (every HCA entry tile and every window tile) arrive as
+    // eight 2D TMA boxes of 64 rows x 64 dims; CSA's selected rows are
+    // gathered 16 bytes at a time with cp.async by all eight producer warps.
+    const int tid = threadIdx.x;                    // 0..255
     const int piece = tid & 63;                     // 16-byte piece of a 1 KB row
     const int region = piece >> 3, c16 = piece & 7;
-    const int kk0 = tid >> 6;                       // keys kk0, kk0+2, ..., kk0+62
+    const int kk0 = tid >> 6;                       // keys kk0, kk0+4, ..., kk0+60
+    constexpr int kStep = kAtProdThreads / 64;
+    // Q (64 heads x 1 KB) is staged in the last K stage, which tile 2 only
+    // reuses once the softmax warps have moved Q into tensor memory.
+    {
+      const uint8_t* qrow0 = reinterpret_cast<const uint8_t*>(P.q + row * 64 * 512);
+      const uint32_t qb = tc::smem_u32(s_k + (kAtStages - 1) * kAtKBytes) + region * kAtRegion + (c16 << 4);
+#pragma unroll 8
+      for (int u = 0; u < 64 / kStep; ++u) {
+        const int h = kk0 + kStep * u;
+        cp_async16((qb + h * 128) ^ ((uint32_t)(h & 7) << 4), qrow0 + (long long)h * 1024 + piece * 16, 16);
+      }
+      cp_async_arrive_noinc(q_full);
+    }
     const int slot0 = t0 * kAtKT;
     if (g.sparse) {
       const int n_sel = (ks.n_c < t1 * kAtKT ? ks.n_c : t1 * kAtKT) - slot0;
-      for (int e = tid; e < n_sel; e += 128) s_idx[e] = idx_row[slot0 + e];
-      named_bar(1, 128);
+      for (int e = tid; e < n_sel; e += kAtProdThreads) s_idx[e] = idx_row[slot0 + e];
+      named_bar(1, kAtProdThreads);
+    }
+    if (tid == 0) {
+      tc::prefetch_tmap(&tm_ckv);
+      tc::prefetch_tmap(&tm_kv);
+      tc::prefetch_tmap(&tm_rotc);
+      tc::prefetch_tmap(&tm_rotw);
     }
     const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.q);
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % kAtStages;
       if (n >= kAtStages && !tc::mbar_wait_backoff(kv_empty + s, ((n - kAtStages) / kAtStages) & 1)) *abort_flag = 1;
+      if (n == kAtStages - 1 && !tc::mbar_wait_backoff(q_ready, 0)) *abort_flag = 1;
       if (*abort_flag) break;
       const int gt = t0 + n;                        // tile index in the query's key list
+      uint8_t* stage = s_k + s * kAtKBytes;
+      if (gt >= ks.tiles_c || !g.sparse) {
+        // ---- contiguous rows: TMA boxes
+        if (tid == 0) {
+          const CUtensorMap* mm;
+          const CUtensorMap* mr;
+          int y;
+          if (gt < ks.tiles_c) {
+            mm = &tm_ckv; mr = &tm_rotc;
+            y = (int)((long long)b * g.Nc + (long long)gt * kAtKT);
+          } else {
+            mm = &tm_kv; mr = &tm_rotw;
+            y = (int)((long long)b * g.Tkv + (ks.wlo - g.kv_pos0) + (long long)(gt - ks.tiles_c) * kAtKT);
+          }
+          tc::mbar_arrive_expect_tx(kv_full + s, kAtKBytes);
+#pragma unroll
+          for (int reg = 0; reg < 7; ++reg) tc::tma_load_2d(stage + reg * kAtRegion, mm, kv_full + s, reg * 64, y);
+          tc::tma_load_2d(stage + 7 * kAtRegion, mr, kv_full + s, 0, y);
+        } else {
+          tc::mbar_arrive(kv_full + s);
+        }
+        continue;
+      }
+      // ---- gathered rows (CSA): per-tile row table, then 16-byte cp.async pieces
       const uint8_t** tab = s_tab + s * kAtKT * 2;
       if (tid < kAtKT) {
         const int kk = tid;
         const uint8_t* rm = nullptr;
         const uint8_t* rr = nullptr;
-        if (gt < ks.tiles_c) {
-          const int slot = gt * kAtKT + kk;
-          if (slot < ks.n_c) {
-            const int j = g.sparse ? s_idx[slot - slot0] : slot;
-            if (j >= 0 && j < g.Nc) {
-              rm = reinterpret_cast<const uint8_t*>(P.ckv + ((long long)b * g.Nc + j) * 512);
-              rr = reinterpret_cast<const uint8_t*>(
-                  P.rot_c + (g.rot_slot ? (row * g.k + slot) : ((long long)b * g.Nc + j)) * 64);
-            } else {
-              report(LCSA_DEV_BAD_INDEX);
-            }
-          }
-        } else {
-          const int w = (gt - ks.tiles_c) * kAtKT + kk;
-          if (w < ks.n_w) {
-            const long long r = ks.wlo + w - g.kv_pos0;
-            rm = reinterpret_cast<const uint8_t*>(P.kv + ((long long)b * g.Tkv + r) * 512);
-            rr = reinterpret_cast<const uint8_t*>(P.rot_w + ((long long)b * g.Tkv + r) * 64);
+        const int slot = gt * kAtKT + kk;
+        if (slot < ks.n_c) {
+          const int j = s_idx[slot - slot0];
+          if (j >= 0 && j < g.Nc) {
+            rm = reinterpret_cast<const uint8_t*>(P.ckv + ((long long)b * g.Nc + j) * 512);
+            rr = reinterpret_cast<const uint8_t*>(
+                P.rot_c + (g.rot_slot ? (row * g.k + slot) : ((long long)b * g.Nc + j)) * 64);
+          } else {
+            report(LCSA_DEV_BAD_INDEX);
           }
         }
         tab[2 * kk] = rm;
         tab[2 * kk + 1] = rr;
       }
-      named_bar(1, 128);
-      const uint32_t kb = tc::smem_u32(s_k + s * kAtKBytes) + region * kAtRegion + (c16 << 4);
+      named_bar(1, kAtProdThreads);
+      const uint32_t kb = tc::smem_u32(stage) + region * kAtRegion + (c16 << 4);
       const int off = region == 7 ? c16 * 16 : piece * 16;
 #pragma unroll 8
-      for (int u = 0; u < 32; ++u) {
-        const int kk = kk0 + 2 * u;
+      for (int u = 0; u < 64 / kStep; ++u) {
+        const int kk = kk0 + kStep * u;
         const uint8_t* base = tab[2 * kk + (region == 7 ? 1 : 0)];
         const uint32_t dst = (kb + kk * 128) ^ ((uint32_t)(kk & 7) << 4);
         cp_async16(dst, base ? base + off : dummy, base ? 16u : 0u);
@@ -251,7 +297,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
       cp_async_arrive_noinc(kv_full + s);
     }
     cp_async_wait_all();                            // nothing may land after the CTA exits
-  } else if (warp == 4) {
+  } else if (warp == kAtMmaWarp) {
     // ============================================================ MMA issuer
     // S(n+1) and PV(n) are independent: whichever is ready is issued first.
     if (tc::elect_one()) {
@@ -318,7 +364,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
     const bool s_owner = lane < 16;                   // lanes 0-15: S rows; lanes 16-31: O rows
     const int h = quarter * 16 + (lane & 15);         // head row this thread owns
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int stid = threadIdx.x - 5 * 32;            // 0..127
+    const int stid = threadIdx.x - kAtSmWarp0 * 32;   // 0..127
     // rotary table at position t (shared by the Q rotation and the -t output rotation)
     if (stid < 32) {
       float c, sn;
@@ -328,15 +374,17 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
     named_bar(2, 128);
     // Q -> TMEM (A operand): lane h holds head h's 512 dims, two per column; the
     // rotary block (dims 448..511) is rotated at t on the way.
+    if (!tc::mbar_wait(q_full, 0)) *abort_flag = 1;
     {
-      const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row * 64 + h) * 512);
-#pragma unroll 1
+      const uint8_t* qs = s_k + (kAtStages - 1) * kAtKBytes + h * 128;
+#pragma unroll 2
       for (int c = 0; c < 16; ++c) {                  // 32 dims = 16 columns per step
         uint32_t r[16];
         if (s_owner) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const uint4 x = __ldg(qrow + 4 * c + v);
+            const int chunk = (c & 1) * 4 + v;        // 16-byte chunk within the 128-byte row of region c/2
+            const uint4 x = *reinterpret_cast<const uint4*>(qs + (c >> 1) * kAtRegion + ((chunk ^ (h & 7)) << 4));
             r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
           }
           if (c >= 14) {
@@ -503,7 +551,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(AtPtrs P, AtGeom
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kAtMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 512);
   }
@@ -641,8 +689,21 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   g.out_bf16 = a->out_dtype == LCSA_BF16;
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
   if (e != cudaSuccess) return e;
+  // Tensor maps for the contiguous tiles (64 rows x 64 dims, 128-byte swizzle).
+  // A map whose tensor is absent is never read; it points at q instead.
+  CUtensorMap m_ckv, m_kv, m_rotc, m_rotw;
+  const uint64_t rows_rotc = pl.rot_slot ? (uint64_t)rows * a->k : (uint64_t)a->B * a->Nc;
+  auto mk = [&](CUtensorMap* m, const void* base, uint64_t nrows, uint64_t cols) {
+    if (base == nullptr || nrows == 0) return make_tmap_bf16_2d(m, a->q, (uint64_t)rows * 64, 512, 512, 64, 64);
+    return make_tmap_bf16_2d(m, base, nrows, cols, cols, 64, 64);
+  };
+  if (!mk(&m_ckv, a->Nc > 0 ? a->ckv : nullptr, (uint64_t)a->B * a->Nc, 512) ||
+      !mk(&m_kv, a->Tkv > 0 ? a->kv : nullptr, (uint64_t)a->B * a->Tkv, 512) ||
+      !mk(&m_rotc, a->Nc > 0 ? (const void*)P.rot_c : nullptr, rows_rotc, 64) ||
+      !mk(&m_rotw, (a->Tkv > 0 && a->W > 0) ? (const void*)P.rot_w : nullptr, (uint64_t)a->B * a->Tkv, 64))
+    return cudaErrorInvalidValue;
   dim3 grid((unsigned)rows, pl.splits);
-  attn_tc_kernel<<<grid, kAtThreads, kAtSmem, st>>>(P, g);
+  attn_tc_kernel<<<grid, kAtThreads, kAtSmem, st>>>(P, g, m_ckv, m_kv, m_rotc, m_rotw);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
