@@ -2,16 +2,21 @@
 // (DeepSeek-V4 CSA Step 2: keep the top-k indexer scores; ties to the lower
 // index; indices emitted ascending, -1 padded.)
 //
-// One CTA per row.  Scores map to 32-bit keys whose unsigned order is the
-// float order (-0 folded onto +0).  Three MSB-first histogram passes over
-// 12, 12 and 8 key bits (4096-bin shared-memory histograms: a score's sign,
-// exponent and top mantissa bits land in distinct bins, which keeps
-// same-address atomics rare) find the k-th largest key K and how many of its
-// ties to keep; a pass stops early once the threshold bucket is taken whole.
-// A last pass in index order writes every key > K plus the first r ties, with
-// output slots from a block-wide prefix count, so the list comes out
-// ascending.  Rows up to kMaxCachedKeys are staged in shared memory once;
-// longer rows are re-read from L2 on every pass.
+// One CTA (16 warps) per row; the row is split into 16 contiguous warp
+// segments.  Scores map to 32-bit keys whose unsigned order is the float
+// order (-0 folded onto +0).
+//   1. A 4096-bin histogram of the keys' top 12 bits (sign, exponent, three
+//      mantissa bits) gives the bin holding the k-th largest key.
+//   2. One sweep counts, per warp segment, the keys above that bin and
+//      compacts the bin's (key, index) pairs into a candidate list.
+//   3. The exact threshold key and the number of its ties to keep are found
+//      on the candidates alone (12- and 8-bit histograms); a bin too full for
+//      the list falls back to the same histograms over the whole row.
+//   4. Each warp emits its segment in index order with ballots: every key
+//      above the threshold plus the first r ties, at slots given by per-warp
+//      prefix counts, so the list comes out ascending without block scans.
+// Rows up to kMaxCachedKeys are staged in shared memory during pass 1;
+// longer rows are re-read from L2 in each pass.
 #pragma once
 #include "common.cuh"
 
@@ -20,6 +25,7 @@ namespace lcsa {
 constexpr int kTopkThreads = 512;
 constexpr int kMaxCachedKeys = 32768;   // 128 KiB of dynamic shared memory
 constexpr int kTopkBins = 4096;
+constexpr int kTopkCand = 2048;         // candidate list capacity
 
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -27,7 +33,7 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan (NT threads); also returns the block total.
+// Exclusive block scan (NT threads); *total receives the block sum.
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -54,20 +60,108 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return s_warp[warp] + x - v;
 }
 
+struct TopkState {
+  uint32_t prefix, mask, kr;
+  int done;
+};
+
+// In a histogram of `nbins` (4096 or 256) bins scanned from the top, find the
+// bin where the running count reaches st->kr and refine *st to it.  All NT
+// threads call this; it ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void topk_pick_bin(const uint32_t* hist, int nbins, int shift, uint32_t dmask,
+                                              TopkState* st, uint32_t* s_warp, uint32_t* s_total,
+                                              uint32_t* s_bincnt) {
+  const uint32_t kr = st->kr;
+  const int per = nbins / NT;                        // 8 bins per thread, or 0 (one bin for the first nbins threads)
+  uint32_t cnt[8], sum = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    int bin = -1;
+    if (per > 0) bin = q < per ? nbins - 1 - per * (int)threadIdx.x - q : -1;
+    else bin = (q == 0 && (int)threadIdx.x < nbins) ? nbins - 1 - (int)threadIdx.x : -1;
+    cnt[q] = bin >= 0 ? hist[bin] : 0u;
+    sum += cnt[q];
+  }
+  const uint32_t excl = block_excl_scan<NT>(sum, s_warp, s_total);
+  if (excl < kr && excl + sum >= kr) {               // exactly one thread
+    uint32_t c = excl;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (c + cnt[q] >= kr) {
+        const int bin = per > 0 ? nbins - 1 - per * (int)threadIdx.x - q : nbins - 1 - (int)threadIdx.x;
+        st->prefix |= (uint32_t)bin << shift;
+        st->mask |= dmask << shift;
+        st->kr = kr - c;
+        st->done = (kr - c == cnt[q]) ? 1 : 0;       // the whole bin is taken: no need to refine
+        *s_bincnt = cnt[q];
+        break;
+      }
+      c += cnt[q];
+    }
+  }
+  __syncthreads();
+}
+
+// Visit every key of [lo, hi) (a warp segment) in index order per lane:
+// lane L handles elements base+4L .. base+4L+3 of each 128-element step, and
+// kUnroll steps are loaded before any is used, so a thread keeps 4*kUnroll
+// scores in flight.  f(i, key, valid) is called for all 4*kUnroll slots of a
+// group; vec4 requires src 16-byte aligned and lo % 4 == 0.
+constexpr int kUnroll = 4;
+template <typename F>
+__device__ __forceinline__ void segment_visit(const float* __restrict__ src, const uint32_t* keys, bool cached,
+                                              bool vec4, int lo, int hi, F&& f) {
+  const int lane = threadIdx.x & 31;
+  for (int base = lo; base < hi; base += 128 * kUnroll) {
+    uint32_t kk[kUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i0 = base + u * 128 + 4 * lane;
+      if (vec4 && i0 + 3 < hi) {
+        if (cached) {
+          const uint4 v = *reinterpret_cast<const uint4*>(keys + i0);
+          kk[u][0] = v.x; kk[u][1] = v.y; kk[u][2] = v.z; kk[u][3] = v.w;
+        } else {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(src + i0));
+          kk[u][0] = score_key(v.x); kk[u][1] = score_key(v.y); kk[u][2] = score_key(v.z); kk[u][3] = score_key(v.w);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = i0 + q;
+          kk[u][q] = i < hi ? (cached ? keys[i] : score_key(__ldg(src + i))) : 0u;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = base + u * 128 + 4 * lane + q;
+        f(u, i, kk[u][q], i < hi);
+      }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT)
 topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
                  const int32_t* __restrict__ n_valid, int k, int32_t* __restrict__ idx_out,
                  int cache_cap) {
   static_assert(kTopkBins == 8 * NT, "each thread owns 8 bins");
+  constexpr int W = NT / 32;
   extern __shared__ uint32_t s_keys[];
   __shared__ uint32_t s_hist[kTopkBins];
+  __shared__ uint32_t s_ckey[kTopkCand];
+  __shared__ int32_t s_cidx[kTopkCand];
   __shared__ uint32_t s_warp[32];
-  __shared__ uint32_t s_total;
-  __shared__ uint32_t s_prefix, s_mask, s_kr;
-  __shared__ int s_done;
+  __shared__ uint32_t s_total, s_bincnt, s_ncand;
+  __shared__ uint32_t s_above[W], s_eq[W];           // per-warp-segment counts
+  __shared__ TopkState s_st;
 
   const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int n = n_cols;
   if (n_valid != nullptr) {
     n = n_valid[row];
@@ -81,71 +175,135 @@ topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
     return;
   }
   const bool cached = n <= cache_cap;
-  if (cached)
-    for (int i = threadIdx.x; i < n; i += NT) s_keys[i] = score_key(__ldg(src + i));
-  if (threadIdx.x == 0) { s_prefix = 0u; s_mask = 0u; s_kr = (uint32_t)k; s_done = 0; }
+  const bool vec4 = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+  // contiguous warp segments [seg_lo, seg_hi), lengths multiples of 128
+  const int seg_len = ((n + W - 1) / W + 127) & ~127;
+  const int seg_lo = warp * seg_len < n ? warp * seg_len : n;
+  const int seg_hi = seg_lo + seg_len < n ? seg_lo + seg_len : n;
 
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
-    const uint32_t dmask = pass == 2 ? 0xFFu : 0xFFFu;
-    for (int i = threadIdx.x; i < kTopkBins; i += NT) s_hist[i] = 0u;
-    __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int i = threadIdx.x; i < n; i += NT) {
-      const uint32_t key = cached ? s_keys[i] : score_key(__ldg(src + i));
-      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & dmask], 1u);
+  for (int i = threadIdx.x; i < kTopkBins; i += NT) s_hist[i] = 0u;
+  if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = (uint32_t)k; s_st.done = 0; s_ncand = 0u; }
+  if (threadIdx.x < W) { s_above[threadIdx.x] = 0u; s_eq[threadIdx.x] = 0u; }
+  __syncthreads();
+
+  // ---- pass 1: top-12-bit histogram (stages the row in shared memory)
+  segment_visit(src, s_keys, false, vec4, seg_lo, seg_hi, [&](int, int i, uint32_t key, bool valid) {
+    if (valid) {
+      if (cached) s_keys[i] = key;
+      atomicAdd(&s_hist[key >> 20], 1u);
     }
-    __syncthreads();
-    // Thread t owns bins [4095-8t-7, 4095-8t] (descending); a block scan of the
-    // per-thread sums locates the bin where the count from the top reaches kr.
-    const uint32_t kr = s_kr;
-    uint32_t cnt[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) { cnt[q] = s_hist[kTopkBins - 1 - 8 * threadIdx.x - q]; sum += cnt[q]; }
-    const uint32_t excl = block_excl_scan<NT>(sum, s_warp, &s_total);
-    if (excl < kr && excl + sum >= kr) {             // exactly one thread
-      uint32_t c = excl;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (c + cnt[q] >= kr) {
-          const uint32_t bin = (uint32_t)(kTopkBins - 1 - 8 * threadIdx.x - q);
-          const uint32_t krem = kr - c;
-          s_prefix = prefix | (bin << shift);
-          s_mask = mask | (dmask << shift);
-          s_kr = krem;
-          s_done = (krem == cnt[q]) ? 1 : 0;       // whole bucket taken: no need to refine
-          break;
-        }
-        c += cnt[q];
+  });
+  __syncthreads();
+  topk_pick_bin<NT>(s_hist, kTopkBins, 20, 0xFFFu, &s_st, s_warp, &s_total, &s_bincnt);
+  const uint32_t prefix1 = s_st.prefix, mask1 = s_st.mask;
+  const bool fits = s_bincnt <= (uint32_t)kTopkCand;
+
+  // ---- pass 2: per-segment counts above the bin; compact the bin's candidates
+  {
+    uint32_t above = 0;
+    segment_visit(src, s_keys, cached, vec4, seg_lo, seg_hi, [&](int, int i, uint32_t key, bool valid) {
+      if (!valid) return;
+      const uint32_t mk = key & mask1;
+      above += mk > prefix1;
+      if (fits && mk == prefix1) {
+        const uint32_t slot = atomicAdd(&s_ncand, 1u);
+        s_ckey[slot] = key;
+        s_cidx[slot] = i;
       }
+    });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    if (lane == 0) s_above[warp] = above;
+  }
+  __syncthreads();
+
+  // ---- resolve the exact threshold: on the candidates, or over the whole row
+  const int ncand = fits ? (int)s_ncand : 0;
+  for (int level = 0; level < 2; ++level) {
+    if (s_st.done) break;                             // uniform: read after a barrier
+    const int shift = level == 0 ? 8 : 0;
+    const uint32_t dmask = level == 0 ? 0xFFFu : 0xFFu;
+    const int nbins = level == 0 ? kTopkBins : 256;
+    for (int i = threadIdx.x; i < nbins; i += NT) s_hist[i] = 0u;
+    __syncthreads();
+    const uint32_t prefix = s_st.prefix, mask = s_st.mask;
+    if (fits) {
+      for (int c = threadIdx.x; c < ncand; c += NT) {
+        const uint32_t key = s_ckey[c];
+        if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & dmask], 1u);
+      }
+    } else {
+      segment_visit(src, s_keys, cached, vec4, seg_lo, seg_hi, [&](int, int, uint32_t key, bool valid) {
+        if (valid && (key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & dmask], 1u);
+      });
     }
     __syncthreads();
-    if (s_done) break;
+    topk_pick_bin<NT>(s_hist, nbins, shift, dmask, &s_st, s_warp, &s_total, &s_bincnt);
   }
+  const uint32_t prefix = s_st.prefix, mask = s_st.mask, kr = s_st.kr;
 
-  // Index-order emission: keys above the bucket, plus the first kr of its ties.
-  const uint32_t prefix = s_prefix, mask = s_mask, kr = s_kr;
-  uint32_t gt_before = 0, eq_before = 0;
-  for (int base = 0; base < n; base += NT) {
-    const int i = base + threadIdx.x;
-    uint32_t a = 0, e = 0;
-    if (i < n) {
-      const uint32_t key = (cached ? s_keys[i] : score_key(__ldg(src + i))) & mask;
-      a = key > prefix;
-      e = key == prefix;
+  // ---- per-segment counts of the threshold bin's keys above / equal to it
+  if (fits) {
+    for (int c = threadIdx.x; c < ncand; c += NT) {
+      const uint32_t key = s_ckey[c] & mask;
+      const int w = s_cidx[c] / seg_len;
+      if (key > prefix) atomicAdd(&s_above[w], 1u);
+      else if (key == prefix) atomicAdd(&s_eq[w], 1u);
     }
-    const uint32_t ex = block_excl_scan<NT>(a | (e << 16), s_warp, &s_total);
-    const uint32_t pa = ex & 0xffffu, pe = ex >> 16;
-    if (a) {
-      const uint32_t eqb = eq_before + pe;
-      dst[gt_before + pa + (eqb < kr ? eqb : kr)] = i;
-    } else if (e && eq_before + pe < kr) {
-      dst[gt_before + pa + eq_before + pe] = i;
+  } else {
+    uint32_t above = 0, eq = 0;
+    segment_visit(src, s_keys, cached, vec4, seg_lo, seg_hi, [&](int, int, uint32_t key, bool valid) {
+      if (valid && (key & mask1) == prefix1) {
+        const uint32_t mk = key & mask;
+        above += mk > prefix;
+        eq += mk == prefix;
+      }
+    });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      above += __shfl_xor_sync(0xffffffffu, above, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
     }
-    const uint32_t tot = s_total;
-    gt_before += tot & 0xffffu;
-    eq_before += tot >> 16;
-    __syncthreads();                                   // s_warp / s_total reuse
+    if (lane == 0) { s_above[warp] += above; s_eq[warp] = eq; }
+  }
+  __syncthreads();
+
+  // ---- emission: every warp walks its own segment in index order; within a
+  // 128-element step lane L owns elements 4L..4L+3, so a warp scan of the
+  // per-lane counts gives each lane its running position.
+  uint32_t run_a = 0, run_e = 0;
+  for (int w = 0; w < warp; ++w) { run_a += s_above[w]; run_e += s_eq[w]; }
+  {
+    uint32_t fa[kUnroll], fe[kUnroll];              // per step: bit q set if element q is above / a tie
+    segment_visit(src, s_keys, cached, vec4, seg_lo, seg_hi, [&](int u, int i, uint32_t key, bool valid) {
+      const int q = i & 3;
+      if (q == 0) { fa[u] = 0u; fe[u] = 0u; }
+      if (valid) {
+        const uint32_t mk = key & mask;
+        fa[u] |= (uint32_t)(mk > prefix) << q;
+        fe[u] |= (uint32_t)(mk == prefix) << q;
+      }
+      if (q == 3) {
+        // packed counts (a in the low half, e in the high half) of this lane's four elements
+        const uint32_t mine = __popc(fa[u]) | (__popc(fe[u]) << 16);
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t ga = run_a + ((incl - mine) & 0xffffu), ge = run_e + ((incl - mine) >> 16);
+        const int i0 = i - 3;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          if ((fa[u] >> qq) & 1u) { dst[ga + (ge < kr ? ge : kr)] = i0 + qq; ++ga; }
+          else if ((fe[u] >> qq) & 1u) { if (ge < kr) dst[ga + ge] = i0 + qq; ++ge; }
+        }
+        run_a += tot & 0xffffu;
+        run_e += tot >> 16;
+      }
+    });
   }
 }
 

@@ -66,9 +66,11 @@ def test_compress_short_sequence(lcsa):
 
 # ------------------------------------------------------------------ top-k
 @pytest.mark.parametrize("n_cols,k,ties", [(64, 8, 0), (1000, 64, 4), (8191, 2048, 0), (8191, 2048, 16),
-                                          (40000, 2048, 0), (5000, 1, 3), (300, 2048, 0)])
+                                          (40000, 2048, 0), (5000, 1, 3), (300, 2048, 0),
+                                          (32768, 2048, 0), (262144, 2048, 0),   # cached / uncached rows
+                                          (40000, 2048, 1), (262144, 2048, 2)])  # threshold bin > candidate list
 def test_topk_bitexact(lcsa, n_cols, k, ties):
-    rows = 37
+    rows = 37 if n_cols < 100000 else 6
     s = gen.make_scores(rows, n_cols, seed=31 + n_cols, device=DEV, tie_levels=ties)
     g = torch.Generator(device="cpu").manual_seed(7)
     nv = torch.randint(0, n_cols + 1, (rows,), generator=g, dtype=torch.int32)
