@@ -360,9 +360,13 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, c
     }
   } else {
     // ============================================================ softmax / epilogue
+    // Every head row h of this warp's 16-lane block is split over two threads:
+    // thread (h % 16) takes keys 0-31 of each tile and dims 0-255 of O,
+    // thread (h % 16) + 16 takes keys 32-63 and dims 256-511 (16x32bx2 TMEM
+    // accesses).  Row maxima and sums meet through one shuffle.
     const int quarter = warp & 3;
-    const bool s_owner = lane < 16;                   // lanes 0-15: S rows; lanes 16-31: O rows
-    const int h = quarter * 16 + (lane & 15);         // head row this thread owns
+    const int half = lane >> 4;                       // 0: keys 0-31 / dims 0-255, 1: keys 32-63 / dims 256-511
+    const int h = quarter * 16 + (lane & 15);         // head row
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int stid = threadIdx.x - kAtSmWarp0 * 32;   // 0..127
     // rotary table at position t (shared by the Q rotation and the -t output rotation)
@@ -372,35 +376,31 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, c
       s_cs[stid] = make_float2(c, sn);
     }
     named_bar(2, 128);
-    // Q -> TMEM (A operand): lane h holds head h's 512 dims, two per column; the
-    // rotary block (dims 448..511) is rotated at t on the way.
+    // Q -> TMEM (A operand, lanes 0-15): head h's dims 256*half .. +255, two per
+    // column; the rotary block (dims 448..511) is rotated at t on the way.
     if (!tc::mbar_wait(q_full, 0)) *abort_flag = 1;
     {
       const uint8_t* qs = s_k + (kAtStages - 1) * kAtKBytes + h * 128;
 #pragma unroll 2
-      for (int c = 0; c < 16; ++c) {                  // 32 dims = 16 columns per step
+      for (int c = 0; c < 8; ++c) {                   // 32 dims = 16 columns per step
+        const int cc = half * 8 + c;                  // 32-dim chunk of the row
         uint32_t r[16];
-        if (s_owner) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int chunk = (c & 1) * 4 + v;        // 16-byte chunk within the 128-byte row of region c/2
-            const uint4 x = *reinterpret_cast<const uint4*>(qs + (c >> 1) * kAtRegion + ((chunk ^ (h & 7)) << 4));
-            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-          }
-          if (c >= 14) {
-#pragma unroll
-            for (int q2 = 0; q2 < 16; ++q2) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r[q2]));
-              const float2 cs = s_cs[(c - 14) * 16 + q2];
-              const __nv_bfloat162 o = __floats2bfloat162_rn(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
-              r[q2] = *reinterpret_cast<const uint32_t*>(&o);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int q2 = 0; q2 < 16; ++q2) r[q2] = 0u;   // O lanes: overwritten by the first PV
+        for (int v = 0; v < 4; ++v) {
+          const int chunk = (cc & 1) * 4 + v;         // 16-byte chunk within the 128-byte row of region cc/2
+          const uint4 x = *reinterpret_cast<const uint4*>(qs + (cc >> 1) * kAtRegion + ((chunk ^ (h & 7)) << 4));
+          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
         }
-        tc::tmem_st16(tmem + lane_base + kTmQ + c * 16, r);
+        if (cc >= 14) {
+#pragma unroll
+          for (int q2 = 0; q2 < 16; ++q2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r[q2]));
+            const float2 cs = s_cs[(cc - 14) * 16 + q2];
+            const __nv_bfloat162 o = __floats2bfloat162_rn(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
+            r[q2] = *reinterpret_cast<const uint32_t*>(&o);
+          }
+        }
+        tc::tmem_st_16x32bx2_x16<128>(tmem + lane_base + kTmQ + c * 16, r);
       }
       tc::tmem_wait_st();
     }
@@ -409,79 +409,75 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, c
     if (lane == 0) tc::mbar_arrive(q_ready);
 
     bool ok = true;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;             // l_run: this thread's half of the row sum
     for (int n = 0; ok && n < n_tiles; ++n) {
       const int sb = n & 1;
       if (*abort_flag) { ok = false; break; }
       if (!tc::mbar_wait(s_full + sb, (n >> 1) & 1)) { ok = false; break; }
       tc::tc_fence_after();
-      uint32_t v[64];
-      tc::tmem_ld32(tmem + lane_base + sb * kAtKT, v);
-      tc::tmem_ld32(tmem + lane_base + sb * kAtKT + 32, v + 32);
+      uint32_t v[32];
+      tc::tmem_ld_16x32bx2_x32<32>(tmem + lane_base + sb * kAtKT, v);
       tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_free + sb);
       const int gt = t0 + n;
       int nvalid = gt < ks.tiles_c ? ks.n_c - gt * kAtKT : ks.n_w - (gt - ks.tiles_c) * kAtKT;
-      nvalid = nvalid < kAtKT ? nvalid : kAtKT;
-      float x[64];
+      nvalid = (nvalid < kAtKT ? nvalid : kAtKT) - 32 * half;   // valid keys among this thread's 32
       float tmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        x[j] = j < nvalid ? __uint_as_float(v[j]) * g.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[j]);
+      for (int j = 0; j < 32; ++j) {
+        const float s = j < nvalid ? __uint_as_float(v[j]) : -INFINITY;
+        v[j] = __float_as_uint(s);
+        tmax = fmaxf(tmax, s);
       }
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16)) * g.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
-      if (s_owner) {
-        if (n == 0) {
-          m_run = tmax;
-        } else if (tmax > m_run + 8.f) {
-          alpha = exp2f(m_run - tmax);
-          m_run = tmax;
-          rescale = true;
-        }
+      if (n == 0) {
+        m_run = tmax;
+      } else if (tmax > m_run + 8.f) {
+        alpha = exp2f(m_run - tmax);
+        m_run = tmax;
+        rescale = true;
       }
-      // the O-owner (lane + 16) rescales the O row when its S-owner asks
-      const float alpha_o = __shfl_sync(0xffffffffu, alpha, lane & 15);
       if (__any_sync(0xffffffffu, rescale)) {
-        // The 32-lane read-modify-write below also rewrites lanes 0-15 (S, Q):
-        // it runs only once PV(n-1) and S(n+1) have finished, when no MMA can
-        // be in flight (S(n+2) and PV(n) both wait for this tile's P).
+        // O (lanes 16-31) is rescaled once PV(n-1) has finished; the 16x32bx2
+        // accesses touch O's lanes only.
         if (!tc::mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1)) ok = false;
-        if (n + 1 < n_tiles && !tc::mbar_wait(s_full + ((n + 1) & 1), ((n + 1) >> 1) & 1)) ok = false;
         tc::tc_fence_after();
-        for (int c = 0; c < 512; c += 16) {
-          uint32_t r[16];
-          tc::tmem_ld16(tmem + lane_base + c, r);
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          uint32_t r[32];
+          tc::tmem_ld_16x32bx2_x32<256>(tmem + lane_base + kTmO + c, r);
           tc::tmem_wait_ld();
-          if (!s_owner) {
 #pragma unroll
-            for (int q2 = 0; q2 < 16; ++q2) r[q2] = __float_as_uint(__uint_as_float(r[q2]) * alpha_o);
-          }
-          tc::tmem_st16(tmem + lane_base + c, r);
+          for (int q2 = 0; q2 < 32; ++q2) r[q2] = __float_as_uint(__uint_as_float(r[q2]) * alpha);
+          tc::tmem_st_16x32bx2_x16<256>(tmem + lane_base + kTmO + c, r);
+          tc::tmem_st_16x32bx2_x16<256>(tmem + lane_base + kTmO + c + 16, r + 16);
         }
         tc::tmem_wait_st();
       }
-      if (s_owner) l_run *= alpha;
+      l_run *= alpha;
       // P buffer sb is free once PV(n-2) is done
       if (n >= 2 && !tc::mbar_wait(pv_done + sb, ((n - 2) >> 1) & 1)) ok = false;
-      if (s_owner) {
+      {
         float psum = 0.f;
         uint8_t* prow = s_p + sb * kAtPBytes + h * 128;
+        const float neg_m = -m_run;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t pk[4];
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
-            const float p0 = exp2f(x[8 * c + 2 * q2] - m_run);
-            const float p1 = exp2f(x[8 * c + 2 * q2 + 1] - m_run);
+            const float p0 = exp2f(fmaf(__uint_as_float(v[8 * c + 2 * q2]), g.scale_log2, neg_m));
+            const float p1 = exp2f(fmaf(__uint_as_float(v[8 * c + 2 * q2 + 1]), g.scale_log2, neg_m));
             psum += p0 + p1;
             __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
             pk[q2] = *reinterpret_cast<uint32_t*>(&bp);
           }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          const int chunk = half * 4 + c;             // keys 8*chunk .. 8*chunk+7
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
         l_run += psum;
       }
@@ -493,21 +489,19 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, c
     // ---------------------------------------------------------- epilogue
     if (ok && !tc::mbar_wait(pv_done + ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1)) ok = false;
     tc::tc_fence_after();
-    // the O-owner (lane >= 16) takes m, l from its S-owner (lane - 16)
-    const float m_o = __shfl_sync(0xffffffffu, m_run, lane & 15);
-    const float l_o = __shfl_sync(0xffffffffu, l_run, lane & 15);
+    const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
     if (ok) {
       const long long orow = row * 64 + h;
       float scale_out;
       if (g.splits > 1) {
         scale_out = 1.f;
-        if (!s_owner) {
+        if (half == 0) {
           float* ml = P.ml_part + ((long long)split * gridDim.x + row) * 128 + 2 * h;
-          ml[0] = m_o;
-          ml[1] = l_o;
+          ml[0] = m_run;
+          ml[1] = l_row;
         }
       } else {
-        float M = m_o, l = l_o;
+        float M = m_run, l = l_row;
         if (P.sink) {
           const float s2 = P.sink[h] * kLog2e;
           const float Mn = fmaxf(M, s2);
@@ -518,33 +512,32 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_ckv, c
           scale_out = 1.f;
         }
         scale_out = l > 0.f ? scale_out / l : 0.f;
-        if (!s_owner && P.lse) P.lse[orow] = l > 0.f ? (M + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        if (half == 0 && P.lse) P.lse[orow] = l > 0.f ? (M + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
-      for (int c = 0; c < 512; c += 32) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
         uint32_t r[32];
-        tc::tmem_ld32(tmem + lane_base + c, r);         // lanes 16-31: O rows
+        tc::tmem_ld_16x32bx2_x32<256>(tmem + lane_base + kTmO + c0, r);   // O dims c0.. (half 0) / 256+c0.. (half 1)
         tc::tmem_wait_ld();
-        if (!s_owner) {
-          float o[32];
+        const int c = half * 256 + c0;
+        float o[32];
 #pragma unroll
-          for (int q2 = 0; q2 < 32; ++q2) o[q2] = __uint_as_float(r[q2]) * scale_out;
-          if (g.splits == 1 && c >= 448) {
+        for (int q2 = 0; q2 < 32; ++q2) o[q2] = __uint_as_float(r[q2]) * scale_out;
+        if (g.splits == 1 && c >= 448) {
 #pragma unroll
-            for (int q2 = 0; q2 < 32; q2 += 2) {
-              const float2 cs = s_cs[(c - 448 + q2) >> 1];          // rotate by -t: (cos, -sin)
-              const float a0 = o[q2], a1 = o[q2 + 1];
-              o[q2] = a0 * cs.x + a1 * cs.y;
-              o[q2 + 1] = -a0 * cs.y + a1 * cs.x;
-            }
+          for (int q2 = 0; q2 < 32; q2 += 2) {
+            const float2 cs = s_cs[(c - 448 + q2) >> 1];            // rotate by -t: (cos, -sin)
+            const float a0 = o[q2], a1 = o[q2 + 1];
+            o[q2] = a0 * cs.x + a1 * cs.y;
+            o[q2 + 1] = -a0 * cs.y + a1 * cs.x;
           }
-          if (g.splits > 1) {
-            float* dst = P.o_part + ((long long)split * gridDim.x * 64 + orow) * 512 + c;
-            store_vec<32>(dst, o);
-          } else if (g.out_bf16) {
-            store_vec<32>(reinterpret_cast<__nv_bfloat16*>(P.out) + orow * 512 + c, o);
-          } else {
-            store_vec<32>(reinterpret_cast<float*>(P.out) + orow * 512 + c, o);
-          }
+        }
+        if (g.splits > 1) {
+          store_vec<32>(P.o_part + ((long long)split * gridDim.x * 64 + orow) * 512 + c, o);
+        } else if (g.out_bf16) {
+          store_vec<32>(reinterpret_cast<__nv_bfloat16*>(P.out) + orow * 512 + c, o);
+        } else {
+          store_vec<32>(reinterpret_cast<float*>(P.out) + orow * 512 + c, o);
         }
       }
     }
