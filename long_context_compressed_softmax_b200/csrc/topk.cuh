@@ -19,6 +19,7 @@
 // longer rows are re-read from L2 in each pass.
 #pragma once
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace lcsa {
 
@@ -307,9 +308,322 @@ topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Rows of up to kMaxCachedKeys scores with 16-byte aligned rows: persistent
+// CTAs, two per SM, one row at a time each.
+//   1. A 512-score sample gives a value range [lo, hi]; the bucket
+//      clamp((v - lo) * 2048 / (hi - lo)) is monotone in v and spreads
+//      typical score rows over many of its 2048 buckets.
+//   2. Pass 1 streams the row from global memory once: bucket histogram,
+//      and the bucket of every score kept as a 16-bit code in shared memory.
+//   3. The bucket holding the k-th score (bpiv) and the rank kr inside it
+//      come from the histogram; its scores (few) are compacted in index
+//      order into a list (scores re-read from global memory).
+//   4. The list's exact top kr (ties to the lower index) is marked: one warp
+//      ranks lists of up to 32; larger lists use 11/11/10-bit radix levels on
+//      the keys; a bucket too full for the list is resolved over the row.
+//   5. Selected list entries get code 2048, the others 0, so the selection
+//      is exactly {code > bpiv}; one ordered compaction pass emits it.
+// ---------------------------------------------------------------------------
+constexpr int kTk2Threads = 512;
+constexpr int kTk2Warps = kTk2Threads / 32;
+constexpr int kTk2Bins = 2048;
+constexpr int kTk2List = 4096;
+constexpr uint16_t kTk2Sel = 2048;                  // code of a selected score of the pivot bucket
+
+// Block-wide k-th largest key (ranks counted from 1) among cnt keys given by
+// get(c, &key) -> valid; refines *st over three digit levels so that on
+// return st->prefix is the exact key and st->kr the number of its copies to
+// keep.  All threads call it; it ends with a barrier.
+template <typename Get>
+__device__ __forceinline__ void tk2_radix(Get&& get, int cnt, uint32_t* hist, TopkState* st, uint32_t* s_warp,
+                                          uint32_t* s_total, uint32_t* s_bincnt) {
+  for (int level = 0; level < 3; ++level) {
+    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+    const uint32_t dmask = level == 2 ? 0x3FFu : 0x7FFu;
+    const int nbins = level == 2 ? 1024 : 2048;
+    for (int i = threadIdx.x; i < nbins; i += kTk2Threads) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t prefix = st->prefix, mask = st->mask;
+    for (int c = threadIdx.x; c < cnt; c += kTk2Threads) {
+      uint32_t key;
+      if (get(c, &key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    topk_pick_bin<kTk2Threads>(hist, nbins, shift, dmask, st, s_warp, s_total, s_bincnt);
+  }
+}
+
+// Ordered compaction helper: lane L holds 4 consecutive elements (bits of
+// `f`); returns the number of set bits of lanes below L, and the warp total.
+__device__ __forceinline__ uint32_t warp_excl_count4(uint32_t f, uint32_t* total) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t before = 0, tot = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (f >> q) & 1u);
+    before += __popc(b & lt);
+    tot += __popc(b);
+  }
+  *total = tot;
+  return before;
+}
+
+__global__ void __launch_bounds__(kTk2Threads, 2)
+topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, const int32_t* __restrict__ n_valid,
+                 int k, int32_t* __restrict__ idx_out, int rows) {
+  extern __shared__ __align__(16) uint16_t s_code[];   // bucket code of every score of the row
+  __shared__ uint32_t s_hist[kTk2Bins];
+  __shared__ uint32_t s_lkey[kTk2List];
+  __shared__ int32_t s_lidx[kTk2List];
+  __shared__ uint32_t s_warp[32];
+  __shared__ uint32_t s_total, s_bincnt;
+  __shared__ uint32_t s_wa[kTk2Warps], s_we[kTk2Warps];
+  __shared__ float s_lo[kTk2Warps], s_hi[kTk2Warps];
+  __shared__ TopkState s_st;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+    int n = n_cols;
+    if (n_valid != nullptr) {
+      n = n_valid[row];
+      n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
+    }
+    const float* src = scores + (long long)row * ld;
+    int32_t* dst = idx_out + (long long)row * k;
+    if (n <= k) {
+      for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = i < n ? i : -1;
+      continue;                                        // no shared memory touched: no barrier needed
+    }
+    // ---- bucket range from a sample
+    {
+      const float v = __ldg(src + (int)(((long long)threadIdx.x * n) / kTk2Threads));
+      float mn = v, mx = v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) { s_lo[warp] = mn; s_hi[warp] = mx; }
+    }
+    for (int i = threadIdx.x; i < kTk2Bins; i += kTk2Threads) s_hist[i] = 0u;
+    if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = (uint32_t)k; s_st.done = 0; }
+    __syncthreads();
+    float lo = s_lo[0], hi = s_hi[0];
+#pragma unroll
+    for (int w = 1; w < kTk2Warps; ++w) { lo = fminf(lo, s_lo[w]); hi = fmaxf(hi, s_hi[w]); }
+    // one bucket for everything when the sampled range is empty or not finite
+    const float scale = (hi > lo && hi - lo < INFINITY) ? (float)kTk2Bins / (hi - lo) : 0.f;
+    auto bucket = [&](float v) -> uint32_t {
+      if (scale == 0.f) return 0u;
+      const float x = (v - lo) * scale;                 // monotone in v; NaN-free rows
+      return x <= 0.f ? 0u : (x >= (float)(kTk2Bins - 1) ? (uint32_t)(kTk2Bins - 1) : (uint32_t)x);
+    };
+    // contiguous warp segments [seg_lo, seg_hi), lengths multiples of 128
+    const int seg = ((n + kTk2Warps - 1) / kTk2Warps + 127) & ~127;
+    const int seg_lo = warp * seg < n ? warp * seg : n;
+    const int seg_hi = seg_lo + seg < n ? seg_lo + seg : n;
+
+    // ---- pass 1: stream the row, bucket histogram and codes
+#pragma unroll 2
+    for (int base = seg_lo; base < seg_hi; base += 128) {
+      const int i0 = base + 4 * lane;
+      uint32_t b[4];
+      if (i0 + 3 < seg_hi) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(src + i0));
+        b[0] = bucket(v.x); b[1] = bucket(v.y); b[2] = bucket(v.z); b[3] = bucket(v.w);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) atomicAdd(&s_hist[b[q]], 1u);
+        *reinterpret_cast<uint2*>(s_code + i0) = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+      } else {
+        for (int q = 0; q < 4; ++q)
+          if (i0 + q < seg_hi) {
+            const uint32_t bq = bucket(__ldg(src + i0 + q));
+            atomicAdd(&s_hist[bq], 1u);
+            s_code[i0 + q] = (uint16_t)bq;
+          }
+      }
+    }
+    __syncthreads();
+    topk_pick_bin<kTk2Threads>(s_hist, kTk2Bins, 0, 0x7FFu, &s_st, s_warp, &s_total, &s_bincnt);
+    const uint32_t bpiv = s_st.prefix, kr = s_st.kr, cnt = s_bincnt;
+    const bool fits = cnt <= (uint32_t)kTk2List;
+
+    // ---- per-warp counts above / in the pivot bucket
+    {
+      uint32_t a = 0, e = 0;
+      for (int base = seg_lo; base < seg_hi; base += 128) {
+        const int i0 = base + 4 * lane;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (i0 + q < seg_hi) {
+            const uint32_t c = s_code[i0 + q];
+            a += c > bpiv;
+            e += c == bpiv;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+      }
+      if (lane == 0) { s_wa[warp] = a; s_we[warp] = e; }
+    }
+    __syncthreads();
+
+    if (fits) {
+      // ---- the pivot bucket's scores, in index order, into the list
+      uint32_t off = 0;
+      for (int w = 0; w < warp; ++w) off += s_we[w];
+      if (s_we[warp] > 0) {
+        for (int base = seg_lo; base < seg_hi; base += 128) {
+          const int i0 = base + 4 * lane;
+          uint32_t f = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] == bpiv) << q;
+          if (!__any_sync(0xffffffffu, f != 0u)) continue;
+          uint32_t tot;
+          uint32_t pos = off + warp_excl_count4(f, &tot);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if ((f >> q) & 1u) {
+              s_lkey[pos] = score_key(__ldg(src + i0 + q));
+              s_lidx[pos] = i0 + q;
+              ++pos;
+            }
+          off += tot;
+        }
+      }
+      __syncthreads();
+      // ---- exact top kr of the list (ties to the lower index, i.e. list order)
+      if (cnt <= 32) {
+        if (warp == 0) {
+          const bool have = lane < (int)cnt;
+          const uint32_t key = have ? s_lkey[lane] : 0u;
+          uint32_t rank = 0;                           // list entries before this one in (key desc, index asc)
+          for (int j = 0; j < (int)cnt; ++j) {
+            const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+            rank += (kj > key || (kj == key && j < lane)) ? 1u : 0u;
+          }
+          if (have) s_code[s_lidx[lane]] = rank < kr ? kTk2Sel : (uint16_t)0;
+          const uint32_t sel = __ballot_sync(0xffffffffu, have && rank < kr);
+          if (have && rank < kr) atomicAdd(&s_wa[s_lidx[lane] / seg], 1u);
+          (void)sel;
+        }
+      } else {
+        if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = kr; }
+        __syncthreads();
+        tk2_radix([&](int c, uint32_t* key) { *key = s_lkey[c]; return true; }, (int)cnt, s_hist, &s_st, s_warp,
+                  &s_total, &s_bincnt);
+        const uint32_t T = s_st.prefix, rT = s_st.kr;  // keep every key > T and the first rT copies of T
+        // list order is index order: the first rT ties win
+        if (threadIdx.x == 0) s_total = 0u;
+        __syncthreads();
+        for (int c0 = 0; c0 < (int)cnt; c0 += kTk2Threads) {
+          const int c = c0 + threadIdx.x;
+          const uint32_t key = c < (int)cnt ? s_lkey[c] : 0u;
+          const bool tie = c < (int)cnt && key == T;
+          const uint32_t tie_before = block_excl_scan<kTk2Threads>(tie ? 1u : 0u, s_warp, &s_bincnt) + s_total;
+          if (c < (int)cnt) {
+            const bool sel = key > T || (tie && tie_before < rT);
+            s_code[s_lidx[c]] = sel ? kTk2Sel : (uint16_t)0;
+            if (sel) atomicAdd(&s_wa[s_lidx[c] / seg], 1u);
+          }
+          __syncthreads();
+          if (threadIdx.x == 0) s_total += s_bincnt;
+          __syncthreads();
+        }
+      }
+    } else {
+      // ---- the pivot bucket overflows the list: exact key over the row
+      // (scores of the pivot bucket re-read from global memory)
+      if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = kr; }
+      __syncthreads();
+      tk2_radix(
+          [&](int c, uint32_t* key) {
+            if (s_code[c] != bpiv) return false;
+            *key = score_key(__ldg(src + c));
+            return true;
+          },
+          n, s_hist, &s_st, s_warp, &s_total, &s_bincnt);
+      const uint32_t T = s_st.prefix, rT = s_st.kr;
+      // ties of T per warp segment, in index order
+      uint32_t e = 0;
+      for (int i = seg_lo + lane; i < seg_hi; i += 32)
+        if (s_code[i] == bpiv) e += score_key(__ldg(src + i)) == T;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      if (lane == 0) s_we[warp] = e;
+      __syncthreads();
+      uint32_t tie_off = 0;
+      for (int w = 0; w < warp; ++w) tie_off += s_we[w];
+      uint32_t sel_cnt = 0;
+      for (int base = seg_lo; base < seg_hi; base += 32) {
+        const int i = base + lane;
+        const bool in = i < seg_hi && s_code[i] == bpiv;
+        const uint32_t key = in ? score_key(__ldg(src + i)) : 0u;
+        const bool tie = in && key == T;
+        const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+        const bool sel = in && (key > T || (tie && tie_off + __popc(tb & ((1u << lane) - 1u)) < rT));
+        if (in) s_code[i] = sel ? kTk2Sel : (uint16_t)0;
+        sel_cnt += sel;
+        tie_off += __popc(tb);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sel_cnt += __shfl_xor_sync(0xffffffffu, sel_cnt, o);
+      if (lane == 0) s_wa[warp] += sel_cnt;
+    }
+    __syncthreads();
+
+    // ---- emission: the selection is {code > bpiv}, written in index order
+    {
+      uint32_t pos = 0;
+      for (int w = 0; w < warp; ++w) pos += s_wa[w];
+      for (int base = seg_lo; base < seg_hi; base += 128) {
+        const int i0 = base + 4 * lane;
+        uint32_t f = 0;
+        if (i0 + 3 < seg_hi) {
+          const uint2 c = *reinterpret_cast<const uint2*>(s_code + i0);
+          f = (uint32_t)((c.x & 0xFFFFu) > bpiv) | ((uint32_t)((c.x >> 16) > bpiv) << 1) |
+              ((uint32_t)((c.y & 0xFFFFu) > bpiv) << 2) | ((uint32_t)((c.y >> 16) > bpiv) << 3);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] > bpiv) << q;
+        }
+        if (!__any_sync(0xffffffffu, f != 0u)) continue;
+        uint32_t tot;
+        uint32_t p = pos + warp_excl_count4(f, &tot);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if ((f >> q) & 1u) dst[p++] = i0 + q;
+        pos += tot;
+      }
+    }
+    __syncthreads();                                    // codes and counters are reused by the next row
+  }
+}
+
+static bool topk_smem_ok(const float* scores, int n_cols, long long ld) {
+  return n_cols <= kMaxCachedKeys && (ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15u) == 0;
+}
+
 static cudaError_t launch_topk(const float* scores, int rows, int n_cols, long long ld, const int32_t* n_valid,
                                int k, int32_t* idx_out, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (topk_smem_ok(scores, n_cols, ld)) {
+    const size_t smem = (size_t)((n_cols + 7) & ~7) * 2;
+    cudaError_t e = cudaFuncSetAttribute(topk_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kMaxCachedKeys * 2);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = rows < 2 * sms ? rows : 2 * sms;
+    count_launch();
+    topk_smem_kernel<<<grid, kTk2Threads, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out, rows);
+    return cudaGetLastError();
+  }
   // Rows longer than k are staged in shared memory when they fit.
   const int cache_cap = n_cols <= k ? 0 : (n_cols < kMaxCachedKeys ? n_cols : kMaxCachedKeys);
   const size_t smem = (size_t)cache_cap * 4;

@@ -68,7 +68,9 @@ def test_compress_short_sequence(lcsa):
 @pytest.mark.parametrize("n_cols,k,ties", [(64, 8, 0), (1000, 64, 4), (8191, 2048, 0), (8191, 2048, 16),
                                           (40000, 2048, 0), (5000, 1, 3), (300, 2048, 0),
                                           (32768, 2048, 0), (262144, 2048, 0),   # cached / uncached rows
-                                          (40000, 2048, 1), (262144, 2048, 2)])  # threshold bin > candidate list
+                                          (40000, 2048, 1), (262144, 2048, 2),   # threshold bin > candidate list
+                                          (32768, 2048, 16), (32768, 2048, 1),   # shared-memory kernel: ties,
+                                          (4096, 2048, 0), (2052, 2048, 3)])     # bucket overflow, n just above k
 def test_topk_bitexact(lcsa, n_cols, k, ties):
     rows = 37 if n_cols < 100000 else 6
     s = gen.make_scores(rows, n_cols, seed=31 + n_cols, device=DEV, tie_levels=ties)
@@ -88,6 +90,24 @@ def test_topk_adversarial_rows(lcsa):
     s = torch.tensor(np.stack(rows), dtype=torch.float32, device=DEV)
     idx = lcsa.topk_from_scores(s, k)
     ref = O.topk_from_scores(s.cpu().double().numpy(), [100] * len(rows), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_skewed_rows(lcsa):
+    """Rows whose value range is dominated by outliers (one sampled bucket
+    holds nearly everything), infinities and constant rows."""
+    n, k = 6000, 2048
+    g = np.random.default_rng(5)
+    base = g.standard_normal((6, n)).astype(np.float32)
+    base[0, 17] = 1e30                                    # one huge outlier
+    base[1, ::7] = -1e30                                  # many huge negatives
+    base[2, 100:110] = np.inf                             # +inf entries
+    base[3, :] = 0.25                                     # constant row
+    base[4, ::2] = -np.inf                                # half the row -inf
+    base[5, :] = np.round(base[5, :] * 4) / 4             # coarse levels, ties everywhere
+    s = torch.tensor(base, device=DEV)
+    idx = lcsa.topk_from_scores(s, k)
+    ref = O.topk_from_scores(s.cpu().double().numpy(), [n] * 6, k)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref)
 
 
