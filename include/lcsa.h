@@ -116,6 +116,14 @@ lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_cha
  *   scores  [rows, ld] fp32 (row stride ld >= n_cols)
  *   n_valid [rows] int32 device, or NULL (= n_cols for every row)
  *   idx_out [rows, k] int32
+ *
+ * lcsa_topk_workspace returns the device scratch (bytes, 16-byte aligned)
+ * that lets rows longer than 32768 columns take the two-phase path (top k of
+ * every 32768-column chunk, then of their union); it is 0 when that path does
+ * not apply (short rows, k not a multiple of 4, more than 32768/k chunks).
+ * Without it, long rows use a single-phase kernel with the same result.
+ * The workspace is owned by the caller and must stay valid until the work on
+ * `stream` is done.
  * ------------------------------------------------------------------------ */
 size_t lcsa_topk_workspace(int rows, int n_cols, int k);
 lcsa_status lcsa_topk_from_scores(const float* scores, int rows, int n_cols, int64_t ld,

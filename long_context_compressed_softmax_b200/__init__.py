@@ -161,15 +161,28 @@ def hca_compress(kv, gate, m=128, out_dtype=None, rms_weight=None, rms_eps=1e-6,
 
 
 # ----------------------------------------------------------------- top-k
-def topk_from_scores(scores, k, n_valid=None, out=None):
-    """scores [rows, n_cols] fp32 (row stride may exceed n_cols) -> idx [rows, k] int32."""
+def topk_workspace_bytes(rows, n_cols, k):
+    """Scratch that lets rows longer than 32768 columns take the two-phase path."""
+    return int(_lib.lcsa_topk_workspace(rows, n_cols, k))
+
+
+def topk_from_scores(scores, k, n_valid=None, out=None, workspace=None):
+    """scores [rows, n_cols] fp32 (row stride may exceed n_cols) -> idx [rows, k] int32.
+
+    workspace: None allocates the scratch of topk_workspace_bytes; a uint8
+    tensor is used as is; False passes none (long rows then use the
+    single-phase kernel)."""
     rows, n_cols = scores.shape
     if scores.stride(1) != 1:
         raise ValueError("scores rows must be contiguous")
     if out is None:
         out = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
-    st = _lib.lcsa_topk_from_scores(_p(scores), rows, n_cols, scores.stride(0), _p(n_valid), k, _p(out), None, 0,
-                                    _stream(scores.device))
+    if workspace is None:
+        nbytes = topk_workspace_bytes(rows, n_cols, k)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=scores.device) if nbytes else False
+    ws_ptr, ws_bytes = (None, 0) if workspace is False else (_p(workspace), workspace.numel())
+    st = _lib.lcsa_topk_from_scores(_p(scores), rows, n_cols, scores.stride(0), _p(n_valid), k, _p(out), ws_ptr,
+                                    ws_bytes, _stream(scores.device))
     _check(st, "topk_from_scores")
     return out
 

@@ -184,22 +184,23 @@ lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_cha
 }
 
 size_t lcsa_topk_workspace(int rows, int n_cols, int k) {
-  (void)rows; (void)n_cols; (void)k;
-  return 0;
+  if (rows <= 0 || n_cols <= 0 || k <= 0) return 0;
+  return topk_long_scratch(rows, n_cols, k);
 }
 
 lcsa_status lcsa_topk_from_scores(const float* scores, int rows, int n_cols, int64_t ld, const int32_t* n_valid,
                                   int k, int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                   void* stream) {
-  (void)workspace; (void)workspace_bytes;
   if (rows < 0 || n_cols < 0 || k <= 0 || ld < n_cols) return LCSA_ERR_INVALID_ARG;
   if (rows == 0) return LCSA_OK;
   if (!idx_out || (n_cols > 0 && !scores)) return LCSA_ERR_INVALID_ARG;
   if (!aligned16(idx_out) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)) ||
       (n_valid && (reinterpret_cast<uintptr_t>(n_valid) & 3u)))
     return LCSA_ERR_INVALID_ARG;
+  if (workspace && !aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
   if (!have_device()) return LCSA_ERR_CUDA;
-  return from_cuda(launch_topk(scores, rows, n_cols, (long long)ld, n_valid, k, idx_out, (cudaStream_t)stream));
+  return from_cuda(launch_topk(scores, rows, n_cols, (long long)ld, n_valid, k, idx_out, (cudaStream_t)stream,
+                               workspace, workspace_bytes));
 }
 
 int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a) { return a && indexer_tc_supported(a) ? 1 : 0; }
@@ -208,8 +209,9 @@ size_t lcsa_indexer_topk_workspace(const lcsa_indexer_args* a) {
   if (!a || a->B <= 0 || a->Tq <= 0) return 0;
   const long long rows = (long long)a->B * a->Tq;
   const long long chunk = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
-  // score chunk + per-row visible counts
-  return align256((size_t)chunk * (size_t)(a->Nc > 0 ? a->Nc : 1) * 4) + align256((size_t)chunk * 4);
+  // score chunk + per-row visible counts + scratch of the two-phase top-k of long rows
+  return align256((size_t)chunk * (size_t)(a->Nc > 0 ? a->Nc : 1) * 4) + align256((size_t)chunk * 4) +
+         topk_long_scratch((int)chunk, a->Nc, a->k);
 }
 
 lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_t workspace_bytes, void* stream) {
@@ -222,13 +224,17 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_
   const int Nc = a->Nc > 0 ? a->Nc : 1;
   // Rows per chunk: as many score rows as the workspace holds (scores + counts).
   const size_t per_row = (size_t)Nc * 4;
-  auto need = [&](long long r) { return align256((size_t)r * per_row) + align256((size_t)r * 4); };
+  auto need = [&](long long r) {
+    return align256((size_t)r * per_row) + align256((size_t)r * 4) + topk_long_scratch((int)r, a->Nc, a->k);
+  };
   long long budget = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
   while (budget > 1 && need(budget) > workspace_bytes) budget >>= 1;
   if (!workspace || need(budget) > workspace_bytes) return LCSA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
   float* sc_ws = (float*)workspace;
   int32_t* nv = (int32_t*)((char*)workspace + align256((size_t)budget * per_row));
+  void* tk_scratch = (char*)workspace + align256((size_t)budget * per_row) + align256((size_t)budget * 4);
+  const size_t tk_bytes = topk_long_scratch((int)budget, a->Nc, a->k);
   const bool tc = indexer_tc_supported(a);
   // Chunk rectangles: whole sequences when a sequence fits, else row ranges of
   // one sequence (a multiple of the 4-row query group).
@@ -251,7 +257,7 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_
       }
       count_launch();
       nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, a->q_pos0, a->m, a->Nc);
-      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st);
+      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st, tk_scratch, tk_bytes);
       if (e != cudaSuccess) return LCSA_ERR_CUDA;
     }
   }

@@ -372,7 +372,11 @@ __device__ __forceinline__ uint32_t warp_excl_count4(uint32_t f, uint32_t* total
 
 __global__ void __launch_bounds__(kTk2Threads, 2)
 topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, const int32_t* __restrict__ n_valid,
-                 int k, int32_t* __restrict__ idx_out, int rows) {
+                 int k, int32_t* __restrict__ idx_out, int rows, int chunk, const int32_t* __restrict__ map,
+                 long long map_ld) {
+  // chunk > 0: virtual row v is columns [c*chunk, (c+1)*chunk) of row v / C
+  // (C = ceil(n_cols / chunk), c = v % C), n_valid counted from c*chunk.
+  // map != NULL: the emitted value of column i is map[row * map_ld + i].
   extern __shared__ __align__(16) uint16_t s_code[];   // bucket code of every score of the row
   __shared__ uint32_t s_hist[kTk2Bins];
   __shared__ uint32_t s_lkey[kTk2List];
@@ -384,16 +388,23 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
   __shared__ TopkState s_st;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+  const int C = chunk > 0 ? (n_cols + chunk - 1) / chunk : 1;
   for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+    const int r = row / C, c = row - r * C;          // real row and column chunk
+    const int c0 = chunk > 0 ? c * chunk : 0;
+    const int width = chunk > 0 ? (n_cols - c0 < chunk ? n_cols - c0 : chunk) : n_cols;
     int n = n_cols;
     if (n_valid != nullptr) {
-      n = n_valid[row];
+      n = n_valid[r];
       n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
     }
-    const float* src = scores + (long long)row * ld;
+    n -= c0;
+    n = n < 0 ? 0 : (n > width ? width : n);
+    const float* src = scores + (long long)r * ld + c0;
     int32_t* dst = idx_out + (long long)row * k;
+    const int32_t* mrow = map ? map + (long long)row * map_ld : nullptr;
     if (n <= k) {
-      for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = i < n ? i : -1;
+      for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = i < n ? (mrow ? mrow[i] : i) : -1;
       continue;                                        // no shared memory touched: no barrier needed
     }
     // ---- bucket range from a sample
@@ -597,7 +608,7 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
         uint32_t p = pos + warp_excl_count4(f, &tot);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          if ((f >> q) & 1u) dst[p++] = i0 + q;
+          if ((f >> q) & 1u) dst[p++] = mrow ? mrow[i0 + q] : i0 + q;
         pos += tot;
       }
     }
@@ -609,20 +620,95 @@ static bool topk_smem_ok(const float* scores, int n_cols, long long ld) {
   return n_cols <= kMaxCachedKeys && (ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15u) == 0;
 }
 
+// Rows longer than kMaxCachedKeys, in two exact phases: the top k of every
+// 32768-column chunk, then the top k of the union of those (in column order,
+// so ties still go to the lower column: an entry that loses inside its chunk
+// has k chunk-mates ahead of it in the global order too).
+constexpr int kTkChunk = kMaxCachedKeys;
+static int topk_long_chunks(int n_cols, int k) {
+  if (n_cols <= kMaxCachedKeys || (k & 3) != 0) return 0;     // candidate rows must stay 16-byte aligned
+  const int C = (n_cols + kTkChunk - 1) / kTkChunk;
+  return (long long)C * k <= kMaxCachedKeys ? C : 0;
+}
+static size_t topk_long_scratch(int rows, int n_cols, int k) {
+  const int C = topk_long_chunks(n_cols, k);
+  if (C == 0) return 0;
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t per = (size_t)rows * C * k * 4;
+  return 3 * al(per) + al((size_t)rows * 4);
+}
+
+// Union of the chunk selections, compacted in column order: scores, columns
+// and the count per row.  One block per row.
+__global__ void __launch_bounds__(256)
+topk_gather_kernel(const float* __restrict__ scores, long long ld, int n_cols, const int32_t* __restrict__ n_valid,
+                   int k, int C, const int32_t* __restrict__ local, float* __restrict__ cs, int32_t* __restrict__ ci,
+                   int32_t* __restrict__ cn) {
+  const int r = blockIdx.x;
+  int n = n_cols;
+  if (n_valid != nullptr) {
+    n = n_valid[r];
+    n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
+  }
+  int off = 0;
+  for (int c = 0; c < C; ++c) {
+    int nc = n - c * kTkChunk;
+    nc = nc < 0 ? 0 : (nc > kTkChunk ? kTkChunk : nc);
+    const int cnt = nc < k ? nc : k;
+    const int32_t* lrow = local + ((long long)r * C + c) * k;
+    for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
+      const int col = c * kTkChunk + lrow[j];
+      cs[(long long)r * C * k + off + j] = scores[(long long)r * ld + col];
+      ci[(long long)r * C * k + off + j] = col;
+    }
+    off += cnt;
+  }
+  if (threadIdx.x == 0) cn[r] = off;
+}
+
+static cudaError_t launch_topk_smem(const float* scores, int rows, int n_cols, long long ld, const int32_t* n_valid,
+                                    int k, int32_t* idx_out, int chunk, const int32_t* map, long long map_ld,
+                                    cudaStream_t st) {
+  const int width = chunk > 0 ? chunk : n_cols;
+  const size_t smem = (size_t)((width + 7) & ~7) * 2;
+  cudaError_t e = cudaFuncSetAttribute(topk_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxCachedKeys * 2);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = rows < 2 * sms ? rows : 2 * sms;
+  count_launch();
+  topk_smem_kernel<<<grid, kTk2Threads, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out, rows, chunk, map,
+                                                    map_ld);
+  return cudaGetLastError();
+}
+
+// `scratch` (topk_long_scratch bytes, 256-byte aligned) enables the two-phase
+// path for long rows; without it long rows use topk_rows_kernel.
 static cudaError_t launch_topk(const float* scores, int rows, int n_cols, long long ld, const int32_t* n_valid,
-                               int k, int32_t* idx_out, cudaStream_t st) {
+                               int k, int32_t* idx_out, cudaStream_t st, void* scratch = nullptr,
+                               size_t scratch_bytes = 0) {
   if (rows == 0) return cudaSuccess;
-  if (topk_smem_ok(scores, n_cols, ld)) {
-    const size_t smem = (size_t)((n_cols + 7) & ~7) * 2;
-    cudaError_t e = cudaFuncSetAttribute(topk_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kMaxCachedKeys * 2);
+  if (topk_smem_ok(scores, n_cols, ld))
+    return launch_topk_smem(scores, rows, n_cols, ld, n_valid, k, idx_out, 0, nullptr, 0, st);
+  const int C = topk_long_chunks(n_cols, k);
+  const size_t need = topk_long_scratch(rows, n_cols, k);
+  if (C > 0 && scratch != nullptr && need > 0 && scratch_bytes >= need && (ld & 3) == 0 &&
+      (reinterpret_cast<uintptr_t>(scores) & 15u) == 0) {
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t per = al((size_t)rows * C * k * 4);
+    uint8_t* w = reinterpret_cast<uint8_t*>(scratch);
+    int32_t* local = reinterpret_cast<int32_t*>(w);
+    float* cs = reinterpret_cast<float*>(w + per);
+    int32_t* ci = reinterpret_cast<int32_t*>(w + 2 * per);
+    int32_t* cn = reinterpret_cast<int32_t*>(w + 3 * per);
+    cudaError_t e = launch_topk_smem(scores, rows * C, n_cols, ld, n_valid, k, local, kTkChunk, nullptr, 0, st);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = rows < 2 * sms ? rows : 2 * sms;
     count_launch();
-    topk_smem_kernel<<<grid, kTk2Threads, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out, rows);
-    return cudaGetLastError();
+    topk_gather_kernel<<<rows, 256, 0, st>>>(scores, ld, n_cols, n_valid, k, C, local, cs, ci, cn);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_topk_smem(cs, rows, C * k, (long long)C * k, cn, k, idx_out, 0, ci, (long long)C * k, st);
   }
   // Rows longer than k are staged in shared memory when they fit.
   const int cache_cap = n_cols <= k ? 0 : (n_cols < kMaxCachedKeys ? n_cols : kMaxCachedKeys);

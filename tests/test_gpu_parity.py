@@ -93,6 +93,21 @@ def test_topk_adversarial_rows(lcsa):
     np.testing.assert_array_equal(idx.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("n_cols,k,ties", [(262144, 2048, 0), (40000, 2048, 1), (70001, 64, 0), (50000, 6, 0)])
+def test_topk_long_rows_both_paths(lcsa, n_cols, k, ties):
+    """Rows longer than one shared-memory chunk: the two-phase path (chunk
+    top-k, then top-k of their union) and the single-phase kernel agree with
+    the oracle; k = 6 has no two-phase path."""
+    rows = 5
+    s = gen.make_scores(rows, n_cols, seed=41 + n_cols, device=DEV, tie_levels=ties)
+    nv = torch.tensor([n_cols, k, n_cols // 2 + 3, 32768 + 5, 32767][:rows], dtype=torch.int32)
+    ref = O.topk_from_scores(s.cpu().double().numpy(), nv.numpy(), k)
+    for ws in (None, False):
+        idx = lcsa.topk_from_scores(s, k, n_valid=nv.to(DEV), workspace=ws)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+    assert (lcsa.topk_workspace_bytes(rows, n_cols, k) > 0) == (k % 4 == 0)
+
+
 def test_topk_skewed_rows(lcsa):
     """Rows whose value range is dominated by outliers (one sampled bucket
     holds nearly everything), infinities and constant rows."""
