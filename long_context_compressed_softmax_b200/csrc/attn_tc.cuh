@@ -79,6 +79,7 @@ struct AtGeom {
   int rot_slot;        // CSA rotary slices indexed by (query, slot) instead of by entry
   int splits;
   int out_bf16;
+  int out_v8;          // the output (or split partials) is 32-byte aligned: 32-byte stores
   int n_items;         // rows * splits
 };
 
@@ -219,6 +220,29 @@ __device__ __forceinline__ void at_q_to_tmem(const uint8_t* qs, const float2* cs
   tc::tmem_wait_st();
 }
 
+// 32 consecutive values as 32-byte stores (p 32-byte aligned).
+__device__ __forceinline__ void st_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+__device__ __forceinline__ void store32_v8(float* p, const float* o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_v8(p + 8 * j, reinterpret_cast<const uint32_t*>(o + 8 * j));
+}
+__device__ __forceinline__ void store32_v8(__nv_bfloat16* p, const float* o) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[16 * j + 2 * e], o[16 * j + 2 * e + 1]);
+      w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    st_v8(p + 16 * j, w);
+  }
+}
+
 // Epilogue of one item, executed by the 128 transition threads.  Row
 // statistics come from the softmax warps through shared memory; O -> sink,
 // normalisation, -t rotation of the rotary block -> output (or split
@@ -282,8 +306,13 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
         o[q2 + 1] = -a0 * e.y + a1 * e.x;
       }
     }
-    if (obf) store_vec<32>(obf + d0, o);
-    else store_vec<32>(of32 + d0, o);
+    if (g.out_v8) {
+      if (obf) store32_v8(obf + d0, o);
+      else store32_v8(of32 + d0, o);
+    } else {
+      if (obf) store_vec<32>(obf + d0, o);
+      else store_vec<32>(of32 + d0, o);
+    }
   }
   return ok;
 }
@@ -923,6 +952,7 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   g.rot_slot = pl.rot_slot;
   g.splits = pl.splits;
   g.out_bf16 = a->out_dtype == LCSA_BF16;
+  g.out_v8 = (reinterpret_cast<uintptr_t>(pl.splits > 1 ? (const void*)P.o_part : a->out) & 31u) == 0 ? 1 : 0;
   g.n_items = (int)(rows * pl.splits);
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
   if (e != cudaSuccess) return e;

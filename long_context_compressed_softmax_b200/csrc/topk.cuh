@@ -389,8 +389,9 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   const int C = chunk > 0 ? (n_cols + chunk - 1) / chunk : 1;
-  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
-    const int r = row / C, c = row - r * C;          // real row and column chunk
+  // scores of (virtual) row v and how many of them count
+  auto setup = [&](int v, const float** src_out) {
+    const int r = v / C, c = v - r * C;              // real row and column chunk
     const int c0 = chunk > 0 ? c * chunk : 0;
     const int width = chunk > 0 ? (n_cols - c0 < chunk ? n_cols - c0 : chunk) : n_cols;
     int n = n_cols;
@@ -399,17 +400,37 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
       n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
     }
     n -= c0;
-    n = n < 0 ? 0 : (n > width ? width : n);
-    const float* src = scores + (long long)r * ld + c0;
+    *src_out = scores + (long long)r * ld + c0;
+    return n < 0 ? 0 : (n > width ? width : n);
+  };
+  // this thread's sample score of a row (issued one row ahead)
+  auto sample = [&](const float* src, int n) {
+    return n > k ? __ldg(src + (int)(((long long)threadIdx.x * n) / kTk2Threads)) : 0.f;
+  };
+  float smp_next = 0.f;
+  if ((int)blockIdx.x < rows) {
+    const float* s0;
+    const int n0 = setup(blockIdx.x, &s0);
+    smp_next = sample(s0, n0);
+  }
+  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+    const float* src;
+    const int n = setup(row, &src);
+    const float smp = smp_next;
     int32_t* dst = idx_out + (long long)row * k;
     const int32_t* mrow = map ? map + (long long)row * map_ld : nullptr;
+    if (row + (int)gridDim.x < rows && n <= k) {
+      const float* s2;
+      const int n2 = setup(row + gridDim.x, &s2);
+      smp_next = sample(s2, n2);
+    }
     if (n <= k) {
       for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = i < n ? (mrow ? mrow[i] : i) : -1;
       continue;                                        // no shared memory touched: no barrier needed
     }
-    // ---- bucket range from a sample
+    // ---- bucket range from the sample
     {
-      const float v = __ldg(src + (int)(((long long)threadIdx.x * n) / kTk2Threads));
+      const float v = smp;
       float mn = v, mx = v;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -437,7 +458,7 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     const int seg_hi = seg_lo + seg < n ? seg_lo + seg : n;
 
     // ---- pass 1: stream the row, bucket histogram and codes
-#pragma unroll 2
+#pragma unroll 4
     for (int base = seg_lo; base < seg_hi; base += 128) {
       const int i0 = base + 4 * lane;
       uint32_t b[4];
@@ -466,12 +487,22 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
       uint32_t a = 0, e = 0;
       for (int base = seg_lo; base < seg_hi; base += 128) {
         const int i0 = base + 4 * lane;
+        if (i0 + 3 < seg_hi) {
+          const uint2 c = *reinterpret_cast<const uint2*>(s_code + i0);
+          const uint32_t cq[4] = {c.x & 0xFFFFu, c.x >> 16, c.y & 0xFFFFu, c.y >> 16};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (i0 + q < seg_hi) {
-            const uint32_t c = s_code[i0 + q];
-            a += c > bpiv;
-            e += c == bpiv;
+          for (int q = 0; q < 4; ++q) {
+            a += cq[q] > bpiv;
+            e += cq[q] == bpiv;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (i0 + q < seg_hi) {
+              const uint32_t c = s_code[i0 + q];
+              a += c > bpiv;
+              e += c == bpiv;
+            }
           }
         }
       }
@@ -588,6 +619,11 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     }
     __syncthreads();
 
+    if (row + (int)gridDim.x < rows) {                 // next row's sample, in flight during the emission
+      const float* s2;
+      const int n2 = setup(row + gridDim.x, &s2);
+      smp_next = sample(s2, n2);
+    }
     // ---- emission: the selection is {code > bpiv}, written in index order
     {
       uint32_t pos = 0;

@@ -247,6 +247,23 @@ def test_attn_bf16_output(lcsa):
     assert_attn_close(np64(out).reshape(ref.shape), ref, max_abs=2e-2, mean_abs=3e-3)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_attn_output_alignment(lcsa, out_dtype):
+    """An output buffer that is 16- but not 32-byte aligned takes the 16-byte
+    store path and gives the same values as an aligned one."""
+    B, H, D, R, m, W, Tq, Nc, q0 = 1, 64, 512, 64, 128, 128, 300, 40, 4800
+    x = _attn_case(B, Tq, H, D, Nc, q0 + Tq, "bf16", seed=85)
+    ref = lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q0, 0, m, W, R, out_dtype=out_dtype)
+    shift = 16 // torch.tensor([], dtype=out_dtype).element_size()
+    buf = torch.empty(B * Tq * H * D + 2 * shift, dtype=out_dtype, device=DEV)
+    base = buf.data_ptr() % 32
+    off = shift if base == 0 else 0                     # start 16 bytes past a 32-byte boundary
+    out = buf[off:off + B * Tq * H * D].view(B, Tq, H, D)
+    assert out.data_ptr() % 32 == 16
+    lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q0, 0, m, W, R, out_dtype=out_dtype, out=out)
+    assert torch.equal(out, ref)
+
+
 def test_layer_shapes_use_tensor_cores(lcsa):
     x = _attn_case(1, 4, 64, 512, 100, 100, "bf16", seed=91)
     assert lcsa.attn_uses_tensor_cores(x["q"], x["ckv"], x["kv"], R=64)
