@@ -51,6 +51,10 @@ CONFIGS = {
     "csa_prefill_32k": WorkloadConfig(name="csa_prefill_32k", dtype="bf16", B=1, T=32768, seed=1),
     # HCA layer prefill, T=131072 (1024 entries).
     "hca_prefill_128k": WorkloadConfig(name="hca_prefill_128k", dtype="bf16", B=1, T=131072, seed=2),
+    # Profiling-sized HCA layer and decode case (a few GB on the device).
+    "hca_prefill_16k": WorkloadConfig(name="hca_prefill_16k", dtype="bf16", B=1, T=16384, seed=7),
+    "csa_decode_8seq": WorkloadConfig(name="csa_decode_8seq", dtype="bf16", B=8, T=1 << 20, seed=8,
+                                      decode=True, boost_frac=0.01),
     # CSA decode at 1M context: 64 sequences, one query each at position 2^20.
     "csa_decode_1m": WorkloadConfig(name="csa_decode_1m", dtype="bf16", B=64, T=1 << 20, seed=3,
                                     decode=True, boost_frac=0.01),
