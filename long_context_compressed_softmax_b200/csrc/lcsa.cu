@@ -257,7 +257,10 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_
       }
       count_launch();
       nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, a->q_pos0, a->m, a->Nc);
-      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st, tk_scratch, tk_bytes);
+      // the longest row of the rectangle is its last position's visible count
+      const long long last_vis = (a->q_pos0 + i0 + ni - 1) / a->m;
+      const int n_max = (int)(last_vis < a->Nc ? last_vis : a->Nc);
+      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st, tk_scratch, tk_bytes, n_max);
       if (e != cudaSuccess) return LCSA_ERR_CUDA;
     }
   }

@@ -325,17 +325,17 @@ topk_rows_kernel(const float* __restrict__ scores, long long ld, int n_cols,
 //   5. Selected list entries get code 2048, the others 0, so the selection
 //      is exactly {code > bpiv}; one ordered compaction pass emits it.
 // ---------------------------------------------------------------------------
-constexpr int kTk2Threads = 512;
-constexpr int kTk2Warps = kTk2Threads / 32;
+// CTA size: 512 threads (two CTAs per SM) for long rows, 256 (four per SM)
+// when the code buffer is at most 32 KB.
 constexpr int kTk2Bins = 2048;
-constexpr int kTk2List = 4096;
+constexpr int kTk2List = 1024;
 constexpr uint16_t kTk2Sel = 2048;                  // code of a selected score of the pivot bucket
 
 // Block-wide k-th largest key (ranks counted from 1) among cnt keys given by
 // get(c, &key) -> valid; refines *st over three digit levels so that on
 // return st->prefix is the exact key and st->kr the number of its copies to
 // keep.  All threads call it; it ends with a barrier.
-template <typename Get>
+template <int kTk2Threads, typename Get>
 __device__ __forceinline__ void tk2_radix(Get&& get, int cnt, uint32_t* hist, TopkState* st, uint32_t* s_warp,
                                           uint32_t* s_total, uint32_t* s_bincnt) {
   for (int level = 0; level < 3; ++level) {
@@ -370,10 +370,14 @@ __device__ __forceinline__ uint32_t warp_excl_count4(uint32_t f, uint32_t* total
   return before;
 }
 
-__global__ void __launch_bounds__(kTk2Threads, 2)
+template <int kTk2Threads>
+__global__ void __launch_bounds__(kTk2Threads, 1024 / kTk2Threads)
 topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, const int32_t* __restrict__ n_valid,
                  int k, int32_t* __restrict__ idx_out, int rows, int chunk, const int32_t* __restrict__ map,
-                 long long map_ld) {
+                 long long map_ld, int code_cap) {
+  // code_cap: capacity of the code buffer (the longest row this launch may
+  // see, from the caller); a longer row is reported and left unselected.
+  constexpr int kTk2Warps = kTk2Threads / 32;
   // chunk > 0: virtual row v is columns [c*chunk, (c+1)*chunk) of row v / C
   // (C = ceil(n_cols / chunk), c = v % C), n_valid counted from c*chunk.
   // map != NULL: the emitted value of column i is map[row * map_ld + i].
@@ -419,13 +423,15 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     const float smp = smp_next;
     int32_t* dst = idx_out + (long long)row * k;
     const int32_t* mrow = map ? map + (long long)row * map_ld : nullptr;
-    if (row + (int)gridDim.x < rows && n <= k) {
+    const bool skip = n <= k || n > code_cap;          // nothing to select (or no room for the codes)
+    if (row + (int)gridDim.x < rows && skip) {
       const float* s2;
       const int n2 = setup(row + gridDim.x, &s2);
       smp_next = sample(s2, n2);
     }
-    if (n <= k) {
-      for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = i < n ? (mrow ? mrow[i] : i) : -1;
+    if (skip) {
+      if (n > code_cap && threadIdx.x == 0) report(LCSA_DEV_BAD_INDEX);
+      for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = (i < n && n <= k) ? (mrow ? mrow[i] : i) : -1;
       continue;                                        // no shared memory touched: no barrier needed
     }
     // ---- bucket range from the sample
@@ -550,15 +556,26 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
             rank += (kj > key || (kj == key && j < lane)) ? 1u : 0u;
           }
           if (have) s_code[s_lidx[lane]] = rank < kr ? kTk2Sel : (uint16_t)0;
-          const uint32_t sel = __ballot_sync(0xffffffffu, have && rank < kr);
           if (have && rank < kr) atomicAdd(&s_wa[s_lidx[lane] / seg], 1u);
-          (void)sel;
+        }
+      } else if (cnt <= (uint32_t)kTk2Threads) {
+        // one entry per thread, ranked against the whole list
+        const int t = threadIdx.x;
+        if (t < (int)cnt) {
+          const uint32_t key = s_lkey[t];
+          uint32_t rank = 0;
+          for (int j = 0; j < (int)cnt; ++j) {
+            const uint32_t kj = s_lkey[j];
+            rank += (kj > key || (kj == key && j < t)) ? 1u : 0u;
+          }
+          s_code[s_lidx[t]] = rank < kr ? kTk2Sel : (uint16_t)0;
+          if (rank < kr) atomicAdd(&s_wa[s_lidx[t] / seg], 1u);
         }
       } else {
         if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = kr; }
         __syncthreads();
-        tk2_radix([&](int c, uint32_t* key) { *key = s_lkey[c]; return true; }, (int)cnt, s_hist, &s_st, s_warp,
-                  &s_total, &s_bincnt);
+        tk2_radix<kTk2Threads>([&](int c, uint32_t* key) { *key = s_lkey[c]; return true; }, (int)cnt, s_hist, &s_st,
+                               s_warp, &s_total, &s_bincnt);
         const uint32_t T = s_st.prefix, rT = s_st.kr;  // keep every key > T and the first rT copies of T
         // list order is index order: the first rT ties win
         if (threadIdx.x == 0) s_total = 0u;
@@ -583,7 +600,7 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
       // (scores of the pivot bucket re-read from global memory)
       if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = kr; }
       __syncthreads();
-      tk2_radix(
+      tk2_radix<kTk2Threads>(
           [&](int c, uint32_t* key) {
             if (s_code[c] != bpiv) return false;
             *key = score_key(__ldg(src + c));
@@ -675,58 +692,77 @@ static size_t topk_long_scratch(int rows, int n_cols, int k) {
 }
 
 // Union of the chunk selections, compacted in column order: scores, columns
-// and the count per row.  One block per row.
+// and the count per row.  One block per (row, chunk); a chunk's offset
+// follows from the row's count alone.
 __global__ void __launch_bounds__(256)
 topk_gather_kernel(const float* __restrict__ scores, long long ld, int n_cols, const int32_t* __restrict__ n_valid,
                    int k, int C, const int32_t* __restrict__ local, float* __restrict__ cs, int32_t* __restrict__ ci,
                    int32_t* __restrict__ cn) {
-  const int r = blockIdx.x;
+  const int r = blockIdx.x / C, c = blockIdx.x - (blockIdx.x / C) * C;
   int n = n_cols;
   if (n_valid != nullptr) {
     n = n_valid[r];
     n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
   }
-  int off = 0;
-  for (int c = 0; c < C; ++c) {
-    int nc = n - c * kTkChunk;
+  auto count = [&](int cc) {
+    int nc = n - cc * kTkChunk;
     nc = nc < 0 ? 0 : (nc > kTkChunk ? kTkChunk : nc);
-    const int cnt = nc < k ? nc : k;
-    const int32_t* lrow = local + ((long long)r * C + c) * k;
-    for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
-      const int col = c * kTkChunk + lrow[j];
-      cs[(long long)r * C * k + off + j] = scores[(long long)r * ld + col];
-      ci[(long long)r * C * k + off + j] = col;
-    }
-    off += cnt;
+    return nc < k ? nc : k;
+  };
+  int off = 0;
+  for (int cc = 0; cc < c; ++cc) off += count(cc);
+  const int cnt = count(c);
+  const int32_t* lrow = local + ((long long)r * C + c) * k;
+  for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
+    const int col = c * kTkChunk + lrow[j];
+    cs[(long long)r * C * k + off + j] = scores[(long long)r * ld + col];
+    ci[(long long)r * C * k + off + j] = col;
   }
-  if (threadIdx.x == 0) cn[r] = off;
+  if (c == C - 1 && threadIdx.x == 0) cn[r] = off + cnt;
+}
+
+template <int NT>
+static cudaError_t launch_topk_smem_nt(const float* scores, int rows, int n_cols, long long ld,
+                                       const int32_t* n_valid, int k, int32_t* idx_out, int chunk,
+                                       const int32_t* map, long long map_ld, cudaStream_t st, int cap8) {
+  const size_t smem = (size_t)(cap8 > 8 ? cap8 : 8) * 2;
+  cudaError_t e = cudaFuncSetAttribute(topk_smem_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxCachedKeys * 2);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_smem_kernel<NT>, NT, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const long long slots = (long long)sms * per_sm;
+  const int grid = rows < slots ? rows : (int)slots;
+  count_launch();
+  topk_smem_kernel<NT><<<grid, NT, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out, rows, chunk, map, map_ld,
+                                               cap8);
+  return cudaGetLastError();
 }
 
 static cudaError_t launch_topk_smem(const float* scores, int rows, int n_cols, long long ld, const int32_t* n_valid,
                                     int k, int32_t* idx_out, int chunk, const int32_t* map, long long map_ld,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, int n_max = -1) {
   const int width = chunk > 0 ? chunk : n_cols;
-  const size_t smem = (size_t)((width + 7) & ~7) * 2;
-  cudaError_t e = cudaFuncSetAttribute(topk_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kMaxCachedKeys * 2);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = rows < 2 * sms ? rows : 2 * sms;
-  count_launch();
-  topk_smem_kernel<<<grid, kTk2Threads, smem, st>>>(scores, ld, n_cols, n_valid, k, idx_out, rows, chunk, map,
-                                                    map_ld);
-  return cudaGetLastError();
+  const int cap = n_max >= 0 && n_max < width ? n_max : width;   // longest row of this launch
+  const int cap8 = (cap + 7) & ~7;
+  if (cap8 <= 16384)
+    return launch_topk_smem_nt<256>(scores, rows, n_cols, ld, n_valid, k, idx_out, chunk, map, map_ld, st, cap8);
+  return launch_topk_smem_nt<512>(scores, rows, n_cols, ld, n_valid, k, idx_out, chunk, map, map_ld, st, cap8);
 }
 
 // `scratch` (topk_long_scratch bytes, 256-byte aligned) enables the two-phase
 // path for long rows; without it long rows use topk_rows_kernel.
+// n_max >= 0: no row of this call has more than n_max valid columns (sizes
+// the shared-memory code buffer; -1 = n_cols).
 static cudaError_t launch_topk(const float* scores, int rows, int n_cols, long long ld, const int32_t* n_valid,
                                int k, int32_t* idx_out, cudaStream_t st, void* scratch = nullptr,
-                               size_t scratch_bytes = 0) {
+                               size_t scratch_bytes = 0, int n_max = -1) {
   if (rows == 0) return cudaSuccess;
   if (topk_smem_ok(scores, n_cols, ld))
-    return launch_topk_smem(scores, rows, n_cols, ld, n_valid, k, idx_out, 0, nullptr, 0, st);
+    return launch_topk_smem(scores, rows, n_cols, ld, n_valid, k, idx_out, 0, nullptr, 0, st, n_max);
   const int C = topk_long_chunks(n_cols, k);
   const size_t need = topk_long_scratch(rows, n_cols, k);
   if (C > 0 && scratch != nullptr && need > 0 && scratch_bytes >= need && (ld & 3) == 0 &&
@@ -741,7 +777,7 @@ static cudaError_t launch_topk(const float* scores, int rows, int n_cols, long l
     cudaError_t e = launch_topk_smem(scores, rows * C, n_cols, ld, n_valid, k, local, kTkChunk, nullptr, 0, st);
     if (e != cudaSuccess) return e;
     count_launch();
-    topk_gather_kernel<<<rows, 256, 0, st>>>(scores, ld, n_cols, n_valid, k, C, local, cs, ci, cn);
+    topk_gather_kernel<<<rows * C, 256, 0, st>>>(scores, ld, n_cols, n_valid, k, C, local, cs, ci, cn);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_topk_smem(cs, rows, C * k, (long long)C * k, cn, k, idx_out, 0, ci, (long long)C * k, st);
