@@ -104,6 +104,11 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// Prefetch `bytes` (multiple of 16, 16-byte aligned address) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
 // Named barrier over `n` threads that also ANDs a predicate across them.
 __device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
   uint32_t r;

@@ -483,6 +483,12 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
           }
       }
     }
+    // the next row's scores into L2 while this row is resolved and emitted
+    if (threadIdx.x == 0 && row + (int)gridDim.x < rows) {
+      const float* s2;
+      const int n2 = setup(row + gridDim.x, &s2);
+      if (n2 > k && n2 <= code_cap && n2 >= 4) tc::bulk_prefetch_l2(s2, (uint32_t)(n2 & ~3) * 4u);
+    }
     __syncthreads();
     topk_pick_bin<kTk2Threads>(s_hist, kTk2Bins, 0, 0x7FFu, &s_st, s_warp, &s_total, &s_bincnt);
     const uint32_t bpiv = s_st.prefix, kr = s_st.kr, cnt = s_bincnt;
