@@ -382,11 +382,11 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
   // (C = ceil(n_cols / chunk), c = v % C), n_valid counted from c*chunk.
   // map != NULL: the emitted value of column i is map[row * map_ld + i].
   extern __shared__ __align__(16) uint16_t s_code[];   // bucket code of every score of the row
-  __shared__ uint32_t s_hist[kTk2Bins];
+  __shared__ __align__(16) uint32_t s_hist[kTk2Bins];
   __shared__ uint32_t s_lkey[kTk2List];
   __shared__ int32_t s_lidx[kTk2List];
   __shared__ uint32_t s_warp[32];
-  __shared__ uint32_t s_total, s_bincnt;
+  __shared__ uint32_t s_total, s_bincnt, s_nlist;
   __shared__ uint32_t s_wa[kTk2Warps], s_we[kTk2Warps];
   __shared__ float s_lo[kTk2Warps], s_hi[kTk2Warps];
   __shared__ TopkState s_st;
@@ -423,12 +423,12 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     const float smp = smp_next;
     int32_t* dst = idx_out + (long long)row * k;
     const int32_t* mrow = map ? map + (long long)row * map_ld : nullptr;
+    // the next row of this CTA (its count is a global load: issued early)
+    const bool has_next = row + (int)gridDim.x < rows;
+    const float* src2 = nullptr;
+    const int n2 = has_next ? setup(row + gridDim.x, &src2) : 0;
     const bool skip = n <= k || n > code_cap;          // nothing to select (or no room for the codes)
-    if (row + (int)gridDim.x < rows && skip) {
-      const float* s2;
-      const int n2 = setup(row + gridDim.x, &s2);
-      smp_next = sample(s2, n2);
-    }
+    if (has_next && skip) smp_next = sample(src2, n2);
     if (skip) {
       if (n > code_cap && threadIdx.x == 0) report(LCSA_DEV_BAD_INDEX);
       for (int i = threadIdx.x; i < k; i += kTk2Threads) dst[i] = (i < n && n <= k) ? (mrow ? mrow[i] : i) : -1;
@@ -458,24 +458,27 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
       const float x = (v - lo) * scale;                 // monotone in v; NaN-free rows
       return x <= 0.f ? 0u : (x >= (float)(kTk2Bins - 1) ? (uint32_t)(kTk2Bins - 1) : (uint32_t)x);
     };
-    // contiguous warp segments [seg_lo, seg_hi), lengths multiples of 128
-    const int seg = ((n + kTk2Warps - 1) / kTk2Warps + 127) & ~127;
+    // contiguous warp segments [seg_lo, seg_hi), lengths multiples of 256:
+    // lane L owns elements 8L .. 8L+7 of each 256-element step
+    const int seg = ((n + kTk2Warps - 1) / kTk2Warps + 255) & ~255;
     const int seg_lo = warp * seg < n ? warp * seg : n;
     const int seg_hi = seg_lo + seg < n ? seg_lo + seg : n;
 
     // ---- pass 1: stream the row, bucket histogram and codes
-#pragma unroll 4
-    for (int base = seg_lo; base < seg_hi; base += 128) {
-      const int i0 = base + 4 * lane;
-      uint32_t b[4];
-      if (i0 + 3 < seg_hi) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(src + i0));
-        b[0] = bucket(v.x); b[1] = bucket(v.y); b[2] = bucket(v.z); b[3] = bucket(v.w);
+#pragma unroll 2
+    for (int base = seg_lo; base < seg_hi; base += 256) {
+      const int i0 = base + 8 * lane;
+      if (i0 + 7 < seg_hi) {
+        const float4 v0 = __ldg(reinterpret_cast<const float4*>(src + i0));
+        const float4 v1 = __ldg(reinterpret_cast<const float4*>(src + i0 + 4));
+        const uint32_t b[8] = {bucket(v0.x), bucket(v0.y), bucket(v0.z), bucket(v0.w),
+                               bucket(v1.x), bucket(v1.y), bucket(v1.z), bucket(v1.w)};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) atomicAdd(&s_hist[b[q]], 1u);
-        *reinterpret_cast<uint2*>(s_code + i0) = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+        for (int q = 0; q < 8; ++q) atomicAdd(&s_hist[b[q]], 1u);
+        *reinterpret_cast<uint4*>(s_code + i0) =
+            make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
       } else {
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (i0 + q < seg_hi) {
             const uint32_t bq = bucket(__ldg(src + i0 + q));
             atomicAdd(&s_hist[bq], 1u);
@@ -484,121 +487,144 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
       }
     }
     // the next row's scores into L2 while this row is resolved and emitted
-    if (threadIdx.x == 0 && row + (int)gridDim.x < rows) {
-      const float* s2;
-      const int n2 = setup(row + gridDim.x, &s2);
-      if (n2 > k && n2 <= code_cap && n2 >= 4) tc::bulk_prefetch_l2(s2, (uint32_t)(n2 & ~3) * 4u);
+    if (threadIdx.x == 0 && has_next && n2 > k && n2 <= code_cap && n2 >= 4)
+      tc::bulk_prefetch_l2(src2, (uint32_t)(n2 & ~3) * 4u);
+    __syncthreads();
+    // bucket of the k-th score, by one warp: lane L sums buckets
+    // 2047-64L .. 1984-64L, a warp scan from the top finds the lane and that
+    // lane the bucket; rank kr inside it, its count cnt
+    if (warp == 0) {
+      const int top = kTk2Bins - 1 - 64 * lane;
+      uint32_t sum = 0;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4*>(s_hist + top - 63 + 4 * q);
+        sum += v.x + v.y + v.z + v.w;
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      // the lane whose 64 buckets hold the k-th score (exactly one)
+      const uint32_t hit = __ballot_sync(0xffffffffu, excl < (uint32_t)k && incl >= (uint32_t)k);
+      const int hl = __ffs(hit) - 1;
+      const uint32_t cum0 = __shfl_sync(0xffffffffu, excl, hl);
+      // its buckets, two per lane from the top: lane L takes 2L and 2L+1
+      const int t0 = kTk2Bins - 1 - 64 * hl - 2 * lane;
+      const uint32_t c0 = s_hist[t0], c1 = s_hist[t0 - 1];
+      const uint32_t pair = c0 + c1;
+      uint32_t pin = pair;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, pin, o);
+        if (lane >= o) pin += y;
+      }
+      const uint32_t pex = cum0 + pin - pair;         // scores in buckets above t0
+      if (pex < (uint32_t)k && pex + pair >= (uint32_t)k) {   // exactly one lane
+        if (pex + c0 >= (uint32_t)k) { s_st.prefix = (uint32_t)t0; s_st.kr = (uint32_t)k - pex; s_bincnt = c0; }
+        else { s_st.prefix = (uint32_t)(t0 - 1); s_st.kr = (uint32_t)k - pex - c0; s_bincnt = c1; }
+      }
+      if (lane == 0) s_nlist = 0u;
     }
     __syncthreads();
-    topk_pick_bin<kTk2Threads>(s_hist, kTk2Bins, 0, 0x7FFu, &s_st, s_warp, &s_total, &s_bincnt);
     const uint32_t bpiv = s_st.prefix, kr = s_st.kr, cnt = s_bincnt;
     const bool fits = cnt <= (uint32_t)kTk2List;
 
-    // ---- per-warp counts above / in the pivot bucket
+    // ---- per-warp counts above the pivot bucket; its scores into the list
+    // (unordered: ranks use the column as the tie break)
     {
-      uint32_t a = 0, e = 0;
-      for (int base = seg_lo; base < seg_hi; base += 128) {
-        const int i0 = base + 4 * lane;
-        if (i0 + 3 < seg_hi) {
-          const uint2 c = *reinterpret_cast<const uint2*>(s_code + i0);
-          const uint32_t cq[4] = {c.x & 0xFFFFu, c.x >> 16, c.y & 0xFFFFu, c.y >> 16};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            a += cq[q] > bpiv;
-            e += cq[q] == bpiv;
-          }
+      uint32_t a = 0;
+      for (int base = seg_lo; base < seg_hi; base += 256) {
+        const int i0 = base + 8 * lane;
+        uint32_t cq[8];
+        if (i0 + 7 < seg_hi) {
+          const uint4 c = *reinterpret_cast<const uint4*>(s_code + i0);
+          cq[0] = c.x & 0xFFFFu; cq[1] = c.x >> 16; cq[2] = c.y & 0xFFFFu; cq[3] = c.y >> 16;
+          cq[4] = c.z & 0xFFFFu; cq[5] = c.z >> 16; cq[6] = c.w & 0xFFFFu; cq[7] = c.w >> 16;
         } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (i0 + q < seg_hi) {
-              const uint32_t c = s_code[i0 + q];
-              a += c > bpiv;
-              e += c == bpiv;
-            }
-          }
+          for (int q = 0; q < 8; ++q) cq[q] = i0 + q < seg_hi ? s_code[i0 + q] : 0u;
+        }
+        uint32_t f = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          a += (i0 + q < seg_hi && cq[q] > bpiv) ? 1u : 0u;
+          f |= (uint32_t)(fits && i0 + q < seg_hi && cq[q] == bpiv) << q;
+        }
+        if (!__any_sync(0xffffffffu, f != 0u)) continue;
+        const uint32_t mine = (uint32_t)__popc(f);
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t base_slot = 0;
+        if (lane == 31) base_slot = atomicAdd(&s_nlist, incl);
+        uint32_t pos = __shfl_sync(0xffffffffu, base_slot, 31) + incl - mine;
+        while (f) {
+          const int q = __ffs(f) - 1;
+          f &= f - 1u;
+          s_lkey[pos] = score_key(__ldg(src + i0 + q));
+          s_lidx[pos] = i0 + q;
+          ++pos;
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        a += __shfl_xor_sync(0xffffffffu, a, o);
-        e += __shfl_xor_sync(0xffffffffu, e, o);
-      }
-      if (lane == 0) { s_wa[warp] = a; s_we[warp] = e; }
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) s_wa[warp] = a;
     }
     __syncthreads();
 
     if (fits) {
-      // ---- the pivot bucket's scores, in index order, into the list
-      uint32_t off = 0;
-      for (int w = 0; w < warp; ++w) off += s_we[w];
-      if (s_we[warp] > 0) {
-        for (int base = seg_lo; base < seg_hi; base += 128) {
-          const int i0 = base + 4 * lane;
-          uint32_t f = 0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] == bpiv) << q;
-          if (!__any_sync(0xffffffffu, f != 0u)) continue;
-          uint32_t tot;
-          uint32_t pos = off + warp_excl_count4(f, &tot);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if ((f >> q) & 1u) {
-              s_lkey[pos] = score_key(__ldg(src + i0 + q));
-              s_lidx[pos] = i0 + q;
-              ++pos;
-            }
-          off += tot;
-        }
-      }
-      __syncthreads();
-      // ---- exact top kr of the list (ties to the lower index, i.e. list order)
+      // ---- exact top kr of the list in (key desc, column asc) order
       if (cnt <= 32) {
         if (warp == 0) {
           const bool have = lane < (int)cnt;
           const uint32_t key = have ? s_lkey[lane] : 0u;
-          uint32_t rank = 0;                           // list entries before this one in (key desc, index asc)
+          const int32_t col = have ? s_lidx[lane] : 0;
+          uint32_t rank = 0;
           for (int j = 0; j < (int)cnt; ++j) {
             const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
-            rank += (kj > key || (kj == key && j < lane)) ? 1u : 0u;
+            const int32_t cj = __shfl_sync(0xffffffffu, col, j);
+            rank += (kj > key || (kj == key && cj < col)) ? 1u : 0u;
           }
-          if (have) s_code[s_lidx[lane]] = rank < kr ? kTk2Sel : (uint16_t)0;
-          if (have && rank < kr) atomicAdd(&s_wa[s_lidx[lane] / seg], 1u);
+          if (have) s_code[col] = rank < kr ? kTk2Sel : (uint16_t)0;
+          if (have && rank < kr) atomicAdd(&s_wa[col / seg], 1u);
         }
       } else if (cnt <= (uint32_t)kTk2Threads) {
-        // one entry per thread, ranked against the whole list
         const int t = threadIdx.x;
         if (t < (int)cnt) {
           const uint32_t key = s_lkey[t];
+          const int32_t col = s_lidx[t];
           uint32_t rank = 0;
           for (int j = 0; j < (int)cnt; ++j) {
             const uint32_t kj = s_lkey[j];
-            rank += (kj > key || (kj == key && j < t)) ? 1u : 0u;
+            rank += (kj > key || (kj == key && s_lidx[j] < col)) ? 1u : 0u;
           }
-          s_code[s_lidx[t]] = rank < kr ? kTk2Sel : (uint16_t)0;
-          if (rank < kr) atomicAdd(&s_wa[s_lidx[t] / seg], 1u);
+          s_code[col] = rank < kr ? kTk2Sel : (uint16_t)0;
+          if (rank < kr) atomicAdd(&s_wa[col / seg], 1u);
         }
       } else {
         if (threadIdx.x == 0) { s_st.prefix = 0u; s_st.mask = 0u; s_st.kr = kr; }
         __syncthreads();
         tk2_radix<kTk2Threads>([&](int c, uint32_t* key) { *key = s_lkey[c]; return true; }, (int)cnt, s_hist, &s_st,
                                s_warp, &s_total, &s_bincnt);
-        const uint32_t T = s_st.prefix, rT = s_st.kr;  // keep every key > T and the first rT copies of T
-        // list order is index order: the first rT ties win
-        if (threadIdx.x == 0) s_total = 0u;
-        __syncthreads();
-        for (int c0 = 0; c0 < (int)cnt; c0 += kTk2Threads) {
-          const int c = c0 + threadIdx.x;
-          const uint32_t key = c < (int)cnt ? s_lkey[c] : 0u;
-          const bool tie = c < (int)cnt && key == T;
-          const uint32_t tie_before = block_excl_scan<kTk2Threads>(tie ? 1u : 0u, s_warp, &s_bincnt) + s_total;
-          if (c < (int)cnt) {
-            const bool sel = key > T || (tie && tie_before < rT);
-            s_code[s_lidx[c]] = sel ? kTk2Sel : (uint16_t)0;
-            if (sel) atomicAdd(&s_wa[s_lidx[c] / seg], 1u);
+        const uint32_t T = s_st.prefix, rT = s_st.kr;  // keep every key > T and the rT lowest columns of T
+        for (int c = threadIdx.x; c < (int)cnt; c += kTk2Threads) {
+          const uint32_t key = s_lkey[c];
+          const int32_t col = s_lidx[c];
+          bool sel = key > T;
+          if (key == T) {
+            uint32_t before = 0;
+            for (int j = 0; j < (int)cnt; ++j) before += (s_lkey[j] == T && s_lidx[j] < col) ? 1u : 0u;
+            sel = before < rT;
           }
-          __syncthreads();
-          if (threadIdx.x == 0) s_total += s_bincnt;
-          __syncthreads();
+          s_code[col] = sel ? kTk2Sel : (uint16_t)0;
+          if (sel) atomicAdd(&s_wa[col / seg], 1u);
         }
       }
     } else {
@@ -642,33 +668,38 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     }
     __syncthreads();
 
-    if (row + (int)gridDim.x < rows) {                 // next row's sample, in flight during the emission
-      const float* s2;
-      const int n2 = setup(row + gridDim.x, &s2);
-      smp_next = sample(s2, n2);
-    }
+    if (has_next) smp_next = sample(src2, n2);         // next row's sample, in flight during the emission
     // ---- emission: the selection is {code > bpiv}, written in index order
     {
       uint32_t pos = 0;
       for (int w = 0; w < warp; ++w) pos += s_wa[w];
-      for (int base = seg_lo; base < seg_hi; base += 128) {
-        const int i0 = base + 4 * lane;
+      for (int base = seg_lo; base < seg_hi; base += 256) {
+        const int i0 = base + 8 * lane;
         uint32_t f = 0;
-        if (i0 + 3 < seg_hi) {
-          const uint2 c = *reinterpret_cast<const uint2*>(s_code + i0);
+        if (i0 + 7 < seg_hi) {
+          const uint4 c = *reinterpret_cast<const uint4*>(s_code + i0);
           f = (uint32_t)((c.x & 0xFFFFu) > bpiv) | ((uint32_t)((c.x >> 16) > bpiv) << 1) |
-              ((uint32_t)((c.y & 0xFFFFu) > bpiv) << 2) | ((uint32_t)((c.y >> 16) > bpiv) << 3);
+              ((uint32_t)((c.y & 0xFFFFu) > bpiv) << 2) | ((uint32_t)((c.y >> 16) > bpiv) << 3) |
+              ((uint32_t)((c.z & 0xFFFFu) > bpiv) << 4) | ((uint32_t)((c.z >> 16) > bpiv) << 5) |
+              ((uint32_t)((c.w & 0xFFFFu) > bpiv) << 6) | ((uint32_t)((c.w >> 16) > bpiv) << 7);
         } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] > bpiv) << q;
+          for (int q = 0; q < 8; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] > bpiv) << q;
         }
-        if (!__any_sync(0xffffffffu, f != 0u)) continue;
-        uint32_t tot;
-        uint32_t p = pos + warp_excl_count4(f, &tot);
+        const uint32_t mine = (uint32_t)__popc(f);
+        uint32_t incl = mine;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if ((f >> q) & 1u) dst[p++] = mrow ? mrow[i0 + q] : i0 + q;
-        pos += tot;
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t p = pos + incl - mine;
+        while (f) {
+          const int q = __ffs(f) - 1;
+          f &= f - 1u;
+          dst[p++] = mrow ? mrow[i0 + q] : i0 + q;
+        }
+        pos += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
     __syncthreads();                                    // codes and counters are reused by the next row

@@ -108,6 +108,30 @@ def test_topk_long_rows_both_paths(lcsa, n_cols, k, ties):
     assert (lcsa.topk_workspace_bytes(rows, n_cols, k) > 0) == (k % 4 == 0)
 
 
+@pytest.mark.parametrize("n_cols", [8000, 20000])
+def test_topk_pivot_bucket_sizes(lcsa, n_cols):
+    """Rows built so that the k-th score sits inside a tight cluster of c
+    scores (one value bucket): c = 20, 150, 600 and 3000 reach the one-warp,
+    one-thread-per-entry, radix and whole-row resolutions of that bucket; the
+    second half of the rows repeats values inside the cluster (ties)."""
+    k = 2048
+    g = np.random.default_rng(11)
+    rows = []
+    for ties in (False, True):
+        for c in (20, 150, 600, 3000):
+            r = g.standard_normal(n_cols).astype(np.float32)
+            above = k - c // 2                               # scores above the cluster
+            pos = g.permutation(n_cols)
+            r[pos[:above]] = 20.0 + g.random(above).astype(np.float32)
+            jit = (np.arange(c) % 7 if ties else np.arange(c)).astype(np.float32) * np.float32(1e-6)
+            r[pos[above:above + c]] = np.float32(10.0) + jit
+            rows.append(r)
+    s = torch.tensor(np.stack(rows), device=DEV)
+    idx = lcsa.topk_from_scores(s, k)
+    ref = O.topk_from_scores(s.cpu().double().numpy(), [n_cols] * len(rows), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
 def test_topk_skewed_rows(lcsa):
     """Rows whose value range is dominated by outliers (one sampled bucket
     holds nearly everything), infinities and constant rows."""
