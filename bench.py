@@ -511,9 +511,35 @@ def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
                         "bytes_per_step": byts, "peak_source": f"hbm_gbs of {peaks['source']}",
                         "note": "whole decode step (indexer keys + gathered rows + window + q/out)"},
-           "gpu_launches": int(launches), "clocks": clocks}
+           "gpu_launches": int(launches), "clocks": clocks,
+           "compress_append_us": append_cost(lcsa, cfg, B, ckv, t, g, dev)}
     del ix, ckv, q, kvw, idx, out, ws_ix, ws_at
     torch.cuda.empty_cache()
+    return res
+
+
+def append_cost(lcsa, cfg, B, ckv, t, g, dev, reps=20):
+    """Incremental compression after token t-1: the CSA entry t/m-1 (window
+    2m) into the decode cache and the HCA entry t/m'-1 (window m') into an HCA
+    cache, both from a ring of the last 128 raw rows; microseconds per call for
+    the whole batch (not part of the timed decode step)."""
+    W = 128
+    ring_kv = gen._randn((B, W, cfg.D), g, dev, 1.0 / math.sqrt(cfg.D), torch.bfloat16)
+    ring_g = gen._randn((B, W, cfg.D), g, dev, 1.0, torch.bfloat16)
+    hca = torch.empty((B, t // cfg.m_hca, cfg.D), dtype=torch.bfloat16, device=dev)
+    res = {}
+    for name, m, window, cache in (("csa", cfg.m, 2 * cfg.m, ckv), ("hca", cfg.m_hca, cfg.m_hca, hca)):
+        call = lambda: lcsa.compress_entries(ring_kv, ring_g, t - W, m, window, t // m - 1, 1, cache)
+        for _ in range(3):
+            call()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        res[name] = round(a.elapsed_time(b) * 1e3 / reps, 2)
+    del ring_kv, ring_g, hca
     return res
 
 

@@ -103,6 +103,34 @@ lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_cha
                               void* out, lcsa_dtype out_dtype, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Incremental KV compression for decode: the pooling above, for the entries
+ * whose windows a buffer of recent raw rows covers.  A decode loop appends
+ * entry j = t/m - 1 of a CSA or HCA cache once the token at position t-1 has
+ * arrived and t % m == 0 (the pages' m-token compression applied as tokens
+ * arrive; the window ring of raw rows kept for the sliding-window branch
+ * holds every token such an entry needs when W >= window).
+ *
+ * Computes c[b,j,:] for j in [j0, j0 + n_entries) with
+ *   S_j = [(j+1)m - window, (j+1)m) clipped at 0
+ * (window 2m for CSA, m for HCA; any window >= 1).  Buffer row i of every
+ * sequence holds position kv_pos0 + i, and every position of every S_j must
+ * lie in [kv_pos0, kv_pos0 + Tkv).
+ *
+ *   kv    [B,Tkv,D] dtype          gate [B,Tkv,D] dtype (gate_per_channel=1)
+ *                                  or [B,Tkv] dtype (=0)
+ *   cache [B,cache_rows,D] out_dtype; entry j is written at row j, nothing
+ *         else is touched
+ * Returns LCSA_ERR_INVALID_ARG when a window leaves the buffer, when
+ * j0 < 0 or j0 + n_entries > cache_rows, or on the layout constraints of
+ * lcsa_csa_compress.  Buffers are caller-owned; the call is stream-ordered.
+ * ------------------------------------------------------------------------ */
+lcsa_status lcsa_compress_entries(const void* kv, const void* gate, int gate_per_channel,
+                                  int B, int Tkv, int D, int64_t kv_pos0, int m, int window,
+                                  int64_t j0, int n_entries, lcsa_dtype dtype,
+                                  const float* rms_weight, float rms_eps,
+                                  void* cache, int64_t cache_rows, lcsa_dtype out_dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * Top-k selection ([p2] CSA Step 2 and its ASCII figure: keep only the top-k
  * scored entries; [p1] section 1: the top 2048 blocks).
  *

@@ -27,6 +27,7 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported combination", 3: "wor
 EXPORTED = [
     "lcsa_version", "lcsa_status_string", "lcsa_get_device_status", "lcsa_kernel_launches",
     "lcsa_csa_compress", "lcsa_hca_compress",
+    "lcsa_compress_entries",
     "lcsa_topk_workspace", "lcsa_topk_from_scores",
     "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
     "lcsa_indexer_topk_noalloc",
@@ -69,6 +70,8 @@ _sig = {
     "lcsa_get_device_status": (_i, [_vp, ctypes.POINTER(_i)]),
     "lcsa_csa_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
     "lcsa_hca_compress": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _i, _vp]),
+    "lcsa_compress_entries": (_i, [_vp, _vp, _i, _i, _i, _i, _i64, _i, _i, _i64, _i, _i, _vp, ctypes.c_float, _vp,
+                                   _i64, _i, _vp]),
     "lcsa_topk_workspace": (_sz, [_i, _i, _i]),
     "lcsa_topk_from_scores": (_i, [_vp, _i, _i, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
     "lcsa_indexer_topk_workspace": (_sz, [ctypes.POINTER(IndexerArgs)]),
@@ -161,6 +164,21 @@ def hca_compress(kv, gate, m=128, out_dtype=None, rms_weight=None, rms_eps=1e-6,
 
 
 # ----------------------------------------------------------------- top-k
+def compress_entries(kv, gate, kv_pos0, m, window, j0, n_entries, cache, rms_weight=None, rms_eps=1e-6):
+    """Entries j0 .. j0+n_entries-1 of a compressed cache from a buffer of raw
+    rows: kv [B,Tkv,D] holds positions kv_pos0 .. kv_pos0+Tkv-1, gate
+    [B,Tkv,D] or [B,Tkv]; window 2m (CSA) or m (HCA); written into cache
+    [B,cache_rows,D] at rows j (incremental decode compression)."""
+    _need_contig(kv, gate, cache)
+    B, Tkv, D = kv.shape
+    per_channel = 1 if gate.dim() == 3 else 0
+    st = _lib.lcsa_compress_entries(_p(kv), _p(gate), per_channel, B, Tkv, D, int(kv_pos0), m, window, int(j0),
+                                    n_entries, _dt(kv), _p(rms_weight), float(rms_eps), _p(cache), cache.shape[1],
+                                    _dt(cache), _stream(kv.device))
+    _check(st, "compress_entries")
+    return cache
+
+
 def topk_workspace_bytes(rows, n_cols, k):
     """Scratch that lets rows longer than 32768 columns take the two-phase path."""
     return int(_lib.lcsa_topk_workspace(rows, n_cols, k))

@@ -13,19 +13,25 @@
 
 namespace lcsa {
 
+// Entries j = j0 .. j0+Nc-1 of every sequence; the token buffer holds T rows
+// per sequence for positions kv_pos0 .. kv_pos0+T-1 (every token of every
+// computed window must be inside it); entry j is written at row j of an
+// output of out_rows rows per sequence.
 template <typename Tin, typename Tout, bool kPerChannelGate>
 __global__ void __launch_bounds__(256)
 compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* __restrict__ out,
                 int T, int D, int m, int window, int Nc, int entries_per_block,
-                const float* __restrict__ rms_w, float rms_eps) {
+                const float* __restrict__ rms_w, float rms_eps, long long j0, long long kv_pos0,
+                long long out_rows) {
   constexpr int V = Elem<Tin>::kVec;
   const int tpe = D / V;                         // threads per entry
   const int e_local = threadIdx.x / tpe;
   const int c = threadIdx.x - e_local * tpe;     // channel vector index
   const int b = blockIdx.y;
-  const int j = blockIdx.x * entries_per_block + e_local;
+  const int jr = blockIdx.x * entries_per_block + e_local;   // entry relative to j0
+  const long long j = j0 + jr;
   extern __shared__ float s_ss[];                // [entries_per_block] sum of squares
-  const bool active = (e_local < entries_per_block) && (j < Nc);
+  const bool active = (e_local < entries_per_block) && (jr < Nc);
   if (rms_w != nullptr && threadIdx.x < entries_per_block) s_ss[threadIdx.x] = 0.f;
 
   float acc[V], run_max[V], run_sum[V];
@@ -33,8 +39,8 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
   for (int v = 0; v < V; ++v) { acc[v] = 0.f; run_max[v] = -INFINITY; run_sum[v] = 0.f; }
 
   if (active) {
-    const long long hi = (long long)(j + 1) * m;
-    const long long lo = hi - window > 0 ? hi - window : 0;
+    const long long hi = (j + 1) * m - kv_pos0;                     // buffer rows
+    const long long lo = (j + 1) * m - window > 0 ? (j + 1) * m - window - kv_pos0 : -kv_pos0;
     const Tin* kvb = kv + ((long long)b * T) * D + (long long)c * V;
     const Tin* gb = kPerChannelGate ? gate + ((long long)b * T) * D + (long long)c * V
                                     : gate + (long long)b * T;
@@ -92,7 +98,7 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
     }
   }
   if (active) {
-    Tout* o = out + ((long long)b * Nc + j) * D + (long long)c * V;
+    Tout* o = out + ((long long)b * out_rows + j) * D + (long long)c * V;
     store_vec<V>(o, acc);
   }
 }
@@ -100,9 +106,11 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
 template <typename Tin, typename Tout>
 static cudaError_t launch_compress_t(const void* kv, const void* gate, int per_channel, int B, int T, int D,
                                      int m, int window, const float* rms_w, float rms_eps, void* out,
-                                     cudaStream_t st) {
+                                     cudaStream_t st, long long j0 = 0, int n_entries = -1, long long kv_pos0 = 0,
+                                     long long out_rows = -1) {
   constexpr int V = Elem<Tin>::kVec;
-  const int Nc = T / m;
+  const int Nc = n_entries >= 0 ? n_entries : T / m;
+  if (out_rows < 0) out_rows = Nc;
   if (Nc == 0 || B == 0) return cudaSuccess;
   const int tpe = D / V;
   int epb = 256 / tpe;
@@ -113,24 +121,31 @@ static cudaError_t launch_compress_t(const void* kv, const void* gate, int per_c
   count_launch();
   if (per_channel)
     compress_kernel<Tin, Tout, true><<<grid, threads, smem, st>>>(
-        (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, window, Nc, epb, rms_w, rms_eps);
+        (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, window, Nc, epb, rms_w, rms_eps, j0, kv_pos0,
+        out_rows);
   else
     compress_kernel<Tin, Tout, false><<<grid, threads, smem, st>>>(
-        (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, window, Nc, epb, rms_w, rms_eps);
+        (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, window, Nc, epb, rms_w, rms_eps, j0, kv_pos0,
+        out_rows);
   return cudaGetLastError();
 }
 
 static cudaError_t launch_compress(const void* kv, const void* gate, int per_channel, int B, int T, int D,
                                    int m, int window, lcsa_dtype dt, const float* rms_w, float rms_eps,
-                                   void* out, lcsa_dtype odt, cudaStream_t st) {
+                                   void* out, lcsa_dtype odt, cudaStream_t st, long long j0 = 0,
+                                   int n_entries = -1, long long kv_pos0 = 0, long long out_rows = -1) {
   if (dt == LCSA_BF16) {
     if (odt == LCSA_BF16)
-      return launch_compress_t<__nv_bfloat16, __nv_bfloat16>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out, st);
-    return launch_compress_t<__nv_bfloat16, float>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out, st);
+      return launch_compress_t<__nv_bfloat16, __nv_bfloat16>(kv, gate, per_channel, B, T, D, m, window, rms_w,
+                                                             rms_eps, out, st, j0, n_entries, kv_pos0, out_rows);
+    return launch_compress_t<__nv_bfloat16, float>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out,
+                                                   st, j0, n_entries, kv_pos0, out_rows);
   }
   if (odt == LCSA_BF16)
-    return launch_compress_t<float, __nv_bfloat16>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out, st);
-  return launch_compress_t<float, float>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out, st);
+    return launch_compress_t<float, __nv_bfloat16>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out,
+                                                   st, j0, n_entries, kv_pos0, out_rows);
+  return launch_compress_t<float, float>(kv, gate, per_channel, B, T, D, m, window, rms_w, rms_eps, out, st, j0,
+                                         n_entries, kv_pos0, out_rows);
 }
 
 }  // namespace lcsa

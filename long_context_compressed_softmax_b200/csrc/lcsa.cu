@@ -183,6 +183,31 @@ lcsa_status lcsa_hca_compress(const void* kv, const void* gate, int gate_per_cha
                          stream);
 }
 
+lcsa_status lcsa_compress_entries(const void* kv, const void* gate, int gate_per_channel, int B, int Tkv, int D,
+                                  int64_t kv_pos0, int m, int window, int64_t j0, int n_entries, lcsa_dtype dtype,
+                                  const float* rms_weight, float rms_eps, void* cache, int64_t cache_rows,
+                                  lcsa_dtype out_dtype, void* stream) {
+  if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return LCSA_ERR_INVALID_ARG;
+  if (B < 0 || Tkv < 0 || D <= 0 || m <= 0 || window <= 0 || kv_pos0 < 0 || j0 < 0 || n_entries < 0 ||
+      cache_rows < 0)
+    return LCSA_ERR_INVALID_ARG;
+  const int vec = dtype == LCSA_BF16 ? 8 : 4;
+  if (D % vec != 0 || D / vec > 1024) return LCSA_ERR_INVALID_ARG;
+  if (out_dtype == LCSA_BF16 && D % 8 != 0) return LCSA_ERR_INVALID_ARG;
+  if ((long long)B * n_entries == 0) return LCSA_OK;
+  if (j0 + n_entries > cache_rows) return LCSA_ERR_INVALID_ARG;
+  // windows move right with j: the first one's start and the last one's end bound them all
+  const long long first_lo = (j0 + 1) * (long long)m - window > 0 ? (j0 + 1) * (long long)m - window : 0;
+  const long long last_hi = (j0 + n_entries) * (long long)m;
+  if (first_lo < kv_pos0 || last_hi > kv_pos0 + Tkv) return LCSA_ERR_INVALID_ARG;
+  if (!kv || !gate || !cache) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(kv) || !aligned16(cache) || (gate_per_channel && !aligned16(gate))) return LCSA_ERR_INVALID_ARG;
+  if (rms_weight && (reinterpret_cast<uintptr_t>(rms_weight) & 3u)) return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  return from_cuda(launch_compress(kv, gate, gate_per_channel, B, Tkv, D, m, window, dtype, rms_weight, rms_eps,
+                                   cache, out_dtype, (cudaStream_t)stream, j0, n_entries, kv_pos0, cache_rows));
+}
+
 size_t lcsa_topk_workspace(int rows, int n_cols, int k) {
   if (rows <= 0 || n_cols <= 0 || k <= 0) return 0;
   return topk_long_scratch(rows, n_cols, k);

@@ -393,16 +393,14 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   const int C = chunk > 0 ? (n_cols + chunk - 1) / chunk : 1;
-  // scores of (virtual) row v and how many of them count
-  auto setup = [&](int v, const float** src_out) {
+  // valid-count word of (virtual) row v, loaded two rows ahead of its use
+  auto raw_n = [&](int v) { return (n_valid != nullptr && v < rows) ? n_valid[v / C] : n_cols; };
+  // scores of (virtual) row v and how many of them count, from its count word
+  auto setup = [&](int v, int raw, const float** src_out) {
     const int r = v / C, c = v - r * C;              // real row and column chunk
     const int c0 = chunk > 0 ? c * chunk : 0;
     const int width = chunk > 0 ? (n_cols - c0 < chunk ? n_cols - c0 : chunk) : n_cols;
-    int n = n_cols;
-    if (n_valid != nullptr) {
-      n = n_valid[r];
-      n = n < 0 ? 0 : (n > n_cols ? n_cols : n);
-    }
+    int n = raw < 0 ? 0 : (raw > n_cols ? n_cols : raw);
     n -= c0;
     *src_out = scores + (long long)r * ld + c0;
     return n < 0 ? 0 : (n > width ? width : n);
@@ -411,22 +409,26 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
   auto sample = [&](const float* src, int n) {
     return n > k ? __ldg(src + (int)(((long long)threadIdx.x * n) / kTk2Threads)) : 0.f;
   };
+  const int G = (int)gridDim.x;
+  int raw_cur = raw_n(blockIdx.x), raw_nxt = raw_n(blockIdx.x + G);
   float smp_next = 0.f;
   if ((int)blockIdx.x < rows) {
     const float* s0;
-    const int n0 = setup(blockIdx.x, &s0);
+    const int n0 = setup(blockIdx.x, raw_cur, &s0);
     smp_next = sample(s0, n0);
   }
-  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+  for (int row = blockIdx.x; row < rows; row += G) {
     const float* src;
-    const int n = setup(row, &src);
+    const int n = setup(row, raw_cur, &src);
     const float smp = smp_next;
     int32_t* dst = idx_out + (long long)row * k;
     const int32_t* mrow = map ? map + (long long)row * map_ld : nullptr;
-    // the next row of this CTA (its count is a global load: issued early)
-    const bool has_next = row + (int)gridDim.x < rows;
+    // the next row of this CTA, and the count word of the one after it
+    const bool has_next = row + G < rows;
     const float* src2 = nullptr;
-    const int n2 = has_next ? setup(row + gridDim.x, &src2) : 0;
+    const int n2 = has_next ? setup(row + G, raw_nxt, &src2) : 0;
+    raw_cur = raw_nxt;
+    raw_nxt = raw_n(row + 2 * G);
     const bool skip = n <= k || n > code_cap;          // nothing to select (or no room for the codes)
     if (has_next && skip) smp_next = sample(src2, n2);
     if (skip) {

@@ -89,6 +89,26 @@ def test_invalid_arguments_rejected_without_launch(lcsa):
     assert L.lcsa_indexer_topk(ctypes.byref(ia), None, 0, None) == 1         # m = 0
 
 
+def test_compress_entries_checks_windows(lcsa):
+    """Incremental compression: windows must stay inside the raw-row buffer
+    and entries inside the cache; checked before any device work."""
+    L = lcsa.lib
+    kv, g, c = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000)
+    bf = lcsa.LCSA_BF16
+    # buffer positions [120, 248): CSA entry 61 pools [240, 248) -> fine; entry 29 pools [112, 120) -> outside
+    args = lambda j0, n, rows, pos0=120, window=8: (kv, g, 1, 1, 128, 512, pos0, 4, window, j0, n, bf, None, 0.0, c,
+                                                    rows, bf, None)
+    assert L.lcsa_compress_entries(*args(29, 1, 64)) == 1              # window starts before the buffer
+    assert L.lcsa_compress_entries(*args(62, 1, 64)) == 1              # window ends after the buffer
+    assert L.lcsa_compress_entries(*args(61, 1, 61)) == 1              # entry beyond the cache
+    assert L.lcsa_compress_entries(*args(-1, 1, 64)) == 1              # negative first entry
+    assert L.lcsa_compress_entries(*args(61, 1, 64, window=0)) == 1    # empty window
+    assert L.lcsa_compress_entries(*args(61, 0, 64)) == 0              # nothing to do
+    if not torch.cuda.is_available():
+        assert L.lcsa_compress_entries(*args(61, 1, 64)) == 4          # valid, but no device: no CPU path
+        assert L.lcsa_compress_entries(*args(31, 30, 64)) == 4         # entries 31..60 pool [120, 244)
+
+
 def test_empty_problems_are_noops(lcsa):
     L = lcsa.lib
     # T < m: no entries, nothing to do, no device needed

@@ -64,6 +64,49 @@ def test_compress_short_sequence(lcsa):
     assert lcsa.csa_compress(x["kv"], x["gate"], 4).shape == (1, 0, 512)
 
 
+@pytest.mark.parametrize("dtype,per_channel,rms", [("bf16", True, False), ("fp32", False, True), ("bf16", False, True)])
+def test_compress_entries_from_a_buffer(lcsa, dtype, per_channel, rms):
+    """Incremental compression from a buffer of raw rows equals the entries of
+    the whole-sequence compression (CSA and HCA windows)."""
+    B, T, D = 2, 1000, 512
+    x = gen.make_compress_inputs(B, T, D, dtype, seed=27, device=DEV, gate_per_channel=per_channel)
+    w = torch.randn(D, device=DEV, generator=torch.Generator(device=DEV).manual_seed(9)) if rms else None
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    for m, window in ((4, 8), (128, 128), (16, 16)):
+        ref = np.stack([O.compress(np64(x["kv"][b]), np64(x["gate"][b]), m, window,
+                                   None if w is None else np64(w)) for b in range(B)])
+        Nc = T // m
+        j0, n = Nc // 3, Nc - Nc // 3 - 1                   # a middle range of entries
+        pos0 = max(0, (j0 + 1) * m - window)
+        hi = (j0 + n) * m
+        cache = torch.zeros((B, Nc, D), dtype=tdt, device=DEV)
+        lcsa.compress_entries(x["kv"][:, pos0:hi].contiguous(), x["gate"][:, pos0:hi].contiguous(), pos0, m, window,
+                              j0, n, cache, rms_weight=w)
+        tol = dict(rtol=8e-3, atol=2e-4) if dtype == "bf16" else dict(rtol=1e-5, atol=2e-6)
+        np.testing.assert_allclose(np64(cache[:, j0:j0 + n]), ref[:, j0:j0 + n], **tol)
+        assert not cache[:, :j0].any() and not cache[:, j0 + n:].any()   # nothing else touched
+
+
+def test_compress_entries_decode_append(lcsa):
+    """Decode: after every arriving token, the entry that just completed is
+    appended from the 128-row window ring (CSA m=4 window 8, HCA m'=128)."""
+    B, T, D, W = 3, 1024, 512, 128
+    x = gen.make_compress_inputs(B, T, D, "bf16", seed=28, device=DEV)
+    caches = {(4, 8): torch.zeros((B, T // 4, D), dtype=torch.bfloat16, device=DEV),
+              (128, 128): torch.zeros((B, T // 128, D), dtype=torch.bfloat16, device=DEV)}
+    for t in range(W, T + 1):                               # t tokens have arrived
+        ring_kv = x["kv"][:, t - W:t].contiguous()
+        ring_g = x["gate"][:, t - W:t].contiguous()
+        for (m, window), cache in caches.items():
+            if t % m == 0:
+                lcsa.compress_entries(ring_kv, ring_g, t - W, m, window, t // m - 1, 1, cache)
+    for (m, window), cache in caches.items():
+        first = (W + m - 1) // m - 1 if W % m else W // m - 1     # first entry appended from the ring
+        ref = np.stack([O.compress(np64(x["kv"][b]), np64(x["gate"][b]), m, window) for b in range(B)])
+        np.testing.assert_allclose(np64(cache[:, first:]), ref[:, first:], rtol=8e-3, atol=2e-4)
+    assert lcsa.get_device_status() == 0
+
+
 # ------------------------------------------------------------------ top-k
 @pytest.mark.parametrize("n_cols,k,ties", [(64, 8, 0), (1000, 64, 4), (8191, 2048, 0), (8191, 2048, 16),
                                           (40000, 2048, 0), (5000, 1, 3), (300, 2048, 0),
@@ -247,6 +290,20 @@ def test_hca_dense_attn_parity(lcsa, dtype, H, D, R, m, W, Tq, Nc, q_pos0, unit,
     ref, ref_lse = O.hca_dense_attn(np64(x["q"]), np64(x["ckv"]), np64(x["kv"]), q_pos0, 0, m, W, _sink(x), R)
     assert_attn_close(np64(out).reshape(ref.shape), ref)
     np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
+
+
+def test_hca_key_range_splits_with_empty_items(lcsa):
+    """290 query rows (< 2 x 148: key ranges split in two) at positions 0..289
+    with m = 1: the first rows have a single key tile, so their second split
+    has no keys and the persistent kernel's empty-item path writes them (zero
+    partial output, -inf partial max) before the combine."""
+    B, H, D, R, m, W, Tq, Nc, q0 = 1, 64, 512, 64, 1, 128, 290, 290, 0
+    x = _attn_case(B, Tq, H, D, Nc, q0 + Tq, "bf16", seed=63)
+    out, lse = lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q0, 0, m, W, R, return_lse=True)
+    ref, ref_lse = O.hca_dense_attn(np64(x["q"]), np64(x["ckv"]), np64(x["kv"]), q0, 0, m, W, _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+    np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
+    assert lcsa.get_device_status() == 0
 
 
 def test_decode_window_ring(lcsa):
