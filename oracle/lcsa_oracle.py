@@ -33,11 +33,17 @@ Readings of points the pages leave open:
     rotary slice is rotated back by -t;
   * logits scale 1/sqrt(D); window = raw tokens s with t-W < s <= t;
     sink = one logit per head added as exp(sigma_h) to the denominator.
+  * FP4 indexer path: MXFP4 blocks (32 values, one power-of-two scale with
+    exponent floor(log2 amax) - 2, E2M1 codes rounded to nearest even and
+    saturated); the query is quantised per (row, head) and the scores use
+    the exact dequantised values.
 
 Parity pins: every function here is checked in tests/test_oracle_pins.py
 against closed forms, a library attention routine, brute force and values the
 pages print.
 """
+import math
+
 import numpy as np
 
 __all__ = [
@@ -158,6 +164,102 @@ def indexer_topk(q_idx, w, k_idx, q_pos0, m, k, score_dtype=np.float32):
     nv = [n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
     s_sel = s.astype(score_dtype).astype(np.float64)
     return topk_from_scores(s_sel, nv, k), s
+
+
+# ----------------------------------------------------------------------------
+# FP4 indexer QK path  ([p2] "FP4 Quantization-Aware Training": the indexer
+# computes its query-key scores in FP4 (E2M1) with block scale factors that a
+# wider format absorbs on dequantisation; [p4] "三、FP4量化": the table row that
+# takes the CSA indexer QK path from FP32 to FP4; CSA Step 2 "Select": the
+# Lightning Indexer runs in FP4 precision)
+#
+# Block format (the pages name E2M1 with block scales but no block size or
+# scale encoding; the plainest reading is the OCP Microscaling MXFP4 format):
+# 32 consecutive values share one power-of-two scale 2^X stored as a UE8M0
+# byte X + 127; each value is the E2M1 number nearest to x / 2^X.
+# ----------------------------------------------------------------------------
+MX_BLOCK = 32
+# E2M1 magnitudes by 3-bit code (exponent bits e1 e0, mantissa bit m):
+# e = 0: m * 0.5 (subnormal); e > 0: (1 + m/2) * 2^(e-1)
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def mx_scale_exponent(amax):
+    """Shared exponent of one block: X = floor(log2(amax)) - 2 (2 = the largest
+    E2M1 exponent, so amax / 2^X lies in [4, 8)), clamped to the UE8M0 range
+    [-127, 127]; an all-zero block takes X = -127."""
+    if amax == 0.0:
+        return -127
+    _, e = math.frexp(amax)          # amax = f * 2^e, f in [0.5, 1)
+    return max(-127, min(127, (e - 1) - 2))
+
+
+def e2m1_code(y):
+    """4-bit E2M1 code of the value nearest to y (round to nearest, ties to the
+    code with an even mantissa bit, magnitudes above 6 saturate to 6); bit 3 is
+    the sign of y."""
+    a = abs(y)
+    d = np.abs(E2M1_VALUES - a)
+    best = np.flatnonzero(d == d.min())
+    c = int(best[0]) if len(best) == 1 else int(best[best % 2 == 0][0])
+    return c | (8 if y < 0 else 0)
+
+
+def quantize_mxfp4(x):
+    """MXFP4 of x[..., C] (C a multiple of 32) along the last axis.
+
+    Returns (codes uint8 [..., C/2], scales uint8 [..., C/32]): byte i of a
+    row's codes holds element 2i in its low nibble and 2i+1 in its high
+    nibble; a block holding a non-finite value gets scale byte 255 and zero
+    codes.  Written for clarity, not speed: loops over blocks."""
+    x = np.asarray(x, dtype=np.float64)
+    C = x.shape[-1]
+    assert C % MX_BLOCK == 0
+    flat = x.reshape(-1, C)
+    codes = np.zeros((flat.shape[0], C // 2), dtype=np.uint8)
+    scales = np.zeros((flat.shape[0], C // MX_BLOCK), dtype=np.uint8)
+    for r in range(flat.shape[0]):
+        for b in range(C // MX_BLOCK):
+            blk = flat[r, b * MX_BLOCK:(b + 1) * MX_BLOCK]
+            if not np.isfinite(blk).all():
+                scales[r, b] = 255
+                continue
+            X = mx_scale_exponent(float(np.abs(blk).max()))
+            scales[r, b] = X + 127
+            for i in range(MX_BLOCK):
+                c = e2m1_code(math.ldexp(float(blk[i]), -X))
+                col = b * MX_BLOCK + i
+                codes[r, col // 2] |= np.uint8(c << (4 * (col % 2)))
+    return codes.reshape(x.shape[:-1] + (C // 2,)), scales.reshape(x.shape[:-1] + (C // MX_BLOCK,))
+
+
+def dequantize_mxfp4(codes, scales):
+    """Exact values (FP64) of MXFP4 codes and scales: E2M1 value times 2^X."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scales = np.asarray(scales, dtype=np.uint8)
+    lo = codes & 0xF
+    hi = codes >> 4
+    nib = np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (codes.shape[-1] * 2,))
+    val = E2M1_VALUES[nib & 7] * np.where(nib & 8, -1.0, 1.0)
+    X = scales.astype(np.float64) - 127.0
+    X = np.where(scales == 255, np.nan, X)
+    return val * np.exp2(np.repeat(X, MX_BLOCK, axis=-1))
+
+
+def indexer_scores_mxfp4(q_idx, w, k_codes, k_scales, q_pos0, m):
+    """Indexer scores of the FP4 QK path: the query is quantised to MXFP4 per
+    (row, head) and both sides are taken at their exact dequantised values;
+    the score formula is the one of indexer_scores."""
+    qc, qs = quantize_mxfp4(q_idx)
+    return indexer_scores(dequantize_mxfp4(qc, qs), w, dequantize_mxfp4(k_codes, k_scales), q_pos0, m)
+
+
+def indexer_topk_mxfp4(q_idx, w, k_codes, k_scales, q_pos0, m, k, score_dtype=np.float32):
+    """Top-k of the FP4-path scores, rounded to the selection precision."""
+    s = indexer_scores_mxfp4(q_idx, w, k_codes, k_scales, q_pos0, m)
+    Tq, Nc = s.shape
+    nv = [n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+    return topk_from_scores(s.astype(score_dtype).astype(np.float64), nv, k), s
 
 
 # ----------------------------------------------------------------------------

@@ -132,6 +132,119 @@ def test_indexer_relu_per_head_then_weighted_sum():
     np.testing.assert_allclose(O.indexer_scores(q[:, p], w1[:, p], k, 100, 4), s1, atol=1e-12)
 
 
+# ---------------------------------------------------------------- FP4 (MXFP4) indexer path
+def _e2m1_from_bits(c):
+    """Value of a 4-bit E2M1 code decoded from its fields: sign bit 3,
+    exponent bits 2-1 (bias 1), mantissa bit 0; exponent 0 is subnormal."""
+    s, e, m = (c >> 3) & 1, (c >> 1) & 3, c & 1
+    mag = m * 0.5 if e == 0 else (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+    return -mag if s else mag
+
+
+def test_e2m1_codes_bruteforce_from_bit_fields():
+    # every multiple of 1/32 in [-8, 8]: nearest code of the same sign, ties to
+    # an even mantissa bit (round to nearest even), large magnitudes saturate
+    for n in range(-256, 257):
+        y = n / 32.0
+        cands = [c for c in range(16) if ((c >> 3) & 1) == (1 if y < 0 else 0)]
+        best = min(abs(y - _e2m1_from_bits(c)) for c in cands)
+        near = [c for c in cands if abs(y - _e2m1_from_bits(c)) == best]
+        want = near[0] if len(near) == 1 else [c for c in near if c % 2 == 0][0]
+        assert O.e2m1_code(y) == want, y
+
+
+def test_mx_round_to_nearest_even_midpoints():
+    # midpoints of the E2M1 grid go to the neighbour with the even mantissa
+    # bit; 7 saturates to 6 (the block's amax 7 fixes X = 0)
+    y = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -0.75, -5.0]
+    want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, -1.0, -4.0]
+    x = np.zeros((1, 32))
+    x[0, :len(y)] = y
+    c, sc = O.quantize_mxfp4(x)
+    assert sc[0, 0] == 127
+    np.testing.assert_array_equal(O.dequantize_mxfp4(c, sc)[0, :len(y)], want)
+
+
+def test_mx_scale_rule():
+    # X = floor(log2(amax)) - 2, clamped to [-127, 127]; UE8M0 byte = X + 127
+    for amax, byte in [(1.0, 125), (6.0, 127), (7.999, 127), (8.0, 128), (0.75, 124),
+                       (2.0 ** -130, 0), (0.0, 0), (2.0 ** 126, 251)]:
+        x = np.zeros((1, 32))
+        x[0, 5] = amax
+        assert O.quantize_mxfp4(x)[1][0, 0] == byte, amax
+    x = np.zeros((1, 64))
+    x[0, 40] = np.inf
+    c, sc = O.quantize_mxfp4(x)
+    assert sc[0, 1] == 255 and not c[0, 16:].any() and sc[0, 0] == 0
+
+
+def test_mx_roundtrip_of_representable_blocks():
+    r = _rng(21)
+    codes = r.integers(0, 256, (6, 64), dtype=np.uint8)
+    codes[:, ::16] = (codes[:, ::16] & 0xF0) | 0x7        # element 0 of every block = +6: X recovers
+    scales = r.integers(100, 140, (6, 4), dtype=np.uint8)
+    v = O.dequantize_mxfp4(codes, scales)
+    c2, s2 = O.quantize_mxfp4(v)
+    np.testing.assert_array_equal(s2, scales)
+    # codes agree up to the sign of zero (a -0 input quantises to +0)
+    np.testing.assert_array_equal(O.dequantize_mxfp4(c2, s2), v)
+
+
+def test_mx_error_within_half_spacing():
+    r = _rng(22)
+    x = r.standard_normal((40, 128)) * np.exp2(r.integers(-20, 20, (40, 1)))
+    c, sc = O.quantize_mxfp4(x)
+    d = O.dequantize_mxfp4(c, sc)
+    X = np.repeat(sc.astype(np.float64) - 127, 32, axis=1)
+    y = np.abs(x) / np.exp2(X)
+    half = np.where(y < 2, 0.25, np.where(y < 4, 0.5, 1.0))
+    err = np.abs(x - d) / np.exp2(X)
+    inside = y <= 6
+    assert (err[inside] <= half[inside] + 1e-12).all()
+    # amax / 2^X lies in [4, 8): magnitudes above 6 saturate to 6
+    assert (y < 8).all() and (np.abs(d[~inside]) / np.exp2(X[~inside]) == 6.0).all()
+    assert (np.sign(d) * np.sign(x) >= 0).all()
+
+
+def test_indexer_mxfp4_exact_on_representable_inputs():
+    # quantisation is the identity on values already on the MXFP4 grid with a
+    # full-range element per block, so the FP4 path reduces to the exact indexer
+    r = _rng(23)
+    Tq, H, Nc, D_I, m, q_pos0 = 3, 4, 40, 64, 4, 150
+
+    def grid(shape):
+        c = r.integers(0, 256, shape[:-1] + (shape[-1] // 2,), dtype=np.uint8)
+        c[..., ::16] = (c[..., ::16] & 0xF0) | 0x6         # a +4 in every block
+        sc = r.integers(118, 128, shape[:-1] + (shape[-1] // 32,), dtype=np.uint8)
+        return c, sc
+
+    qc, qs = grid((Tq, H, D_I))
+    kc, ks = grid((Nc, D_I))
+    q = O.dequantize_mxfp4(qc, qs)
+    k = O.dequantize_mxfp4(kc, ks)
+    w = r.standard_normal((Tq, H))
+    s_fp4 = O.indexer_scores_mxfp4(q, w, kc, ks, q_pos0, m)
+    s_ref = O.indexer_scores(q, w, k, q_pos0, m)
+    np.testing.assert_array_equal(s_fp4, s_ref)
+    idx, _ = O.indexer_topk_mxfp4(q, w, kc, ks, q_pos0, m, 8)
+    idx_ref, _ = O.indexer_topk(q, w, k, q_pos0, m, 8)
+    np.testing.assert_array_equal(idx, idx_ref)
+
+
+def test_indexer_mxfp4_quantises_the_query():
+    # a query off the grid scores as its rounded copy does
+    r = _rng(24)
+    q = r.standard_normal((2, 3, 32))
+    k_raw = r.standard_normal((10, 32))
+    kc, ks = O.quantize_mxfp4(k_raw)
+    w = r.standard_normal((2, 3))
+    qc, qs = O.quantize_mxfp4(q)
+    a = O.indexer_scores_mxfp4(q, w, kc, ks, 44, 4)
+    b = O.indexer_scores(O.dequantize_mxfp4(qc, qs), w, O.dequantize_mxfp4(kc, ks), 44, 4)
+    np.testing.assert_array_equal(a, b)
+    assert not np.array_equal(a, O.indexer_scores(q, w, O.dequantize_mxfp4(kc, ks), 44, 4))
+
+
 def test_visibility_boundary():
     # j visible iff j < floor(t/m): m=4 -> t=0..3 see 0, t=4..7 see 1, t=8 sees 2
     assert [O.n_visible(t, 4, 100) for t in range(10)] == [0, 0, 0, 0, 1, 1, 1, 1, 2, 2]
