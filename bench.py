@@ -223,7 +223,7 @@ def _barrier():
         torch.distributed.barrier()
 
 
-def timed(fn, steps, warmup, bus_id, sample_clocks=True):
+def timed(fn, steps, warmup, bus_id, sample_clocks=True, on_start=None):
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -235,6 +235,8 @@ def timed(fn, steps, warmup, bus_id, sample_clocks=True):
         time.sleep(0.4)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
+    if on_start:
+        on_start()
     for _ in range(steps):
         fn()
     b.record()
@@ -442,19 +444,40 @@ def run_e2e(args, cfg, runner, layers, units, world):
     h2d = sum(t.numel() * t.element_size() for L in layers for t in hosts[L.kind].values())
     d2h = out_host.numel() * out_host.element_size()
 
+    # Host-to-device copies run on their own stream, one event per layer in
+    # each direction: layer li's inputs are refilled as soon as layer li of
+    # the previous step has consumed them, so the copies of later layers (and
+    # of the next step) proceed under the kernels of earlier ones, and the
+    # output readback (compute stream) overlaps the next step's input copies
+    # on the other PCIe direction.  Every step still moves all of its inputs
+    # in and its output out inside the timed region.
+    main = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in layers]
+    free = [torch.cuda.Event() for _ in layers]
+    for ev in free:
+        ev.record(main)
+
     def step():
         for li, L in enumerate(layers):
-            for n, t in hosts[L.kind].items():
-                getattr(L, n).copy_(t, non_blocking=True)
+            copy.wait_event(free[li])
+            with torch.cuda.stream(copy):
+                for n, t in hosts[L.kind].items():
+                    getattr(L, n).copy_(t, non_blocking=True)
+            ready[li].record(copy)
+        for li in range(len(layers)):
+            main.wait_event(ready[li])
             runner.layer(li)
+            free[li].record(main)
         out_host.copy_(runner.out, non_blocking=True)
 
-    steps = max(1, min(args.steps, 2))
-    ms, _ = timed(step, steps, 1, None, sample_clocks=False)
+    steps = max(1, min(args.steps, 3))
+    ms, _ = timed(step, steps, 1, None, sample_clocks=False, on_start=lambda: copy.wait_stream(main))
     ms = max_over_ranks(ms)
     del hosts, out_host
     return {"value": weak_scaling_throughput(units, ms / 1e3, world), "unit": "tokens/s", "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "input copies on a second stream, per-layer events"}
 
 
 def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
@@ -513,7 +536,47 @@ def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
                         "note": "whole decode step (indexer keys + gathered rows + window + q/out)"},
            "gpu_launches": int(launches), "clocks": clocks,
            "compress_append_us": append_cost(lcsa, cfg, B, ckv, t, g, dev)}
-    del ix, ckv, q, kvw, idx, out, ws_ix, ws_at
+
+    # The FP4 QK path: the indexer-key cache held as MXFP4 (quantised once,
+    # as a cache is written), the queries quantised inside the call.
+    kc, ks = lcsa.quantize_mxfp4(ix["k_idx"])
+    idx4 = torch.empty_like(idx)
+    ws_ix4 = torch.empty(lcsa.indexer_mxfp4_workspace_bytes(ix["q_idx"], kc, cfg.k), dtype=torch.uint8, device=dev)
+    ev4 = []
+
+    def step4(record=False):
+        a = torch.cuda.Event(enable_timing=True) if record else None
+        if a:
+            a.record()
+        lcsa.indexer_topk_mxfp4(ix["q_idx"], ix["w"], kc, ks, t, cfg.m, cfg.k, workspace=ws_ix4, idx_out=idx4)
+        b = torch.cuda.Event(enable_timing=True) if record else None
+        if b:
+            b.record()
+        lcsa.csa_sparse_attn(q, ckv, idx4, kvw, sink, t, t - cfg.W + 1, cfg.m, cfg.W, cfg.R, out=out,
+                             workspace=ws_at)
+        if record:
+            c = torch.cuda.Event(enable_timing=True)
+            c.record()
+            ev4.append((a, b, c))
+
+    ms4, clocks4 = timed(lambda: step4(True), args.steps * 4, args.warmup, bus_id)
+    ms4 = max_over_ranks(ms4)
+    sel16, sel4 = idx[:, 0].cpu().numpy(), idx4[:, 0].cpu().numpy()
+    recall = float(np.mean([len(set(sel16[b].tolist()) & set(sel4[b].tolist())) / cfg.k for b in range(B)]))
+    byts4 = byts - B * Nc * cfg.D_I * 2 + B * Nc * (cfg.D_I // 2 + cfg.D_I // 32)
+    gbs4 = byts4 / (ms4 / 1e3) / 1e9
+    res["fp4_indexer"] = {
+        "value": weak_scaling_throughput(B, ms4 / 1e3, world), "unit": "queries/s", "ms_per_step": ms4,
+        "indexer_topk_ms": statistics.mean(a.elapsed_time(b) for a, b, _ in ev4),
+        "csa_sparse_attn_ms": statistics.mean(b.elapsed_time(c) for _, b, c in ev4),
+        "recall_vs_bf16_keys": round(recall, 4),
+        "roofline": {"bound": "hbm", "achieved": round(gbs4, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs4 / peaks["hbm_gbs"], 4), "bytes_per_step": byts4,
+                     "peak_source": f"hbm_gbs of {peaks['source']}"},
+        "clocks": clocks4,
+        "note": "indexer keys as MXFP4 (64 code bytes + 4 scale bytes per entry), queries quantised per head; "
+                "recall = share of the BF16-key selection kept"}
+    del ix, ckv, q, kvw, idx, out, ws_ix, ws_at, kc, ks, idx4, ws_ix4
     torch.cuda.empty_cache()
     return res
 

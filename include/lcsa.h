@@ -187,6 +187,68 @@ lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace,
 int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a);
 
 /* ------------------------------------------------------------------------
+ * MXFP4 quantisation for the FP4 indexer QK path ([p2] "FP4
+ * Quantization-Aware Training": the indexer's query-key scores are computed
+ * in FP4 E2M1 with block scale factors; [p4] "三、FP4量化": E2M1 = 2 exponent
+ * bits + 1 mantissa bit, and the CSA indexer QK path goes from FP32 to FP4).
+ * The pages give no block size or scale encoding; this is the OCP
+ * Microscaling MXFP4 format:
+ *   - 32 consecutive values of a row form a block with scale 2^X,
+ *     X = floor(log2(max |x|)) - 2 clamped to [-127, 127] (-127 for an
+ *     all-zero block), stored as the byte X + 127;
+ *   - each value is the E2M1 number nearest to x / 2^X (ties to an even
+ *     mantissa bit, magnitudes above 6 saturate), sign bit = (x < 0);
+ *   - a block holding Inf or NaN gets scale byte 255 and zero codes.
+ *
+ *   x      [rows, cols] dtype (cols a multiple of 32), device, aligned to its
+ *          element size
+ *   codes  [rows, cols/2] uint8, device: element 2i in the low nibble of byte i
+ *   scales [rows, cols/32] uint8, device
+ * Codes and scales are a pure function of x (bit-exact with any other exact
+ * implementation of the definition above).
+ * ------------------------------------------------------------------------ */
+lcsa_status lcsa_quantize_mxfp4(const void* x, int64_t rows, int cols, lcsa_dtype dtype, uint8_t* codes,
+                                uint8_t* scales, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Indexer + top-k on the FP4 QK path.  Same scores and selection as
+ * lcsa_indexer_topk, with both sides of every dot product taken at their
+ * MXFP4 values: the keys come quantised (the indexer-key cache in MXFP4,
+ * e.g. written by lcsa_quantize_mxfp4 with cols = D_I), the BF16 queries are
+ * quantised per (row, head) inside the call.  The products of the
+ * dequantised values are exact and accumulate in FP32 (the kernel stages
+ * each key entry and query head as FP8 E4M3 relative to its largest block
+ * scale, exact while the entry's block scales lie within 2^13 of it; a block
+ * further below rounds to the E4M3 grid).
+ *
+ *   q_idx     [B,Tq,64,128] BF16, 16-byte aligned; finite values
+ *   w         [B,Tq,64] FP32
+ *   k_codes   [B,Nc,64] uint8 (MXFP4 codes of the 128-dim keys), 16-byte aligned
+ *   k_scales  [B,Nc,4] uint8, 4-byte aligned
+ *   idx_out, scores_out, q_pos0, m, k: as lcsa_indexer_args
+ * Only H_I = 64 and D_I = 128 (LCSA_ERR_UNSUPPORTED otherwise).  The
+ * workspace (size from lcsa_indexer_topk_mxfp4_workspace) holds the score
+ * chunk, the top-k scratch and the prepared queries of a chunk; a smaller
+ * one processes fewer rows at a time (LCSA_ERR_WORKSPACE below one row).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* q_idx;
+  const float* w;
+  const uint8_t* k_codes;
+  const uint8_t* k_scales;
+  int B, Tq, Nc, H_I, D_I;
+  int64_t q_pos0;
+  int m;
+  int k;
+  int32_t* idx_out;
+  float* scores_out;
+} lcsa_indexer_mxfp4_args;
+
+size_t lcsa_indexer_topk_mxfp4_workspace(const lcsa_indexer_mxfp4_args* a);
+lcsa_status lcsa_indexer_topk_mxfp4(const lcsa_indexer_mxfp4_args* a, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * Indexer + top-k without a caller workspace.  The pages have no counterpart
  * to this call: it exists for callers that cannot allocate device memory when
  * they call the library (an allocator or arena they do not own, a runtime

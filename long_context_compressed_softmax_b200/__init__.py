@@ -31,6 +31,7 @@ EXPORTED = [
     "lcsa_topk_workspace", "lcsa_topk_from_scores",
     "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
     "lcsa_indexer_topk_noalloc",
+    "lcsa_quantize_mxfp4", "lcsa_indexer_topk_mxfp4_workspace", "lcsa_indexer_topk_mxfp4",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
 ]
 
@@ -47,6 +48,16 @@ class IndexerArgs(ctypes.Structure):
         ("B", ctypes.c_int), ("Tq", ctypes.c_int), ("Nc", ctypes.c_int), ("H_I", ctypes.c_int),
         ("D_I", ctypes.c_int), ("dtype", ctypes.c_int), ("q_pos0", ctypes.c_int64), ("m", ctypes.c_int),
         ("k", ctypes.c_int), ("idx_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
+    ]
+
+
+class IndexerMxfp4Args(ctypes.Structure):
+    _fields_ = [
+        ("q_idx", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k_codes", ctypes.c_void_p),
+        ("k_scales", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Tq", ctypes.c_int), ("Nc", ctypes.c_int), ("H_I", ctypes.c_int),
+        ("D_I", ctypes.c_int), ("q_pos0", ctypes.c_int64), ("m", ctypes.c_int), ("k", ctypes.c_int),
+        ("idx_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
     ]
 
 
@@ -78,6 +89,9 @@ _sig = {
     "lcsa_indexer_topk": (_i, [ctypes.POINTER(IndexerArgs), _vp, _sz, _vp]),
     "lcsa_indexer_uses_tensor_cores": (_i, [ctypes.POINTER(IndexerArgs)]),
     "lcsa_indexer_topk_noalloc": (_i, [ctypes.POINTER(IndexerArgs), _vp]),
+    "lcsa_quantize_mxfp4": (_i, [_vp, _i64, _i, _i, _vp, _vp, _vp]),
+    "lcsa_indexer_topk_mxfp4_workspace": (_sz, [ctypes.POINTER(IndexerMxfp4Args)]),
+    "lcsa_indexer_topk_mxfp4": (_i, [ctypes.POINTER(IndexerMxfp4Args), _vp, _sz, _vp]),
     "lcsa_attn_workspace": (_sz, [ctypes.POINTER(AttnArgs), _i]),
     "lcsa_csa_sparse_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
@@ -240,6 +254,55 @@ def indexer_topk(q_idx, w, k_idx, q_pos0, m, k, return_scores=False, workspace=N
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     st = _lib.lcsa_indexer_topk(ctypes.byref(a), _p(workspace), workspace.numel(), _stream(dev))
     _check(st, "indexer_topk")
+    return (idx_out, scores) if return_scores else idx_out
+
+
+# ----------------------------------------------------------------- FP4 indexer path
+def quantize_mxfp4(x, codes=None, scales=None):
+    """MXFP4 of x [..., C] (BF16 or FP32, C a multiple of 32) along the last
+    axis -> (codes uint8 [..., C/2], scales uint8 [..., C/32])."""
+    _need_contig(x)
+    C = x.shape[-1]
+    rows = x.numel() // C if C else 0
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (C // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (C // 32,), dtype=torch.uint8, device=x.device)
+    st = _lib.lcsa_quantize_mxfp4(_p(x), rows, C, _dt(x), _p(codes), _p(scales), _stream(x.device))
+    _check(st, "quantize_mxfp4")
+    return codes, scales
+
+
+def _indexer_mxfp4_args(q_idx, w, k_codes, k_scales, q_pos0, m, k, idx_out, scores_out):
+    B, Tq, H_I, D_I = q_idx.shape
+    return IndexerMxfp4Args(_p(q_idx), _p(w), _p(k_codes), _p(k_scales), B, Tq, k_codes.shape[1], H_I, D_I,
+                            int(q_pos0), m, k, _p(idx_out), _p(scores_out))
+
+
+def indexer_mxfp4_workspace_bytes(q_idx, k_codes, k):
+    B, Tq, H_I, D_I = q_idx.shape
+    a = IndexerMxfp4Args(None, None, None, None, B, Tq, k_codes.shape[1], H_I, D_I, 0, 1, k, None, None)
+    return int(_lib.lcsa_indexer_topk_mxfp4_workspace(ctypes.byref(a)))
+
+
+def indexer_topk_mxfp4(q_idx, w, k_codes, k_scales, q_pos0, m, k, return_scores=False, workspace=None,
+                       idx_out=None):
+    """FP4 QK path: q_idx [B,Tq,64,128] BF16, w [B,Tq,64] fp32, MXFP4 keys
+    k_codes [B,Nc,64] / k_scales [B,Nc,4] uint8 -> idx [B,Tq,k] int32 (and
+    scores [B,Tq,Nc] fp32 when return_scores)."""
+    _need_contig(q_idx, w, k_codes, k_scales)
+    B, Tq = q_idx.shape[:2]
+    Nc = k_codes.shape[1]
+    dev = q_idx.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Tq, k), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, Tq, Nc), dtype=torch.float32, device=dev) if return_scores else None
+    a = _indexer_mxfp4_args(q_idx, w, k_codes, k_scales, q_pos0, m, k, idx_out, scores)
+    if workspace is None:       # a smaller caller workspace processes fewer rows at a time
+        need = int(_lib.lcsa_indexer_topk_mxfp4_workspace(ctypes.byref(a)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = _lib.lcsa_indexer_topk_mxfp4(ctypes.byref(a), _p(workspace), workspace.numel(), _stream(dev))
+    _check(st, "indexer_topk_mxfp4")
     return (idx_out, scores) if return_scores else idx_out
 
 

@@ -1,0 +1,350 @@
+// Lightning-Indexer scores on the FP4 QK path (DeepSeek-V4 "FP4
+// Quantization-Aware Training": the indexer computes its query-key scores in
+// FP4; CSA Step 2 "Select": the Lightning Indexer runs in FP4 precision).
+// H_I = 64, D_I = 128.
+//
+// The indexer keys live in HBM as MXFP4 (64 bytes of E2M1 codes + 4 scale
+// bytes per entry, a quarter of BF16), which is what bounds long-context
+// decode: every decode step streams all of them.  Per 128-entry tile:
+//   TMA        packed codes -> shared memory (8-deep ring)
+//   dequant    8 warps, two per tile (4 tiles in flight), write E4M3 in the
+//              128B-swizzled K-major layout, each entry relative to its
+//              largest block exponent (exact for blocks within 2^13 of it,
+//              see mxfp4.cuh)
+//   MMA        tcgen05 kind::f8f6f4, M = 128 entries, N = 64 heads x up to 4
+//              query rows (E4M3 queries prepared by indexer_q8_kernel), K = 128
+//   epilogue   8 warps: ReLU, head weights (with the query factors folded
+//              in) and the entry factor 2^(Xref - 6), one score per lane;
+//              with 3-4 query rows each warp scores 2 rows of every tile,
+//              with 1-2 rows the two warps of a lane quarter take alternate
+//              tiles (one accumulator each).
+// Warp roles (576 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
+// 2-9 epilogue, 10-17 dequantisers.  Every wait is bounded (tc::mbar_wait);
+// on expiry the CTA stops, records LCSA_DEV_TIMEOUT, drains its in-flight
+// copies and frees TMEM.
+#pragma once
+#include "tc_ptx.cuh"
+#include "mxfp4.cuh"
+#include "indexer_tc.cuh"
+
+namespace lcsa {
+
+constexpr int kI4CStages = 8;                  // packed-code ring
+constexpr int kI4DqWarp0 = 10;
+constexpr int kI4DqWarps = 8;                  // warps 2t, 2t+1 of the group expand tiles t, t+4, t+8, ...
+constexpr int kI4AStages = kI4DqWarps / 2;     // E4M3 key tiles in flight: one per dequantiser pair
+constexpr int kI4Threads = (kI4DqWarp0 + kI4DqWarps) * 32;   // 576
+constexpr uint32_t kI4QBytes = 256 * 128;      // 4 query rows x 64 heads x 128 E4M3
+constexpr uint32_t kI4ABytes = kIxTileE * 128; // 128 entries x 128 E4M3
+constexpr uint32_t kI4CBytes = kIxTileE * 64;  // 128 entries x 64 code bytes
+constexpr size_t kI4Smem = 1024 + kI4QBytes + kI4AStages * kI4ABytes + kI4CStages * kI4CBytes + kIxRows * 64 * 4 +
+                           256;
+// Piece order of the dequantisers: the lane of row r handles code block
+// p = kI4Perm[(r >> 1) & 3] ^ i at step i, so that both the 64-byte-strided
+// code reads and the swizzled 16-byte writes of 8 consecutive rows hit 8
+// different bank groups (p -> kI4Perm[p] is multiplication by a primitive
+// element of GF(4), so kI4Perm[k] and kI4Perm[k] ^ k are both permutations).
+__device__ __constant__ int kI4Perm[4] = {0, 2, 3, 1};
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A/B (format 0) and FP32 D.
+__host__ __device__ __forceinline__ uint32_t idesc_e4m3(int M, int N) {
+  uint32_t d = 0;
+  d |= 1u << 4;
+  d |= (uint32_t)((N >> 3) & 0x3F) << 17;
+  d |= (uint32_t)((M >> 4) & 0x1F) << 24;
+  return d;
+}
+__device__ __forceinline__ void mma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ int max_scale_byte(uint32_t sw) {
+  const uint32_t a = max(sw & 0xFFu, (sw >> 8) & 0xFFu), b = max((sw >> 16) & 0xFFu, sw >> 24);
+  return (int)max(a, b);
+}
+
+__global__ void __launch_bounds__(kI4Threads, 1)
+indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap c_map,
+                   const uint32_t* __restrict__ k_scales, const float* __restrict__ w8,
+                   float* __restrict__ scores, IxGeom g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_q = smem;
+  uint8_t* s_a = s_q + kI4QBytes;
+  uint8_t* s_c = s_a + kI4AStages * kI4ABytes;
+  float* s_w = reinterpret_cast<float*>(s_c + kI4CStages * kI4CBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + kIxRows * 64);
+  uint64_t* q_full = bars;
+  uint64_t* c_full = bars + 1;
+  uint64_t* c_empty = c_full + kI4CStages;
+  uint64_t* a_full = c_empty + kI4CStages;
+  uint64_t* a_empty = a_full + kI4AStages;
+  uint64_t* acc_full = a_empty + kI4AStages;
+  uint64_t* acc_empty = acc_full + 2;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work unit (as indexer_tc_kernel: heaviest query groups first)
+  const int n_groups = g.nb * g.gps;
+  const int grp = n_groups - 1 - (int)blockIdx.x;
+  const int split = blockIdx.y;
+  const int bl = grp / g.gps;
+  const int b = g.b0 + bl;
+  const int gi = grp - bl * g.gps;
+  const int i_first = g.i0 + gi * kIxRows;
+  int rows = g.i0 + g.ni - i_first;
+  rows = rows < kIxRows ? rows : kIxRows;
+  long long nv = (g.q_pos0 + i_first + rows - 1) / g.m;
+  if (nv > g.Nc) nv = g.Nc;
+  const int tiles_all = (int)((nv + kIxTileE - 1) / kIxTileE);
+  const int per_split = (tiles_all + g.splits - 1) / g.splits;
+  const int t_begin = split * per_split;
+  int t_end = t_begin + per_split;
+  t_end = t_end < tiles_all ? t_end : tiles_all;
+  const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
+  if (n_tiles == 0) return;
+  const long long rect_row = (long long)bl * g.ni + (i_first - g.i0);   // first query row in the rectangle
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int s = 0; s < kI4CStages; ++s) { tc::mbar_init(c_full + s, 1); tc::mbar_init(c_empty + s, 2); }
+    for (int s = 0; s < kI4AStages; ++s) { tc::mbar_init(a_full + s, 2); tc::mbar_init(a_empty + s, 1); }
+    // rows > 2: all 8 epilogue warps read every accumulator; else 4 per accumulator
+    for (int a = 0; a < 2; ++a) { tc::mbar_init(acc_full + a, 1); tc::mbar_init(acc_empty + a, rows > 2 ? 8 : 4); }
+    tc::fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 1) { tc::tmem_alloc(&s_tmem, 512); tc::tmem_relinquish(); }
+  for (int e = threadIdx.x; e < kIxRows * 64; e += kI4Threads) {
+    const int q = e >> 6;
+    s_w[e] = q < rows ? w8[(rect_row + q) * 64 + (e & 63)] : 0.f;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+  const long long ent0 = (long long)b * g.Nc;          // first entry row of this sequence
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&q_map);
+      tc::prefetch_tmap(&c_map);
+      tc::mbar_arrive_expect_tx(q_full, kI4QBytes);
+      tc::tma_load_2d(s_q, &q_map, q_full, 0, (int)(rect_row * 64));
+      int issued = 0;
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % kI4CStages, r = n / kI4CStages;
+        if (r > 0 && !tc::mbar_wait(c_empty + s, (r - 1) & 1)) { *abort_flag = 1; break; }
+        if (*abort_flag) break;
+        tc::mbar_arrive_expect_tx(c_full + s, kI4CBytes);
+        tc::tma_load_2d(s_c + s * kI4CBytes, &c_map, c_full + s, 0,
+                        (int)(ent0 + (long long)(t_begin + n) * kIxTileE));
+        ++issued;
+      }
+      for (int n = issued - kI4CStages > 0 ? issued - kI4CStages : 0; n < issued; ++n)
+        tc::mbar_wait(c_full + n % kI4CStages, (n / kI4CStages) & 1);
+      tc::mbar_wait(q_full, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      const uint32_t idesc = idesc_e4m3(128, 64 * rows);
+      bool ok = tc::mbar_wait(q_full, 0);
+      const uint32_t b_base = tc::smem_u32(s_q);
+      for (int n = 0; ok && n < n_tiles; ++n) {
+        const int s = n % kI4AStages, r = n / kI4AStages;
+        const int a = n & 1, ra = n >> 1;
+        if (*abort_flag) break;
+        if (!tc::mbar_wait(a_full + s, r & 1)) { ok = false; break; }
+        if (ra > 0 && !tc::mbar_wait(acc_empty + a, (ra - 1) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t a_base = tc::smem_u32(s_a + s * kI4ABytes);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = tc::sdesc_sw128(a_base + ks * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(b_base + ks * 32, 16, 1024);
+          mma_e4m3_ss(tmem + a * 256, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(a_empty + s);
+        tc::mma_commit(acc_full + a);
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp < kI4DqWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;                 // 0..7
+    const int quarter = warp & 3;           // TMEM lanes [32*quarter, 32*quarter+32)
+    const int half = e >> 2;                // query rows {2*half, 2*half+1}
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    // rows > 2: rows {2 half, 2 half + 1} of every tile; rows <= 2: every row
+    // of the tiles n with n % 2 == half (accumulator `half`)
+    const bool by_tile = rows <= 2;                      // CTA-uniform
+    const int n_q = by_tile ? rows : min(2, max(0, rows - 2 * half));
+    const int q0 = by_tile ? 0 : 2 * half;
+    const int n_first = by_tile ? half : 0, n_step = by_tile ? 2 : 1;
+    auto scale_word = [&](int n) -> uint32_t {           // this lane's entry of tile n
+      const long long j = (long long)(t_begin + n) * kIxTileE + quarter * 32 + lane;
+      return n < n_tiles && j < g.Nc ? __ldg(k_scales + ent0 + j) : 0x7F7F7F7Fu;
+    };
+    // scale words of the next three tiles this warp scores
+    uint32_t sw1 = scale_word(n_first), sw2 = scale_word(n_first + n_step), sw3 = scale_word(n_first + 2 * n_step);
+    for (int n = n_first; n_q > 0 && n < n_tiles; n += n_step) {
+      const int a = n & 1, ra = n >> 1;
+      const long long j = (long long)(t_begin + n) * kIxTileE + quarter * 32 + lane;
+      const uint32_t sw = sw1;
+      sw1 = sw2; sw2 = sw3; sw3 = scale_word(n + 3 * n_step);
+      // waits end on the same decision in every lane (a split warp would stall at the warp syncs)
+      bool ok = !*abort_flag && tc::mbar_wait(acc_full + a, ra & 1);
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      tc::tc_fence_after();
+      float sc[2] = {0.f, 0.f};
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        if (qq < n_q) {
+          const uint32_t col = tmem + lane_addr + (uint32_t)(a * 256 + (q0 + qq) * 64);
+          const uint32_t wq = tc::smem_u32(s_w + (q0 + qq) * 64);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};     // four partial sums over heads h = 4i + c
+#pragma unroll
+          for (int hb = 0; hb < 64; hb += 32) {     // 32 heads at a time
+            uint32_t v[32];
+            tc::tmem_ld32(col + hb, v);
+            tc::tmem_wait_ld();
+            if (qq == n_q - 1 && hb == 32) {       // accumulator read out: hand it back to the MMA warp
+              tc::tc_fence_before();
+              __syncwarp();
+              if (lane == 0) tc::mbar_arrive(acc_empty + a);
+            }
+#pragma unroll
+            for (int h = 0; h < 32; h += 4) {
+              const float4 w4 = tc::lds128f(wq + (hb + h) * 4);
+              acc[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[h]), 0.f), acc[0]);
+              acc[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), acc[1]);
+              acc[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), acc[2]);
+              acc[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), acc[3]);
+            }
+          }
+          sc[qq] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+      }
+      const float f = pow2f(max_scale_byte(sw) - 127 - 6);
+      if (j < g.Nc) {
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq)
+          if (qq < n_q) scores[(rect_row + q0 + qq) * g.Nc + j] = sc[qq] * f;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dequantisers
+    // warps 2t and 2t+1 of the group expand tiles n = t, t + 4, ... into E4M3
+    // stage t; the lane of warp 2t + hh handles entry rows lane + 32 (2 hh + jr)
+    const int dq = (warp - kI4DqWarp0) >> 1, hh = (warp - kI4DqWarp0) & 1;
+    const int pb = kI4Perm[(lane >> 1) & 3];
+    const uint32_t sw_row = (uint32_t)(lane & 7);
+    auto scale_words = [&](int n, uint32_t* sw) {
+#pragma unroll
+      for (int jr = 0; jr < 2; ++jr) {
+        const long long j = (long long)(t_begin + n) * kIxTileE + lane + 32 * (2 * hh + jr);
+        sw[jr] = n < n_tiles && j < g.Nc ? __ldg(k_scales + ent0 + j) : 0x7F7F7F7Fu;
+      }
+    };
+    uint32_t cur[2], nxt[2];                    // this warp's next two tiles
+    scale_words(dq, cur);
+    scale_words(dq + kI4AStages, nxt);
+    for (int n = dq; n < n_tiles; n += kI4AStages) {
+      const int cs = n % kI4CStages, rc = n / kI4CStages;
+      const int ra = n / kI4AStages;
+      uint32_t sw[2];
+#pragma unroll
+      for (int jr = 0; jr < 2; ++jr) { sw[jr] = cur[jr]; cur[jr] = nxt[jr]; }
+      scale_words(n + 2 * kI4AStages, nxt);
+      bool ok = !*abort_flag && tc::mbar_wait(c_full + cs, rc & 1);
+      ok = ok && (ra == 0 || tc::mbar_wait(a_empty + dq, (ra - 1) & 1));
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+#pragma unroll
+      for (int jr = 0; jr < 2; ++jr) {
+        const int r = lane + 32 * (2 * hh + jr);
+        const uint32_t w = sw[jr];
+        const int xref = max_scale_byte(w);
+        const uint32_t src = tc::smem_u32(s_c) + cs * kI4CBytes + r * 64;
+        const uint32_t dst = tc::smem_u32(s_a) + dq * kI4ABytes + r * 128;
+        uint4 c[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = tc::lds128(src + (uint32_t)(pb ^ i) * 16);   // code block pb ^ i
+        // every block within 2^11 of the entry's largest: table by exponent-field arithmetic
+        const bool fast = ((w & 0xFFu) + 11 >= (uint32_t)xref) && (((w >> 8) & 0xFFu) + 11 >= (uint32_t)xref) &&
+                          (((w >> 16) & 0xFFu) + 11 >= (uint32_t)xref) && ((w >> 24) + 11 >= (uint32_t)xref);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int p = pb ^ i;                            // dims [32p, 32p+32)
+          const int sb = (int)((w >> (8 * p)) & 0xFFu);
+          uint32_t lo, hi;
+          if (fast) {
+            const uint32_t d = (uint32_t)(xref - sb) * 8u;
+            lo = 0x6C686000u - d * 0x01010100u;
+            hi = 0x7C787470u - d * 0x01010101u;
+          } else {
+            e4m3_table(sb - xref + 6, lo, hi);
+          }
+          const uint2 e0 = e2m1x8_to_e4m3(c[i].x, lo, hi), e1 = e2m1x8_to_e4m3(c[i].y, lo, hi);
+          const uint2 e2 = e2m1x8_to_e4m3(c[i].z, lo, hi), e3 = e2m1x8_to_e4m3(c[i].w, lo, hi);
+          tc::sts128(dst + (((uint32_t)(2 * p) ^ sw_row) << 4), make_uint4(e0.x, e0.y, e1.x, e1.y));
+          tc::sts128(dst + (((uint32_t)(2 * p + 1) ^ sw_row) << 4), make_uint4(e2.x, e2.y, e3.x, e3.y));
+        }
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) { tc::mbar_arrive(c_empty + cs); tc::mbar_arrive(a_full + dq); }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// Scores of the chunk rectangle (sequences [b0, b0+nb), rows [i0, i0+ni)),
+// rows laid out [nb][ni][Nc].  q8 / w8: the prepared queries of the rectangle.
+static cudaError_t launch_indexer_fp4_rect(const uint8_t* k_codes, const uint8_t* k_scales, int B, int Nc,
+                                           long long q_pos0, int m, const uint8_t* q8, const float* w8,
+                                           float* scores, int b0, int nb, int i0, int ni, cudaStream_t st) {
+  CUtensorMap qm, cm;
+  if (!make_tmap_2d(&qm, q8, 1, (uint64_t)nb * ni * 64, 128, 128, 128, 256)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&cm, k_codes, 1, (uint64_t)B * Nc, 64, 64, 64, kIxTileE, false)) return cudaErrorInvalidValue;
+  IxGeom g;
+  g.Tq = 0; g.Nc = Nc; g.H = 64;
+  g.b0 = b0; g.nb = nb; g.i0 = i0; g.ni = ni;
+  g.gps = (ni + kIxRows - 1) / kIxRows;
+  g.q_pos0 = q_pos0; g.m = m;
+  const int n_groups = nb * g.gps;
+  long long nv = (q_pos0 + i0 + ni - 1) / m;
+  if (nv > Nc) nv = Nc;
+  const int tiles = (int)((nv + kIxTileE - 1) / kIxTileE);
+  int splits = 1;
+  if (n_groups < 4 * 148) {
+    splits = (4 * 148 + n_groups - 1) / n_groups;
+    const int max_splits = tiles / 8 > 1 ? tiles / 8 : 1;
+    splits = splits < max_splits ? splits : max_splits;
+  }
+  g.splits = splits;
+  cudaError_t e = cudaFuncSetAttribute(indexer_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_groups, splits);
+  indexer_fp4_kernel<<<grid, kI4Threads, kI4Smem, st>>>(qm, cm, reinterpret_cast<const uint32_t*>(k_scales), w8,
+                                                         scores, g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace lcsa

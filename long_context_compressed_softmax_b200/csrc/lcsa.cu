@@ -13,6 +13,7 @@
 #include "rope.cuh"
 #include "indexer_tc.cuh"
 #include "attn_tc.cuh"
+#include "indexer_fp4.cuh"
 
 using namespace lcsa;
 
@@ -136,6 +137,67 @@ __global__ void nvalid_kernel(int32_t* nv, int rows, int i0, int ni, long long q
   nv[r] = (int32_t)(v < Nc ? v : Nc);
 }
 
+// Rows of one indexer chunk: at most kIndexerChunkRows score rows at a time.
+long long indexer_chunk_budget(int B, int Tq) {
+  const long long rows = (long long)B * Tq;
+  return rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
+}
+
+// Workspace of a chunk of r rows: scores + visible counts + the two-phase
+// top-k scratch + `extra_per_row` bytes per row for the score kernels.
+size_t indexer_ws_need(long long r, int Nc, int k, size_t extra_per_row) {
+  const size_t per_row = (size_t)(Nc > 0 ? Nc : 1) * 4;
+  size_t n = align256((size_t)r * per_row) + align256((size_t)r * 4) + topk_long_scratch((int)r, Nc, k);
+  if (extra_per_row) n += align256((size_t)r * 64 * 128) + align256((size_t)r * (extra_per_row - 64 * 128));
+  return n;
+}
+
+// Indexer + top-k over chunk rectangles: whole sequences when a sequence fits
+// the chunk, else row ranges of one sequence (a multiple of the 4-row query
+// group).  `scores_fn(sc, b0, nb, i0, ni, extra)` writes the rectangle's
+// scores [nb*ni][Nc] to sc; then the visible counts and the top-k follow.
+template <typename F>
+lcsa_status indexer_by_chunks(int B, int Tq, int Nc, int k, long long q_pos0, int m, int32_t* idx_out,
+                              float* scores_out, void* workspace, size_t workspace_bytes, size_t extra_per_row,
+                              cudaStream_t st, F&& scores_fn) {
+  long long budget = indexer_chunk_budget(B, Tq);
+  while (budget > 1 && indexer_ws_need(budget, Nc, k, extra_per_row) > workspace_bytes) budget >>= 1;
+  if (!workspace || indexer_ws_need(budget, Nc, k, extra_per_row) > workspace_bytes) return LCSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
+  const size_t per_row = (size_t)(Nc > 0 ? Nc : 1) * 4;
+  char* base = (char*)workspace;
+  float* sc_ws = (float*)base;
+  int32_t* nv = (int32_t*)(base + align256((size_t)budget * per_row));
+  char* tk_scratch = base + align256((size_t)budget * per_row) + align256((size_t)budget * 4);
+  const size_t tk_bytes = topk_long_scratch((int)budget, Nc, k);
+  void* extra = extra_per_row ? (void*)(tk_scratch + tk_bytes) : nullptr;
+  int nb_step, ni_step;
+  if (Tq <= budget) { nb_step = (int)(budget / Tq); ni_step = Tq; }
+  else { nb_step = 1; ni_step = budget >= 4 ? (int)(budget & ~3LL) : (int)budget; }
+  for (int b0 = 0; b0 < B; b0 += nb_step) {
+    const int nb = B - b0 < nb_step ? B - b0 : nb_step;
+    for (int i0 = 0; i0 < Tq; i0 += ni_step) {
+      const int ni = Tq - i0 < ni_step ? Tq - i0 : ni_step;
+      const long long row0 = (long long)b0 * Tq + i0;      // rectangle rows are contiguous
+      const int nr = nb * ni;
+      float* sc = scores_out ? scores_out + row0 * (long long)Nc : sc_ws;
+      cudaError_t e = cudaSuccess;
+      if (Nc > 0) {
+        e = scores_fn(sc, b0, nb, i0, ni, extra);
+        if (e != cudaSuccess) return LCSA_ERR_CUDA;
+      }
+      count_launch();
+      nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, q_pos0, m, Nc);
+      // the longest row of the rectangle is its last position's visible count
+      const long long last_vis = (q_pos0 + i0 + ni - 1) / m;
+      const int n_max = (int)(last_vis < Nc ? last_vis : Nc);
+      e = launch_topk(sc, nr, Nc, Nc, nv, k, idx_out + row0 * k, st, tk_scratch, tk_bytes, n_max);
+      if (e != cudaSuccess) return LCSA_ERR_CUDA;
+    }
+  }
+  return LCSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -232,64 +294,90 @@ int lcsa_indexer_uses_tensor_cores(const lcsa_indexer_args* a) { return a && ind
 
 size_t lcsa_indexer_topk_workspace(const lcsa_indexer_args* a) {
   if (!a || a->B <= 0 || a->Tq <= 0) return 0;
-  const long long rows = (long long)a->B * a->Tq;
-  const long long chunk = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
-  // score chunk + per-row visible counts + scratch of the two-phase top-k of long rows
-  return align256((size_t)chunk * (size_t)(a->Nc > 0 ? a->Nc : 1) * 4) + align256((size_t)chunk * 4) +
-         topk_long_scratch((int)chunk, a->Nc, a->k);
+  return indexer_ws_need(indexer_chunk_budget(a->B, a->Tq), a->Nc, a->k, 0);
 }
 
 lcsa_status lcsa_indexer_topk(const lcsa_indexer_args* a, void* workspace, size_t workspace_bytes, void* stream) {
   lcsa_status s = check_indexer(a);
   if (s != LCSA_OK) return s;
-  const long long rows = (long long)a->B * a->Tq;
-  if (rows == 0) return LCSA_OK;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
   if (!have_device()) return LCSA_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  const int Nc = a->Nc > 0 ? a->Nc : 1;
-  // Rows per chunk: as many score rows as the workspace holds (scores + counts).
-  const size_t per_row = (size_t)Nc * 4;
-  auto need = [&](long long r) {
-    return align256((size_t)r * per_row) + align256((size_t)r * 4) + topk_long_scratch((int)r, a->Nc, a->k);
-  };
-  long long budget = rows < kIndexerChunkRows ? rows : kIndexerChunkRows;
-  while (budget > 1 && need(budget) > workspace_bytes) budget >>= 1;
-  if (!workspace || need(budget) > workspace_bytes) return LCSA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
-  float* sc_ws = (float*)workspace;
-  int32_t* nv = (int32_t*)((char*)workspace + align256((size_t)budget * per_row));
-  void* tk_scratch = (char*)workspace + align256((size_t)budget * per_row) + align256((size_t)budget * 4);
-  const size_t tk_bytes = topk_long_scratch((int)budget, a->Nc, a->k);
   const bool tc = indexer_tc_supported(a);
-  // Chunk rectangles: whole sequences when a sequence fits, else row ranges of
-  // one sequence (a multiple of the 4-row query group).
-  int nb_step, ni_step;
-  if (a->Tq <= budget) { nb_step = (int)(budget / a->Tq); ni_step = a->Tq; }
-  else { nb_step = 1; ni_step = budget >= 4 ? (int)(budget & ~3LL) : (int)budget; }
-  for (int b0 = 0; b0 < a->B; b0 += nb_step) {
-    const int nb = a->B - b0 < nb_step ? a->B - b0 : nb_step;
-    for (int i0 = 0; i0 < a->Tq; i0 += ni_step) {
-      const int ni = a->Tq - i0 < ni_step ? a->Tq - i0 : ni_step;
-      const long long row0 = (long long)b0 * a->Tq + i0;      // rectangle rows are contiguous
-      const int nr = nb * ni;
-      float* sc = a->scores_out ? a->scores_out + row0 * (long long)a->Nc : sc_ws;
-      cudaError_t e = cudaSuccess;
-      if (a->Nc > 0) {
-        if (tc) e = launch_indexer_tc_rect(a, sc, b0, nb, i0, ni, st);
-        else if (a->dtype == LCSA_BF16) e = launch_indexer_generic_t<__nv_bfloat16>(a, sc, (int)row0, nr, st);
-        else e = launch_indexer_generic_t<float>(a, sc, (int)row0, nr, st);
-        if (e != cudaSuccess) return LCSA_ERR_CUDA;
-      }
-      count_launch();
-      nvalid_kernel<<<(nr + 255) / 256, 256, 0, st>>>(nv, nr, i0, ni, a->q_pos0, a->m, a->Nc);
-      // the longest row of the rectangle is its last position's visible count
-      const long long last_vis = (a->q_pos0 + i0 + ni - 1) / a->m;
-      const int n_max = (int)(last_vis < a->Nc ? last_vis : a->Nc);
-      e = launch_topk(sc, nr, a->Nc, a->Nc, nv, a->k, a->idx_out + row0 * a->k, st, tk_scratch, tk_bytes, n_max);
-      if (e != cudaSuccess) return LCSA_ERR_CUDA;
-    }
-  }
+  return indexer_by_chunks(a->B, a->Tq, a->Nc, a->k, a->q_pos0, a->m, a->idx_out, a->scores_out, workspace,
+                           workspace_bytes, 0, st,
+                           [&](float* sc, int b0, int nb, int i0, int ni, void*) -> cudaError_t {
+                             const long long row0 = (long long)b0 * a->Tq + i0;
+                             if (tc) return launch_indexer_tc_rect(a, sc, b0, nb, i0, ni, st);
+                             if (a->dtype == LCSA_BF16)
+                               return launch_indexer_generic_t<__nv_bfloat16>(a, sc, (int)row0, nb * ni, st);
+                             return launch_indexer_generic_t<float>(a, sc, (int)row0, nb * ni, st);
+                           });
+}
+
+// ------------------------------------------------------------------ FP4 indexer path
+lcsa_status lcsa_quantize_mxfp4(const void* x, int64_t rows, int cols, lcsa_dtype dtype, uint8_t* codes,
+                                uint8_t* scales, void* stream) {
+  if (!valid_dtype(dtype) || rows < 0 || cols <= 0 || cols % 32 != 0) return LCSA_ERR_INVALID_ARG;
+  if (rows == 0) return LCSA_OK;
+  if (!x || !codes || !scales) return LCSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) % esize(dtype) != 0) return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  const long long n_blocks = rows * (long long)(cols / 32);
+  const long long want = (n_blocks + 7) / 8;                       // 8 warps (blocks of 32 values) per CTA
+  const int grid = (int)(want < 148LL * 64 ? want : 148LL * 64);
+  count_launch();
+  if (dtype == LCSA_BF16)
+    mxfp4_quantize_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (const __nv_bfloat16*)x, n_blocks, codes, scales);
+  else
+    mxfp4_quantize_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>((const float*)x, n_blocks, codes, scales);
+  return from_cuda(cudaGetLastError());
+}
+
+static lcsa_status check_indexer_mxfp4(const lcsa_indexer_mxfp4_args* a) {
+  if (!a) return LCSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->Tq < 0 || a->Nc < 0 || a->H_I <= 0 || a->D_I <= 0 || a->m <= 0 || a->k <= 0 || a->q_pos0 < 0)
+    return LCSA_ERR_INVALID_ARG;
+  if (a->H_I != 64 || a->D_I != 128) return LCSA_ERR_UNSUPPORTED;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if (!a->q_idx || !a->w || !a->idx_out || (a->Nc > 0 && (!a->k_codes || !a->k_scales))) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(a->q_idx) || !aligned16(a->w) || !aligned16(a->idx_out) ||
+      (a->k_codes && !aligned16(a->k_codes)) || (a->k_scales && (reinterpret_cast<uintptr_t>(a->k_scales) & 3u)) ||
+      (a->scores_out && !aligned16(a->scores_out)))
+    return LCSA_ERR_INVALID_ARG;
   return LCSA_OK;
+}
+
+// prepared queries of one rectangle: E4M3 [rows*64, 128] + head weights [rows*64]
+static constexpr size_t kQ8PerRow = 64 * 128 + 64 * 4;
+
+size_t lcsa_indexer_topk_mxfp4_workspace(const lcsa_indexer_mxfp4_args* a) {
+  if (!a || a->B <= 0 || a->Tq <= 0) return 0;
+  return indexer_ws_need(indexer_chunk_budget(a->B, a->Tq), a->Nc, a->k, kQ8PerRow);
+}
+
+lcsa_status lcsa_indexer_topk_mxfp4(const lcsa_indexer_mxfp4_args* a, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  lcsa_status s = check_indexer_mxfp4(a);
+  if (s != LCSA_OK) return s;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  return indexer_by_chunks(
+      a->B, a->Tq, a->Nc, a->k, a->q_pos0, a->m, a->idx_out, a->scores_out, workspace, workspace_bytes, kQ8PerRow,
+      st, [&](float* sc, int b0, int nb, int i0, int ni, void* extra) -> cudaError_t {
+        const long long nr = (long long)nb * ni;
+        uint8_t* q8 = (uint8_t*)extra;
+        float* w8 = (float*)(q8 + align256((size_t)nr * 64 * 128));
+        count_launch();
+        indexer_q8_kernel<<<(unsigned)((nr * 64 + 7) / 8), 256, 0, st>>>(
+            (const __nv_bfloat16*)a->q_idx, a->w, a->Tq, b0, nb, i0, ni, q8, w8);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_indexer_fp4_rect(a->k_codes, a->k_scales, a->B, a->Nc, a->q_pos0, a->m, q8, w8, sc, b0, nb,
+                                       i0, ni, st);
+      });
 }
 
 int lcsa_attn_uses_tensor_cores(const lcsa_attn_args* a) { return a && attn_tc_supported(a) ? 1 : 0; }

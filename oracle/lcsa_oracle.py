@@ -185,24 +185,30 @@ E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
 def mx_scale_exponent(amax):
-    """Shared exponent of one block: X = floor(log2(amax)) - 2 (2 = the largest
-    E2M1 exponent, so amax / 2^X lies in [4, 8)), clamped to the UE8M0 range
-    [-127, 127]; an all-zero block takes X = -127."""
-    if amax == 0.0:
-        return -127
-    _, e = math.frexp(amax)          # amax = f * 2^e, f in [0.5, 1)
-    return max(-127, min(127, (e - 1) - 2))
+    """Shared exponent of blocks with largest magnitudes `amax` (array):
+    X = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent, so amax / 2^X
+    lies in [4, 8)), clamped to the UE8M0 range [-127, 127]; an all-zero
+    block takes X = -127."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, e = np.frexp(amax)            # amax = f * 2^e, f in [0.5, 1)
+    X = np.clip((e - 1) - 2, -127, 127)
+    return np.where(amax == 0.0, -127, X).astype(np.int64)
+
+
+def e2m1_codes(y):
+    """4-bit E2M1 codes of the values nearest to y (array): round to nearest,
+    ties to the code with an even mantissa bit (code bit 0), magnitudes above
+    6 saturate to 6; bit 3 is the sign of y."""
+    y = np.asarray(y, dtype=np.float64)
+    d = np.abs(np.abs(y)[..., None] - E2M1_VALUES)          # distance to each magnitude
+    near = d == d.min(axis=-1, keepdims=True)
+    even = near & (np.arange(8) % 2 == 0)
+    c = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(near, axis=-1))
+    return (c | np.where(y < 0, 8, 0)).astype(np.uint8)
 
 
 def e2m1_code(y):
-    """4-bit E2M1 code of the value nearest to y (round to nearest, ties to the
-    code with an even mantissa bit, magnitudes above 6 saturate to 6); bit 3 is
-    the sign of y."""
-    a = abs(y)
-    d = np.abs(E2M1_VALUES - a)
-    best = np.flatnonzero(d == d.min())
-    c = int(best[0]) if len(best) == 1 else int(best[best % 2 == 0][0])
-    return c | (8 if y < 0 else 0)
+    return int(e2m1_codes(np.array([y]))[0])
 
 
 def quantize_mxfp4(x):
@@ -211,26 +217,25 @@ def quantize_mxfp4(x):
     Returns (codes uint8 [..., C/2], scales uint8 [..., C/32]): byte i of a
     row's codes holds element 2i in its low nibble and 2i+1 in its high
     nibble; a block holding a non-finite value gets scale byte 255 and zero
-    codes.  Written for clarity, not speed: loops over blocks."""
+    codes."""
     x = np.asarray(x, dtype=np.float64)
     C = x.shape[-1]
     assert C % MX_BLOCK == 0
-    flat = x.reshape(-1, C)
-    codes = np.zeros((flat.shape[0], C // 2), dtype=np.uint8)
-    scales = np.zeros((flat.shape[0], C // MX_BLOCK), dtype=np.uint8)
-    for r in range(flat.shape[0]):
-        for b in range(C // MX_BLOCK):
-            blk = flat[r, b * MX_BLOCK:(b + 1) * MX_BLOCK]
-            if not np.isfinite(blk).all():
-                scales[r, b] = 255
-                continue
-            X = mx_scale_exponent(float(np.abs(blk).max()))
-            scales[r, b] = X + 127
-            for i in range(MX_BLOCK):
-                c = e2m1_code(math.ldexp(float(blk[i]), -X))
-                col = b * MX_BLOCK + i
-                codes[r, col // 2] |= np.uint8(c << (4 * (col % 2)))
-    return codes.reshape(x.shape[:-1] + (C // 2,)), scales.reshape(x.shape[:-1] + (C // MX_BLOCK,))
+    rows = x.size // C if C else 0
+    if rows > 8192:                   # bound the temporaries: quantise in row slices
+        flat = x.reshape(rows, C)
+        parts = [quantize_mxfp4(flat[r:r + 8192]) for r in range(0, rows, 8192)]
+        return (np.concatenate([p[0] for p in parts]).reshape(x.shape[:-1] + (C // 2,)),
+                np.concatenate([p[1] for p in parts]).reshape(x.shape[:-1] + (C // MX_BLOCK,)))
+    blk = x.reshape(x.shape[:-1] + (C // MX_BLOCK, MX_BLOCK))
+    finite = np.isfinite(blk).all(axis=-1)
+    amax = np.where(finite, np.abs(np.where(np.isfinite(blk), blk, 0.0)).max(axis=-1), 0.0)
+    X = mx_scale_exponent(amax)
+    y = np.ldexp(np.where(np.isfinite(blk), blk, 0.0), -X[..., None])   # exact: a power-of-two scaling
+    c = np.where(finite[..., None], e2m1_codes(y), 0).astype(np.uint8).reshape(x.shape)
+    codes = (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+    scales = np.where(finite, X + 127, 255).astype(np.uint8)
+    return codes, scales
 
 
 def dequantize_mxfp4(codes, scales):

@@ -45,7 +45,9 @@ def test_struct_layouts_match_header(lcsa, tmp_path):
     """The ctypes mirrors have the C structs' size and field offsets (gcc)."""
     import subprocess
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "lcsa.h"', 'int main(void){']
-    for cname, py in (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs)):
+    structs = (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs),
+               ("lcsa_indexer_mxfp4_args", lcsa.IndexerMxfp4Args))
+    for cname, py in structs:
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in py._fields_:
             lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
@@ -55,7 +57,7 @@ def test_struct_layouts_match_header(lcsa, tmp_path):
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines())
-    for cname, py in (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs)):
+    for cname, py in structs:
         assert int(got[cname]) == ctypes.sizeof(py)
         for f, _ in py._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -107,6 +109,30 @@ def test_compress_entries_checks_windows(lcsa):
     if not torch.cuda.is_available():
         assert L.lcsa_compress_entries(*args(61, 1, 64)) == 4          # valid, but no device: no CPU path
         assert L.lcsa_compress_entries(*args(31, 30, 64)) == 4         # entries 31..60 pool [120, 244)
+
+
+def test_mxfp4_calls_check_arguments(lcsa):
+    L = lcsa.lib
+    x, c, sc = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000)
+    assert L.lcsa_quantize_mxfp4(x, 4, 48, lcsa.LCSA_BF16, c, sc, None) == 1       # cols not a multiple of 32
+    assert L.lcsa_quantize_mxfp4(None, 4, 64, lcsa.LCSA_BF16, c, sc, None) == 1    # null input
+    assert L.lcsa_quantize_mxfp4(ctypes.c_void_p(0x1001), 4, 64, lcsa.LCSA_BF16, c, sc, None) == 1   # misaligned
+    assert L.lcsa_quantize_mxfp4(None, 0, 64, lcsa.LCSA_BF16, None, None, None) == 0  # nothing to do
+    a = lcsa.IndexerMxfp4Args()
+    a.q_idx, a.w, a.k_codes, a.k_scales, a.idx_out = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000
+    a.B, a.Tq, a.Nc, a.H_I, a.D_I, a.m, a.k = 1, 4, 8, 64, 64, 4, 8
+    assert L.lcsa_indexer_topk_mxfp4(ctypes.byref(a), None, 0, None) == 2         # D_I = 64: unsupported
+    a.D_I = 128
+    a.k_scales = 0x4002
+    assert L.lcsa_indexer_topk_mxfp4(ctypes.byref(a), None, 0, None) == 1         # misaligned scales
+    a.k_scales, a.m = 0x4000, 0
+    assert L.lcsa_indexer_topk_mxfp4(ctypes.byref(a), None, 0, None) == 1         # m = 0
+    a.m = 4
+    assert L.lcsa_indexer_topk_mxfp4_workspace(ctypes.byref(a)) > L.lcsa_indexer_topk_workspace(
+        ctypes.byref(lcsa.IndexerArgs(None, None, None, 1, 4, 8, 64, 128, lcsa.LCSA_BF16, 0, 4, 8, None, None)))
+    if not torch.cuda.is_available():
+        ws = ctypes.c_void_p(0x10000)
+        assert L.lcsa_indexer_topk_mxfp4(ctypes.byref(a), ws, 1 << 20, None) == 4   # no device: no CPU path
 
 
 def test_empty_problems_are_noops(lcsa):

@@ -168,6 +168,30 @@ def test_csa_decode_1m_full(lcsa):
     assert lcsa.get_device_status() == 0
 
 
+def test_csa_decode_1m_fp4_indexer_full(lcsa):
+    """FP4 QK path at the decode size: MXFP4 keys (bit-exact with the oracle's
+    quantiser), scores within 1e-3 relative of the oracle's on the quantised
+    values, selection bit-exact on the GPU's scores."""
+    cfg = get_config("csa_decode_1m")
+    B, T, Nc, m = cfg.B, cfg.T, cfg.T // cfg.m, cfg.m
+    ix = gen.make_indexer_inputs(B, 1, Nc, cfg.H_I, cfg.D_I, "bf16", seed=1211, device=DEV,
+                                 boost_frac=cfg.boost_frac)
+    kc, ks = lcsa.quantize_mxfp4(ix["k_idx"])
+    idx, sc = lcsa.indexer_topk_mxfp4(ix["q_idx"], ix["w"], kc, ks, T, m, cfg.k, return_scores=True)
+    for b in (0, 63):
+        rkc, rks = O.quantize_mxfp4(np64(ix["k_idx"][b]))
+        np.testing.assert_array_equal(kc[b].cpu().numpy(), rkc)
+        np.testing.assert_array_equal(ks[b].cpu().numpy(), rks)
+        ref_idx, ref_s = O.indexer_topk_mxfp4(np64(ix["q_idx"][b]), np64(ix["w"][b]), rkc, rks, T, m, cfg.k)
+        got_s, ref = np64(sc[b, 0]), ref_s[0]
+        scale = np.maximum(np.abs(ref), np.sqrt(np.mean(ref * ref)))
+        assert (np.abs(got_s - ref) <= 1e-3 * scale).all()
+        got = idx[b, 0].cpu().numpy()
+        np.testing.assert_array_equal(got, O.topk_select(got_s, cfg.k))
+        assert len(set(got.tolist()) & set(ref_idx[0].tolist())) >= 0.999 * cfg.k
+    assert lcsa.get_device_status() == 0
+
+
 def test_stack_layers_full(lcsa):
     cfg = get_config("stack_4layer_128k")
     _run_csa_layer(lcsa, cfg, seed=1301, n_rows=12)

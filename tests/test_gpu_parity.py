@@ -241,6 +241,104 @@ def test_indexer_scores_and_recall(lcsa, dtype, H_I, D_I, Tq, Nc, m, k, q_pos0):
     assert hits >= 0.999 * tot, f"recall {hits / tot:.5f}"
 
 
+# ------------------------------------------------------------------ FP4 (MXFP4) indexer path
+def _mx_inputs(seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(37, 160, generator=g) * torch.exp2(torch.randint(-30, 30, (37, 1), generator=g).float())
+    # round-to-nearest-even midpoints and saturation (amax 7 fixes X = 0)
+    x[0, :32] = torch.tensor([7.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.75, -5.0, -0.25, 0.0] + [0.1] * 20)
+    x[1, :32] = 0.0                                   # all-zero block
+    x[1, 32:64] = -0.0
+    x[2, :32] = 1e-40 * torch.arange(32)              # FP32 subnormals
+    x[3, 64:96] = torch.linspace(-6, 6, 32) * 2.0 ** 100
+    x[4, 96:128] = torch.linspace(-1, 1, 32) * 2.0 ** -126
+    return x
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_quantize_mxfp4_bit_exact(lcsa, dtype):
+    x = _mx_inputs(61)
+    if dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    codes, scales = lcsa.quantize_mxfp4(x.to(DEV))
+    rc, rs = O.quantize_mxfp4(x.double().numpy())
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+
+
+def test_quantize_mxfp4_nonfinite_blocks(lcsa):
+    x = torch.randn(3, 96, generator=torch.Generator().manual_seed(62))
+    x[0, 3] = float("nan")
+    x[1, 40] = float("inf")
+    x[2, 95] = -float("inf")
+    codes, scales = lcsa.quantize_mxfp4(x.to(DEV))
+    rc, rs = O.quantize_mxfp4(x.double().numpy())
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    assert rs[0, 0] == 255 and rs[1, 1] == 255 and rs[2, 2] == 255
+
+
+@pytest.mark.parametrize("Tq,Nc,m,k,q_pos0", [
+    (260, 1030, 4, 256, 3900),      # 4-row query groups, several tiles + ragged tail
+    (37, 700, 4, 2048, 0),          # N_vis < k everywhere
+    (1, 3000, 4, 512, 12000),       # decode: one row per sequence, entry-range splits
+    (6, 2100, 4, 128, 8000),        # a 4-row and a 2-row group
+    (3, 20000, 4, 2048, 80000),     # long rows: two-phase top-k
+])
+def test_indexer_mxfp4_scores_and_selection(lcsa, Tq, Nc, m, k, q_pos0):
+    B = 2
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=43, device=DEV)
+    kc, ks = lcsa.quantize_mxfp4(x["k_idx"])
+    idx, sc = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    hits = tot = 0
+    for b in range(B):
+        rkc, rks = O.quantize_mxfp4(np64(x["k_idx"][b]))
+        np.testing.assert_array_equal(kc[b].cpu().numpy(), rkc)
+        np.testing.assert_array_equal(ks[b].cpu().numpy(), rks)
+        ref_idx, ref_s = O.indexer_topk_mxfp4(np64(x["q_idx"][b]), np64(x["w"][b]), rkc, rks, q_pos0, m, k)
+        nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+        _score_err_ok(np64(sc[b]), ref_s, nv)
+        got = idx[b].cpu().numpy()
+        for i in range(Tq):
+            v = got[i][got[i] >= 0]
+            assert (np.diff(v) > 0).all() and (v < max(nv[i], 1)).all()
+            assert len(v) == min(k, nv[i]) and (got[i][len(v):] == -1).all()
+            hits += len(set(v) & set(ref_idx[i][ref_idx[i] >= 0]))
+            tot += int((ref_idx[i] >= 0).sum())
+        np.testing.assert_array_equal(got, O.topk_from_scores(np64(sc[b]), nv, k))
+    assert hits >= 0.999 * tot, f"recall {hits / tot:.5f}"
+
+
+def test_indexer_mxfp4_wide_block_scales(lcsa):
+    # entries whose blocks differ by up to 2^13 stay exact on the E4M3 staging;
+    # one block 2^20 below its entry's largest rounds there, within tolerance
+    B, Tq, Nc, m, k, q_pos0 = 1, 4, 300, 4, 64, 1400
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=44, device=DEV)
+    kf = x["k_idx"].float()
+    kf[0, :, 32:64] *= 2.0 ** -13
+    kf[0, :, 64:96] *= 2.0 ** 6
+    kf[0, 7, 96:128] *= 2.0 ** -20
+    k_idx = kf.to(torch.bfloat16)
+    kc, ks = lcsa.quantize_mxfp4(k_idx)
+    idx, sc = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    rkc, rks = O.quantize_mxfp4(np64(k_idx[0]))
+    ref_idx, ref_s = O.indexer_topk_mxfp4(np64(x["q_idx"][0]), np64(x["w"][0]), rkc, rks, q_pos0, m, k)
+    nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+    _score_err_ok(np64(sc[0]), ref_s, nv)
+    np.testing.assert_array_equal(idx[0].cpu().numpy(), O.topk_from_scores(np64(sc[0]), nv, k))
+
+
+def test_indexer_mxfp4_small_workspace_chunks(lcsa):
+    B, Tq, Nc, m, k, q_pos0 = 2, 40, 900, 4, 128, 3600
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=45, device=DEV)
+    kc, ks = lcsa.quantize_mxfp4(x["k_idx"])
+    full = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k)
+    need = lcsa.indexer_mxfp4_workspace_bytes(x["q_idx"], kc, k)
+    small = torch.empty(need // 9, dtype=torch.uint8, device=DEV)     # a few rows at a time
+    part = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, workspace=small)
+    assert torch.equal(full, part)
+
+
 # ------------------------------------------------------------------ attention
 def _attn_case(B, Tq, H, D, Nc, Tkv, dtype, seed, unit=True, sink=True):
     return gen.make_attn_inputs(B, Tq, H, D, Nc, Tkv, dtype, seed=seed, device=DEV, unit_scale=unit,
