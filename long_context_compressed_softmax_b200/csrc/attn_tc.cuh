@@ -890,13 +890,6 @@ static AtPlan attn_tc_plan(const lcsa_attn_args* a, int sparse) {
 
 static size_t attn_tc_workspace(const lcsa_attn_args* a, int sparse) { return attn_tc_plan(a, sparse).total; }
 
-static int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws, cudaStream_t st) {
   const AtPlan pl = attn_tc_plan(a, sparse);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);

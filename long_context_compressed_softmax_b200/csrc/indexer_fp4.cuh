@@ -7,12 +7,14 @@
 // bytes per entry, a quarter of BF16), which is what bounds long-context
 // decode: every decode step streams all of them.  Per 128-entry tile:
 //   TMA        packed codes -> shared memory (8-deep ring)
-//   dequant    8 warps, two per tile (4 tiles in flight), write E4M3 in the
+//   dequant    8 warps, two per tile (4 tiles in flight, 8 stages), write E4M3 in the
 //              128B-swizzled K-major layout, each entry relative to its
 //              largest block exponent (exact for blocks within 2^13 of it,
 //              see mxfp4.cuh)
 //   MMA        tcgen05 kind::f8f6f4, M = 128 entries, N = 64 heads x up to 4
 //              query rows (E4M3 queries prepared by indexer_q8_kernel), K = 128
+//   accumulators  512 TMEM columns split into 2-8 slots (64 x query rows
+//              columns each), so the MMA runs up to 8 tiles ahead of the epilogue
 //   epilogue   8 warps: ReLU, head weights (with the query factors folded
 //              in) and the entry factor 2^(Xref - 6), one score per lane;
 //              with 3-4 query rows each warp scores 2 rows of every tile,
@@ -32,13 +34,18 @@ namespace lcsa {
 constexpr int kI4CStages = 8;                  // packed-code ring
 constexpr int kI4DqWarp0 = 10;
 constexpr int kI4DqWarps = 8;                  // warps 2t, 2t+1 of the group expand tiles t, t+4, t+8, ...
-constexpr int kI4AStages = kI4DqWarps / 2;     // E4M3 key tiles in flight: one per dequantiser pair
+constexpr int kI4Pairs = kI4DqWarps / 2;       // tiles being expanded at once
+constexpr int kI4AStages = 2 * kI4Pairs;       // E4M3 key tiles: two per pair, so a pair never waits for the
+                                               // MMA of the tile it just handed over
 constexpr int kI4Threads = (kI4DqWarp0 + kI4DqWarps) * 32;   // 576
 constexpr uint32_t kI4QBytes = 256 * 128;      // 4 query rows x 64 heads x 128 E4M3
 constexpr uint32_t kI4ABytes = kIxTileE * 128; // 128 entries x 128 E4M3
 constexpr uint32_t kI4CBytes = kIxTileE * 64;  // 128 entries x 64 code bytes
+constexpr int kI4MaxAcc = 8;                   // TMEM accumulator slots (512 / (64 x query rows), up to 8)
+constexpr int kI4Bars = 1 + 2 * kI4CStages + 2 * kI4AStages + 2 * kI4MaxAcc;
 constexpr size_t kI4Smem = 1024 + kI4QBytes + kI4AStages * kI4ABytes + kI4CStages * kI4CBytes + kIxRows * 64 * 4 +
-                           256;
+                           kI4Bars * 8;
+static_assert(kI4Smem + 64 <= 232448, "shared memory of the FP4 indexer kernel");
 // Piece order of the dequantisers: the lane of row r handles code block
 // p = kI4Perm[(r >> 1) & 3] ^ i at step i, so that both the 64-byte-strided
 // code reads and the swizzled 16-byte writes of 8 consecutive rows hit 8
@@ -86,7 +93,7 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
   uint64_t* a_full = c_empty + kI4CStages;
   uint64_t* a_empty = a_full + kI4AStages;
   uint64_t* acc_full = a_empty + kI4AStages;
-  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* acc_empty = acc_full + kI4MaxAcc;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -112,13 +119,20 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
   const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
   if (n_tiles == 0) return;
   const long long rect_row = (long long)bl * g.ni + (i_first - g.i0);   // first query row in the rectangle
+  // TMEM accumulator slots: 64 x rows columns each, as many as fit in 512 (8, 4 or 2);
+  // with 1-2 rows the epilogue halves take alternate tiles, so every slot stays with one half
+  const int n_acc = rows == 1 ? 8 : rows == 2 ? 4 : 2;
+  const uint32_t acc_cols = 512u / (uint32_t)n_acc;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
     for (int s = 0; s < kI4CStages; ++s) { tc::mbar_init(c_full + s, 1); tc::mbar_init(c_empty + s, 2); }
     for (int s = 0; s < kI4AStages; ++s) { tc::mbar_init(a_full + s, 2); tc::mbar_init(a_empty + s, 1); }
     // rows > 2: all 8 epilogue warps read every accumulator; else 4 per accumulator
-    for (int a = 0; a < 2; ++a) { tc::mbar_init(acc_full + a, 1); tc::mbar_init(acc_empty + a, rows > 2 ? 8 : 4); }
+    for (int a = 0; a < kI4MaxAcc; ++a) {
+      tc::mbar_init(acc_full + a, 1);
+      tc::mbar_init(acc_empty + a, rows > 2 ? 8 : 4);
+    }
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -163,17 +177,17 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
       const uint32_t b_base = tc::smem_u32(s_q);
       for (int n = 0; ok && n < n_tiles; ++n) {
         const int s = n % kI4AStages, r = n / kI4AStages;
-        const int a = n & 1, ra = n >> 1;
+        const int a = n % n_acc, ra = n / n_acc;
         if (*abort_flag) break;
-        if (!tc::mbar_wait(a_full + s, r & 1)) { ok = false; break; }
-        if (ra > 0 && !tc::mbar_wait(acc_empty + a, (ra - 1) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait_spin(a_full + s, r & 1)) { ok = false; break; }
+        if (ra > 0 && !tc::mbar_wait_spin(acc_empty + a, (ra - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t a_base = tc::smem_u32(s_a + s * kI4ABytes);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ad = tc::sdesc_sw128(a_base + ks * 32, 16, 1024);
           const uint64_t bd = tc::sdesc_sw128(b_base + ks * 32, 16, 1024);
-          mma_e4m3_ss(tmem + a * 256, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          mma_e4m3_ss(tmem + (uint32_t)a * acc_cols, ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         tc::mma_commit(a_empty + s);
         tc::mma_commit(acc_full + a);
@@ -199,7 +213,7 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
     // scale words of the next three tiles this warp scores
     uint32_t sw1 = scale_word(n_first), sw2 = scale_word(n_first + n_step), sw3 = scale_word(n_first + 2 * n_step);
     for (int n = n_first; n_q > 0 && n < n_tiles; n += n_step) {
-      const int a = n & 1, ra = n >> 1;
+      const int a = n % n_acc, ra = n / n_acc;
       const long long j = (long long)(t_begin + n) * kIxTileE + quarter * 32 + lane;
       const uint32_t sw = sw1;
       sw1 = sw2; sw2 = sw3; sw3 = scale_word(n + 3 * n_step);
@@ -211,9 +225,11 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         if (qq < n_q) {
-          const uint32_t col = tmem + lane_addr + (uint32_t)(a * 256 + (q0 + qq) * 64);
+          const uint32_t col = tmem + lane_addr + (uint32_t)a * acc_cols + (uint32_t)((q0 + qq) * 64);
           const uint32_t wq = tc::smem_u32(s_w + (q0 + qq) * 64);
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};     // four partial sums over heads h = 4i + c
+          // w relu(x) = (w/2) x + (w/2) |x| on the FMA pipe (the prepared weights
+          // carry the 1/2); eight partial sums: heads h = 4i + c, x and |x| terms
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int hb = 0; hb < 64; hb += 32) {     // 32 heads at a time
             uint32_t v[32];
@@ -227,13 +243,15 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 #pragma unroll
             for (int h = 0; h < 32; h += 4) {
               const float4 w4 = tc::lds128f(wq + (hb + h) * 4);
-              acc[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[h]), 0.f), acc[0]);
-              acc[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), acc[1]);
-              acc[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), acc[2]);
-              acc[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), acc[3]);
+              const float x0 = __uint_as_float(v[h]), x1 = __uint_as_float(v[h + 1]);
+              const float x2 = __uint_as_float(v[h + 2]), x3 = __uint_as_float(v[h + 3]);
+              acc[0] = fmaf(w4.x, x0, acc[0]); acc[4] = fmaf(w4.x, fabsf(x0), acc[4]);
+              acc[1] = fmaf(w4.y, x1, acc[1]); acc[5] = fmaf(w4.y, fabsf(x1), acc[5]);
+              acc[2] = fmaf(w4.z, x2, acc[2]); acc[6] = fmaf(w4.z, fabsf(x2), acc[6]);
+              acc[3] = fmaf(w4.w, x3, acc[3]); acc[7] = fmaf(w4.w, fabsf(x3), acc[7]);
             }
           }
-          sc[qq] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          sc[qq] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
         }
       }
       const float f = pow2f(max_scale_byte(sw) - 127 - 6);
@@ -246,10 +264,16 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
   } else {
     // ------------------------------------------------------------ dequantisers
     // warps 2t and 2t+1 of the group expand tiles n = t, t + 4, ... into E4M3
-    // stage t; the lane of warp 2t + hh handles entry rows lane + 32 (2 hh + jr)
+    // stage n % 8; the lane of warp 2t + hh handles entry rows lane + 32 (2 hh + jr)
     const int dq = (warp - kI4DqWarp0) >> 1, hh = (warp - kI4DqWarp0) & 1;
     const int pb = kI4Perm[(lane >> 1) & 3];
-    const uint32_t sw_row = (uint32_t)(lane & 7);
+    // per-lane constants: step i reads code block p = pb ^ i at byte offset
+    // (pb ^ i) * 16 of the row and writes its two 16-byte E4M3 chunks 2p, 2p+1
+    // at swizzled offsets ((2p + h) ^ (row & 7)) * 16 = st_base ^ (32 i) ^ (16 h)
+    const uint32_t ld_base = (uint32_t)pb << 4;
+    const uint32_t st_base = ((uint32_t)(2 * pb) ^ (uint32_t)(lane & 7)) << 4;
+    // byte i of prmt(w, 0, psel) = scale byte of block pb ^ i
+    const uint32_t psel = (uint32_t)pb | ((uint32_t)(pb ^ 1) << 4) | ((uint32_t)(pb ^ 2) << 8) | ((uint32_t)(pb ^ 3) << 12);
     auto scale_words = [&](int n, uint32_t* sw) {
 #pragma unroll
       for (int jr = 0; jr < 2; ++jr) {
@@ -259,51 +283,51 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
     };
     uint32_t cur[2], nxt[2];                    // this warp's next two tiles
     scale_words(dq, cur);
-    scale_words(dq + kI4AStages, nxt);
-    for (int n = dq; n < n_tiles; n += kI4AStages) {
+    scale_words(dq + kI4Pairs, nxt);
+    for (int n = dq; n < n_tiles; n += kI4Pairs) {
       const int cs = n % kI4CStages, rc = n / kI4CStages;
-      const int ra = n / kI4AStages;
+      const int as = n % kI4AStages, ra = n / kI4AStages;
       uint32_t sw[2];
 #pragma unroll
       for (int jr = 0; jr < 2; ++jr) { sw[jr] = cur[jr]; cur[jr] = nxt[jr]; }
-      scale_words(n + 2 * kI4AStages, nxt);
+      scale_words(n + 2 * kI4Pairs, nxt);
       bool ok = !*abort_flag && tc::mbar_wait(c_full + cs, rc & 1);
-      ok = ok && (ra == 0 || tc::mbar_wait(a_empty + dq, (ra - 1) & 1));
+      ok = ok && (ra == 0 || tc::mbar_wait(a_empty + as, (ra - 1) & 1));
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
 #pragma unroll
       for (int jr = 0; jr < 2; ++jr) {
         const int r = lane + 32 * (2 * hh + jr);
         const uint32_t w = sw[jr];
-        const int xref = max_scale_byte(w);
-        const uint32_t src = tc::smem_u32(s_c) + cs * kI4CBytes + r * 64;
-        const uint32_t dst = tc::smem_u32(s_a) + dq * kI4ABytes + r * 128;
+        const uint32_t xref = (uint32_t)max_scale_byte(w);
+        const uint32_t src = tc::smem_u32(s_c) + cs * kI4CBytes + r * 64;      // 64-byte aligned
+        const uint32_t dst = tc::smem_u32(s_a) + as * kI4ABytes + r * 128;     // 128-byte aligned
         uint4 c[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c[i] = tc::lds128(src + (uint32_t)(pb ^ i) * 16);   // code block pb ^ i
+        for (int i = 0; i < 4; ++i) c[i] = tc::lds128(src | (ld_base ^ (uint32_t)(16 * i)));
+        // byte i of dl: xref - (scale byte of block pb ^ i), never borrowing
+        const uint32_t dl = xref * 0x01010101u - __byte_perm(w, 0, psel);
         // every block within 2^11 of the entry's largest: table by exponent-field arithmetic
-        const bool fast = ((w & 0xFFu) + 11 >= (uint32_t)xref) && (((w >> 8) & 0xFFu) + 11 >= (uint32_t)xref) &&
-                          (((w >> 16) & 0xFFu) + 11 >= (uint32_t)xref) && ((w >> 24) + 11 >= (uint32_t)xref);
+        const bool fast = ((dl | (dl + 0x04040404u)) & 0xF0F0F0F0u) == 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int p = pb ^ i;                            // dims [32p, 32p+32)
-          const int sb = (int)((w >> (8 * p)) & 0xFFu);
+          const uint32_t d = (dl >> (8 * i)) & 0xFFu;
           uint32_t lo, hi;
           if (fast) {
-            const uint32_t d = (uint32_t)(xref - sb) * 8u;
-            lo = 0x6C686000u - d * 0x01010100u;
-            hi = 0x7C787470u - d * 0x01010101u;
+            lo = 0x6C686000u - d * 0x08080800u;
+            hi = 0x7C787470u - d * 0x08080808u;
           } else {
-            e4m3_table(sb - xref + 6, lo, hi);
+            e4m3_table(6 - (int)d, lo, hi);
           }
           const uint2 e0 = e2m1x8_to_e4m3(c[i].x, lo, hi), e1 = e2m1x8_to_e4m3(c[i].y, lo, hi);
           const uint2 e2 = e2m1x8_to_e4m3(c[i].z, lo, hi), e3 = e2m1x8_to_e4m3(c[i].w, lo, hi);
-          tc::sts128(dst + (((uint32_t)(2 * p) ^ sw_row) << 4), make_uint4(e0.x, e0.y, e1.x, e1.y));
-          tc::sts128(dst + (((uint32_t)(2 * p + 1) ^ sw_row) << 4), make_uint4(e2.x, e2.y, e3.x, e3.y));
+          const uint32_t o = st_base ^ (uint32_t)(32 * i);
+          tc::sts128(dst | o, make_uint4(e0.x, e0.y, e1.x, e1.y));
+          tc::sts128(dst | (o ^ 16u), make_uint4(e2.x, e2.y, e3.x, e3.y));
         }
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) { tc::mbar_arrive(c_empty + cs); tc::mbar_arrive(a_full + dq); }
+      if (lane == 0) { tc::mbar_arrive(c_empty + cs); tc::mbar_arrive(a_full + as); }
     }
   }
   tc::tc_fence_before();
@@ -331,12 +355,7 @@ static cudaError_t launch_indexer_fp4_rect(const uint8_t* k_codes, const uint8_t
   long long nv = (q_pos0 + i0 + ni - 1) / m;
   if (nv > Nc) nv = Nc;
   const int tiles = (int)((nv + kIxTileE - 1) / kIxTileE);
-  int splits = 1;
-  if (n_groups < 4 * 148) {
-    splits = (4 * 148 + n_groups - 1) / n_groups;
-    const int max_splits = tiles / 8 > 1 ? tiles / 8 : 1;
-    splits = splits < max_splits ? splits : max_splits;
-  }
+  const int splits = indexer_splits(n_groups, tiles);
   g.splits = splits;
   cudaError_t e = cudaFuncSetAttribute(indexer_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem);
   if (e != cudaSuccess) return e;

@@ -194,6 +194,31 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_consta
   }
 }
 
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// Entry-range splits per query group when there are few groups (decode): the
+// split count s (at most tiles / 8, so a CTA keeps >= 8 tiles) that minimises
+// the waves of one-CTA-per-SM launches times the tiles per CTA, with a
+// per-CTA start-up cost of about 6 tiles.  Many groups: no split.
+static int indexer_splits(int n_groups, int tiles) {
+  const int sms = sm_count();
+  if (n_groups >= 4 * sms) return 1;
+  const int max_splits = tiles / 8 > 1 ? tiles / 8 : 1;
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= max_splits; ++s) {
+    const long long waves = ((long long)n_groups * s + sms - 1) / sms;
+    const long long cost = waves * ((tiles + s - 1) / s + 6);
+    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
+  }
+  return best;
+}
+
 // Scores for the chunk rectangle: sequences [b0, b0+nb), query rows [i0, i0+ni)
 // of each; scores rows laid out [nb][ni][Nc].
 static cudaError_t launch_indexer_tc_rect(const lcsa_indexer_args* a, float* scores, int b0, int nb, int i0, int ni,
@@ -209,16 +234,10 @@ static cudaError_t launch_indexer_tc_rect(const lcsa_indexer_args* a, float* sco
   g.gps = (ni + kIxRows - 1) / kIxRows;
   g.q_pos0 = a->q_pos0; g.m = a->m;
   const int n_groups = nb * g.gps;
-  // Few groups (decode): split each group's entry range so that ~4 waves of CTAs cover the SMs.
   long long nv = (a->q_pos0 + i0 + ni - 1) / a->m;
   if (nv > a->Nc) nv = a->Nc;
   const int tiles = (int)((nv + kIxTileE - 1) / kIxTileE);
-  int splits = 1;
-  if (n_groups < 4 * 148) {
-    splits = (4 * 148 + n_groups - 1) / n_groups;
-    const int max_splits = tiles / 8 > 1 ? tiles / 8 : 1;   // keep >= 8 tiles per CTA
-    splits = splits < max_splits ? splits : max_splits;
-  }
+  const int splits = indexer_splits(n_groups, tiles);
   g.splits = splits;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIxSmem);
   if (e != cudaSuccess) return e;

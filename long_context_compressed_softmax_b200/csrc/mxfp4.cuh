@@ -115,8 +115,9 @@ __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const T* __restrict
 // Query preparation for the FP4 indexer: every (row, head) of q [.., 64, 128]
 // BF16 in the rectangle (sequences [b0, b0+nb), rows [i0, i0+ni)) is
 // quantised to MXFP4 (4 blocks) and staged as E4M3 relative to its largest
-// block exponent; the head weight absorbs the factor:
-//   q8 [nb*ni*64, 128] E4M3,  w8 [nb*ni*64] = w * 2^(Xref - 6).
+// block exponent; the head weight absorbs the factor and a 1/2 (the scoring
+// epilogue forms w relu(x) as (w/2) x + (w/2) |x|):
+//   q8 [nb*ni*64, 128] E4M3,  w8 [nb*ni*64] = w * 2^(Xref - 7).
 // One warp per (row, head); lane l holds dims [4l, 4l+4) (block l / 8).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) indexer_q8_kernel(const __nv_bfloat16* __restrict__ q,
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(256) indexer_q8_kernel(const __nv_bfloat16* __
   e4m3_table(X - Xref + 6, lo, hi);
   const uint2 e = e2m1x8_to_e4m3(word, lo, hi);     // codes 4-7 are zero
   reinterpret_cast<uint32_t*>(q8 + unit * 128)[lane] = e.x;
-  if (lane == 0) w8[unit] = w[src_row] * pow2f(Xref - 6);
+  if (lane == 0) w8[unit] = w[src_row] * pow2f(Xref - 7);
 }
 
 }  // namespace lcsa

@@ -67,6 +67,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait by polling without suspending, for a single thread on the
+// critical path (a suspended try_wait can resume well after the phase
+// completes).  Same limit and error report as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      report(LCSA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Bounded wait for threads off the critical path: sleeps between polls so
 // the waiting warps leave issue slots to the warps doing the work.
 __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity) {
