@@ -411,7 +411,7 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     # cpu baseline (oracle on a bounded sample) on rank 0 at N=1
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        t_sample, t_full, desc = oracle_sample(cfg, 16, seed=7)
+        t_sample, t_full, desc = oracle_sample(cfg, 256, seed=7)     # ~10 s of CPU work
         cpu = {"value": units / t_full, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
                "sample": desc + f"; {t_sample:.1f} s of CPU work"}
 
