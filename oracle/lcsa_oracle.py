@@ -37,6 +37,9 @@ Readings of points the pages leave open:
     exponent floor(log2 amax) - 2, E2M1 codes rounded to nearest even and
     saturated); the query is quantised per (row, head) and the scores use
     the exact dequantised values.
+  * grouped output projection: g groups of consecutive heads, each projected
+    to d_g, concatenated and projected to d; the intermediate is stored in
+    BF16 (the pages give neither g nor d_g).
 
 Parity pins: every function here is checked in tests/test_oracle_pins.py
 against closed forms, a library attention routine, brute force and values the
@@ -371,3 +374,41 @@ def hca_dense_attn(q, ckv, kv, q_pos0, kv_pos0, m, W, sink, R, base=10000.0,
         outs.append(o)
         lses.append(l)
     return np.stack(outs), np.stack(lses)
+
+
+# ----------------------------------------------------------------------------
+# Step 4: grouped output projection  ([p3] "第四步，grouped output projection" and
+# the sentence explaining it: with head dimension c = 512, projecting all head
+# outputs straight back to d would be costly, so the n_h heads are split into g
+# groups, each group is first projected to an intermediate width d_g, and the
+# concatenated groups are projected back to d; V4-Flash's hidden size is 4096)
+# ----------------------------------------------------------------------------
+def grouped_out_proj(o, w_group, w_out, round_mid=True):
+    """y = W_out . concat_g(W_group[g] . o_g) for every token.
+
+    o       [T, n_h, c]  attention outputs (heads of group g: g*n_h/g .. +n_h/g)
+    w_group [g, d_g, (n_h/g)*c]  per-group projection, rows = outputs
+    w_out   [d, g*d_g]           merge projection, rows = outputs
+    The intermediate group projections are rounded to BF16 when `round_mid`
+    (they are stored between the two projections in BF16).  FP64 otherwise.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    w_group = np.asarray(w_group, dtype=np.float64)
+    w_out = np.asarray(w_out, dtype=np.float64)
+    T, n_h, c = o.shape
+    g, d_g, kg = w_group.shape
+    assert n_h % g == 0 and kg == (n_h // g) * c and w_out.shape[1] == g * d_g
+    x = o.reshape(T, g, kg)
+    mid = np.stack([x[:, j, :] @ w_group[j].T for j in range(g)], axis=1).reshape(T, g * d_g)
+    if round_mid:
+        mid = _round_bf16(mid)
+    return mid @ w_out.T
+
+
+def _round_bf16(x):
+    """Nearest BF16 value (8 significant bits, exponent range of FP32; ties to
+    even) of each FP64 value: x / ulp(x) rounded half-to-even, times ulp(x)."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(np.where(x == 0, 1.0, x))          # |x| = f * 2^e, f in [0.5, 1)
+    ulp_exp = np.maximum(e - 8, -133)                    # 8 significant bits; BF16 subnormal spacing 2^-133
+    return np.ldexp(np.rint(np.ldexp(x, -ulp_exp)), ulp_exp)

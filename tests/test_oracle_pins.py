@@ -449,3 +449,53 @@ def test_hca_pipeline_strictly_causal():
     out2 = run(kv2, g2)
     np.testing.assert_array_equal(base[:30], out2[:30])
     assert not np.allclose(base[30], out2[30])
+
+
+# ---------------------------------------------------------------- grouped output projection
+def test_round_bf16_matches_fp32_rounding_and_ties():
+    # inputs that are FP32 values round in one step, so torch's FP32 -> BF16 is the reference
+    r = _rng(31)
+    x = (r.standard_normal(20000) * np.exp2(r.integers(-120, 120, 20000))).astype(np.float32).astype(np.float64)
+    ref = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(O._round_bf16(x), ref)
+    # exact midpoints go to the even neighbour; BF16 values stay put
+    np.testing.assert_array_equal(O._round_bf16(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(2 + 2.0 ** -7), 1.5])),
+                                  [1.0, 1 + 2.0 ** -6, -2.0, 1.5])
+
+
+def test_grouped_out_proj_equals_composed_dense_projection():
+    # without the BF16 intermediate the grouped projection is one linear map:
+    # W_out . blockdiag(W_group[0..g-1]) applied to the flattened head outputs
+    r = _rng(32)
+    T, n_h, c, g, d_g, d = 5, 8, 16, 4, 12, 20
+    o = r.standard_normal((T, n_h, c))
+    w1 = r.standard_normal((g, d_g, n_h // g * c))
+    w2 = r.standard_normal((d, g * d_g))
+    kg = n_h // g * c
+    bd = np.zeros((g * d_g, n_h * c))
+    for j in range(g):
+        bd[j * d_g:(j + 1) * d_g, j * kg:(j + 1) * kg] = w1[j]
+    np.testing.assert_allclose(O.grouped_out_proj(o, w1, w2, round_mid=False), o.reshape(T, -1) @ (w2 @ bd).T,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_out_proj_single_identity_group_is_plain_projection():
+    r = _rng(33)
+    T, n_h, c, d = 4, 2, 8, 6
+    o = torch.randn(T, n_h, c, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).double().numpy()
+    w2 = r.standard_normal((d, n_h * c))
+    y = O.grouped_out_proj(o, np.eye(n_h * c)[None], w2)       # BF16 inputs: the BF16 intermediate is exact
+    np.testing.assert_allclose(y, o.reshape(T, -1) @ w2.T, rtol=1e-13, atol=1e-13)
+
+
+def test_grouped_out_proj_group_permutation():
+    r = _rng(34)
+    T, n_h, c, g, d_g, d = 3, 8, 4, 4, 5, 7
+    o = r.standard_normal((T, n_h, c))
+    w1 = r.standard_normal((g, d_g, n_h // g * c))
+    w2 = r.standard_normal((d, g * d_g))
+    p = np.array([2, 0, 3, 1])
+    hp = np.concatenate([np.arange(j * (n_h // g), (j + 1) * (n_h // g)) for j in p])
+    cp = np.concatenate([np.arange(j * d_g, (j + 1) * d_g) for j in p])
+    np.testing.assert_allclose(O.grouped_out_proj(o[:, hp], w1[p], w2[:, cp], round_mid=False),
+                               O.grouped_out_proj(o, w1, w2, round_mid=False), rtol=1e-12, atol=1e-12)
