@@ -408,6 +408,11 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     if not args.no_e2e:
         e2e = run_e2e(args, cfg, runner, layers, units, world)
 
+    # grouped output projection of the stack's last output (not part of the step)
+    out_proj = None
+    if not args.no_out_proj:
+        out_proj = run_out_proj(lcsa, runner, cfg, dev, peaks)
+
     # cpu baseline (oracle on a bounded sample) on rank 0 at N=1
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -426,7 +431,42 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
                        "l2": "inputs larger than L2 (GBs per layer); no flush"},
             "layer_ms": layer_ms, "kernels": summary, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
+    if out_proj is not None:
+        line["grouped_out_proj"] = out_proj
     return line
+
+
+def run_out_proj(lcsa, runner, cfg, dev, peaks, g=8, d_g=1024, d=4096, reps=5):
+    """Grouped output projection of the attention output [B*T, 64, 512]: g
+    groups of 64/g heads projected to d_g, then merged to d (V4-Flash hidden
+    size); random BF16 weights.  Timed alone with CUDA events."""
+    o = runner.out.view(-1, cfg.H, cfg.D)
+    T = o.shape[0]
+    K = cfg.H // g * cfg.D
+    gg = gen._gen(4242, dev)
+    w1 = gen._randn((g, d_g, K), gg, dev, 1.0 / math.sqrt(K), torch.bfloat16)
+    w2 = gen._randn((d, g * d_g), gg, dev, 1.0 / math.sqrt(g * d_g), torch.bfloat16)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(lcsa.grouped_out_proj_workspace_bytes(T, g, d_g), dtype=torch.uint8, device=dev)
+    call = lambda: lcsa.grouped_out_proj(o, w1, w2, out=y, workspace=ws)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    flops = 2.0 * T * (g * d_g * K + d * g * d_g)
+    tf = flops / ms / 1e9
+    peak = peaks["bf16_tflops"]
+    del w1, w2, y, ws
+    return {"tokens": T, "g": g, "d_g": d_g, "d": d, "ms": round(ms, 3), "tflops": round(tf, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4), "peak_source": f"bf16_tflops of {peaks['source']}"},
+            "note": "two GEMMs per call (per-group projection, merge); BF16 intermediate; not in the timed step"}
 
 
 def run_e2e(args, cfg, runner, layers, units, world):
@@ -624,6 +664,7 @@ def main():
     ap.add_argument("--workload", default="stack_4layer_128k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-out-proj", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

@@ -249,6 +249,37 @@ lcsa_status lcsa_indexer_topk_mxfp4(const lcsa_indexer_mxfp4_args* a, void* work
                                    void* stream);
 
 /* ------------------------------------------------------------------------
+ * Grouped output projection ([p3] "第四步，grouped output projection" and its
+ * explanation: with head dimension 512, projecting all heads straight back
+ * to d would be costly, so the n_h heads are split into g groups, each group
+ * is projected to an intermediate width d_g, and the concatenated groups are
+ * projected back to d).  The pages give no g or d_g.
+ *
+ *   mid[t, j*d_g + i] = sum_k o[t, j*K + k] * w_group[j, i, k]    (K = n_h/g * c)
+ *   y[t, e]           = sum_i mid[t, i] * w_out[e, i]              (i < g*d_g)
+ *
+ *   o       [T, n_h, c] BF16 (attention outputs; group j = heads j*n_h/g ..)
+ *   w_group [g, d_g, K] BF16 (rows = outputs)
+ *   w_out   [d, g*d_g]  BF16 (rows = outputs)
+ *   y       [T, d]      BF16
+ * BF16 operands, FP32 accumulation; mid is rounded to BF16 in the caller's
+ * workspace (size from lcsa_grouped_out_proj_workspace).  Requirements: g
+ * divides n_h, K and g*d_g multiples of 64, d_g and d multiples of 8, all
+ * pointers 16-byte aligned (LCSA_ERR_INVALID_ARG otherwise).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* o;
+  const void* w_group;
+  const void* w_out;
+  void* y;
+  int T, n_h, c, g, d_g, d;
+} lcsa_out_proj_args;
+
+size_t lcsa_grouped_out_proj_workspace(const lcsa_out_proj_args* a);
+lcsa_status lcsa_grouped_out_proj(const lcsa_out_proj_args* a, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* ------------------------------------------------------------------------
  * Indexer + top-k without a caller workspace.  The pages have no counterpart
  * to this call: it exists for callers that cannot allocate device memory when
  * they call the library (an allocator or arena they do not own, a runtime

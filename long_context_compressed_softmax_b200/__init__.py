@@ -32,6 +32,7 @@ EXPORTED = [
     "lcsa_indexer_topk_workspace", "lcsa_indexer_topk", "lcsa_indexer_uses_tensor_cores",
     "lcsa_indexer_topk_noalloc",
     "lcsa_quantize_mxfp4", "lcsa_indexer_topk_mxfp4_workspace", "lcsa_indexer_topk_mxfp4",
+    "lcsa_grouped_out_proj_workspace", "lcsa_grouped_out_proj",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
 ]
 
@@ -58,6 +59,14 @@ class IndexerMxfp4Args(ctypes.Structure):
         ("B", ctypes.c_int), ("Tq", ctypes.c_int), ("Nc", ctypes.c_int), ("H_I", ctypes.c_int),
         ("D_I", ctypes.c_int), ("q_pos0", ctypes.c_int64), ("m", ctypes.c_int), ("k", ctypes.c_int),
         ("idx_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
+    ]
+
+
+class OutProjArgs(ctypes.Structure):
+    _fields_ = [
+        ("o", ctypes.c_void_p), ("w_group", ctypes.c_void_p), ("w_out", ctypes.c_void_p), ("y", ctypes.c_void_p),
+        ("T", ctypes.c_int), ("n_h", ctypes.c_int), ("c", ctypes.c_int), ("g", ctypes.c_int), ("d_g", ctypes.c_int),
+        ("d", ctypes.c_int),
     ]
 
 
@@ -92,6 +101,8 @@ _sig = {
     "lcsa_quantize_mxfp4": (_i, [_vp, _i64, _i, _i, _vp, _vp, _vp]),
     "lcsa_indexer_topk_mxfp4_workspace": (_sz, [ctypes.POINTER(IndexerMxfp4Args)]),
     "lcsa_indexer_topk_mxfp4": (_i, [ctypes.POINTER(IndexerMxfp4Args), _vp, _sz, _vp]),
+    "lcsa_grouped_out_proj_workspace": (_sz, [ctypes.POINTER(OutProjArgs)]),
+    "lcsa_grouped_out_proj": (_i, [ctypes.POINTER(OutProjArgs), _vp, _sz, _vp]),
     "lcsa_attn_workspace": (_sz, [ctypes.POINTER(AttnArgs), _i]),
     "lcsa_csa_sparse_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
@@ -304,6 +315,30 @@ def indexer_topk_mxfp4(q_idx, w, k_codes, k_scales, q_pos0, m, k, return_scores=
     st = _lib.lcsa_indexer_topk_mxfp4(ctypes.byref(a), _p(workspace), workspace.numel(), _stream(dev))
     _check(st, "indexer_topk_mxfp4")
     return (idx_out, scores) if return_scores else idx_out
+
+
+# ----------------------------------------------------------------- grouped output projection
+def grouped_out_proj_workspace_bytes(T, g, d_g):
+    a = OutProjArgs(None, None, None, None, T, g, 1, g, d_g, 8)
+    return int(_lib.lcsa_grouped_out_proj_workspace(ctypes.byref(a)))
+
+
+def grouped_out_proj(o, w_group, w_out, out=None, workspace=None):
+    """o [T, n_h, c] BF16, w_group [g, d_g, n_h/g*c] BF16, w_out [d, g*d_g] BF16
+    -> y [T, d] BF16 (per-group projection to d_g, merge projection to d)."""
+    _need_contig(o, w_group, w_out)
+    T, n_h, c = o.shape
+    g, d_g, _ = w_group.shape
+    d = w_out.shape[0]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=o.device)
+    a = OutProjArgs(_p(o), _p(w_group), _p(w_out), _p(out), T, n_h, c, g, d_g, d)
+    if workspace is None:
+        need = int(_lib.lcsa_grouped_out_proj_workspace(ctypes.byref(a)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=o.device)
+    st = _lib.lcsa_grouped_out_proj(ctypes.byref(a), _p(workspace), workspace.numel(), _stream(o.device))
+    _check(st, "grouped_out_proj")
+    return out
 
 
 # ----------------------------------------------------------------- attention

@@ -14,6 +14,7 @@
 #include "indexer_tc.cuh"
 #include "attn_tc.cuh"
 #include "indexer_fp4.cuh"
+#include "gemm_tc.cuh"
 
 using namespace lcsa;
 
@@ -378,6 +379,47 @@ lcsa_status lcsa_indexer_topk_mxfp4(const lcsa_indexer_mxfp4_args* a, void* work
         return launch_indexer_fp4_rect(a->k_codes, a->k_scales, a->B, a->Nc, a->q_pos0, a->m, q8, w8, sc, b0, nb,
                                        i0, ni, st);
       });
+}
+
+// ------------------------------------------------------------------ grouped output projection
+static lcsa_status check_out_proj(const lcsa_out_proj_args* a) {
+  if (!a) return LCSA_ERR_INVALID_ARG;
+  if (a->T < 0 || a->n_h <= 0 || a->c <= 0 || a->g <= 0 || a->d_g <= 0 || a->d <= 0) return LCSA_ERR_INVALID_ARG;
+  if (a->n_h % a->g != 0) return LCSA_ERR_INVALID_ARG;
+  const long long K = (long long)(a->n_h / a->g) * a->c;
+  if (K % 64 != 0 || ((long long)a->g * a->d_g) % 64 != 0 || a->d_g % 8 != 0 || a->d % 8 != 0)
+    return LCSA_ERR_INVALID_ARG;
+  if (K > (1 << 30) || (long long)a->g * a->d_g > (1 << 30)) return LCSA_ERR_INVALID_ARG;
+  if (a->T == 0) return LCSA_OK;
+  if (!a->o || !a->w_group || !a->w_out || !a->y) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(a->o) || !aligned16(a->w_group) || !aligned16(a->w_out) || !aligned16(a->y))
+    return LCSA_ERR_INVALID_ARG;
+  return LCSA_OK;
+}
+
+size_t lcsa_grouped_out_proj_workspace(const lcsa_out_proj_args* a) {
+  if (!a || a->T <= 0 || a->g <= 0 || a->d_g <= 0) return 0;
+  return align256((size_t)a->T * (size_t)a->g * (size_t)a->d_g * 2);
+}
+
+lcsa_status lcsa_grouped_out_proj(const lcsa_out_proj_args* a, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  lcsa_status s = check_out_proj(a);
+  if (s != LCSA_OK) return s;
+  if (a->T == 0) return LCSA_OK;
+  if (!workspace || workspace_bytes < lcsa_grouped_out_proj_workspace(a)) return LCSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int K = a->n_h / a->g * a->c;
+  const long long gd = (long long)a->g * a->d_g;
+  __nv_bfloat16* mid = (__nv_bfloat16*)workspace;
+  const int sms = sm_count();
+  cudaError_t e = launch_gemm_bf16(a->o, (long long)a->n_h * a->c, a->w_group, mid, gd, a->T, a->d_g, K, a->g, sms,
+                                   st);
+  if (e != cudaSuccess) return LCSA_ERR_CUDA;
+  e = launch_gemm_bf16(mid, gd, a->w_out, (__nv_bfloat16*)a->y, a->d, a->T, a->d, (int)gd, 1, sms, st);
+  return from_cuda(e);
 }
 
 int lcsa_attn_uses_tensor_cores(const lcsa_attn_args* a) { return a && attn_tc_supported(a) ? 1 : 0; }

@@ -46,7 +46,7 @@ def test_struct_layouts_match_header(lcsa, tmp_path):
     import subprocess
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "lcsa.h"', 'int main(void){']
     structs = (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs),
-               ("lcsa_indexer_mxfp4_args", lcsa.IndexerMxfp4Args))
+               ("lcsa_indexer_mxfp4_args", lcsa.IndexerMxfp4Args), ("lcsa_out_proj_args", lcsa.OutProjArgs))
     for cname, py in structs:
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in py._fields_:
@@ -133,6 +133,22 @@ def test_mxfp4_calls_check_arguments(lcsa):
     if not torch.cuda.is_available():
         ws = ctypes.c_void_p(0x10000)
         assert L.lcsa_indexer_topk_mxfp4(ctypes.byref(a), ws, 1 << 20, None) == 4   # no device: no CPU path
+
+
+def test_grouped_out_proj_checks_arguments(lcsa):
+    L = lcsa.lib
+    P = lambda **kw: lcsa.OutProjArgs(**{"o": 0x1000, "w_group": 0x2000, "w_out": 0x3000, "y": 0x4000, "T": 16,
+                                        "n_h": 64, "c": 512, "g": 8, "d_g": 1024, "d": 4096, **kw})
+    ws = ctypes.c_void_p(0x10000)
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P(g=7)), ws, 1 << 30, None) == 1        # g does not divide n_h
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P(c=36)), ws, 1 << 30, None) == 1       # K = 288, not a multiple of 64
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P(d=100)), ws, 1 << 30, None) == 1      # d not a multiple of 8
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P(y=0x4008)), ws, 1 << 30, None) == 1   # misaligned output
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P()), ws, 64, None) == 3                # workspace too small
+    assert L.lcsa_grouped_out_proj(ctypes.byref(P(T=0)), None, 0, None) == 0            # nothing to do
+    assert L.lcsa_grouped_out_proj_workspace(ctypes.byref(P())) == 16 * 8 * 1024 * 2
+    if not torch.cuda.is_available():
+        assert L.lcsa_grouped_out_proj(ctypes.byref(P()), ws, 1 << 30, None) == 4       # no device: no CPU path
 
 
 def test_empty_problems_are_noops(lcsa):

@@ -339,6 +339,29 @@ def test_indexer_mxfp4_small_workspace_chunks(lcsa):
     assert torch.equal(full, part)
 
 
+# ------------------------------------------------------------------ grouped output projection
+@pytest.mark.parametrize("T,n_h,c,g,d_g,d", [
+    (300, 64, 512, 8, 1024, 4096),     # layer shapes, ragged token count (3 m-tiles, tail of 44)
+    (129, 64, 512, 4, 512, 1024),      # other grouping
+    (64, 8, 64, 2, 224, 136),          # N not a multiple of the 256-column tile, small K
+    (17, 64, 512, 1, 1024, 512),       # one group
+])
+def test_grouped_out_proj_parity(lcsa, T, n_h, c, g, d_g, d):
+    gen_ = torch.Generator(device=DEV).manual_seed(71)
+    o = torch.randn(T, n_h, c, device=DEV, generator=gen_).to(torch.bfloat16)
+    K = n_h // g * c
+    w1 = (torch.randn(g, d_g, K, device=DEV, generator=gen_) / K ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(d, g * d_g, device=DEV, generator=gen_) / (g * d_g) ** 0.5).to(torch.bfloat16)
+    y = lcsa.grouped_out_proj(o, w1, w2)
+    ref = O.grouped_out_proj(np64(o), np64(w1), np64(w2))
+    got = np64(y)
+    scale = np.sqrt(np.mean(ref * ref))
+    err = np.abs(got - ref)
+    # BF16 output (relative 2^-9) plus FP32 accumulation and BF16 intermediate rounding differences
+    assert err.max() <= 2e-2 * scale + 8e-3 * np.abs(ref).max(), f"max err {err.max():.3e} (rms {scale:.3e})"
+    assert err.mean() <= 2e-3 * scale, f"mean err {err.mean():.3e}"
+
+
 # ------------------------------------------------------------------ attention
 def _attn_case(B, Tq, H, D, Nc, Tkv, dtype, seed, unit=True, sink=True):
     return gen.make_attn_inputs(B, Tq, H, D, Nc, Tkv, dtype, seed=seed, device=DEV, unit_scale=unit,
