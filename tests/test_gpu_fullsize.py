@@ -192,6 +192,26 @@ def test_csa_decode_1m_fp4_indexer_full(lcsa):
     assert lcsa.get_device_status() == 0
 
 
+def test_grouped_out_proj_full(lcsa):
+    """Grouped output projection over the stack's token count (2 x 131072
+    tokens, 64 heads x 512, g=8, d_g=1024, d=4096), sampled rows against the
+    oracle."""
+    T, n_h, c, g, d_g, d = 2 * 131072, 64, 512, 8, 1024, 4096
+    gg = torch.Generator(device=DEV).manual_seed(1501)
+    o = torch.randn(T, n_h, c, device=DEV, generator=gg).to(torch.bfloat16)
+    K = n_h // g * c
+    w1 = (torch.randn(g, d_g, K, device=DEV, generator=gg) / K ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(d, g * d_g, device=DEV, generator=gg) / (g * d_g) ** 0.5).to(torch.bfloat16)
+    y = lcsa.grouped_out_proj(o, w1, w2)
+    rows = sample_rows(T, 24, 1502)
+    ref = O.grouped_out_proj(np64(o[rows]), np64(w1), np64(w2))
+    got = np64(y[rows])
+    scale = np.sqrt(np.mean(ref * ref))
+    err = np.abs(got - ref)
+    assert err.max() <= 2e-2 * scale + 8e-3 * np.abs(ref).max() and err.mean() <= 2e-3 * scale
+    assert lcsa.get_device_status() == 0
+
+
 def test_stack_layers_full(lcsa):
     cfg = get_config("stack_4layer_128k")
     _run_csa_layer(lcsa, cfg, seed=1301, n_rows=12)
