@@ -141,7 +141,7 @@ class Layer:
         self.kind = kind
         m = cfg.m if kind == "csa" else cfg.m_hca
         self.m = m
-        self.Nc = T // m
+        self.Nc = T // m if kind != "swa" else 0    # swa: sliding window only, no compressed entries
         g = gen._gen(seed, dev)
         self.kv = gen._randn((B, T, D), g, dev, 1.0 / math.sqrt(D), torch.bfloat16)
         self.gate = gen._randn((B, T, D), g, dev, 1.0, torch.bfloat16)
@@ -154,7 +154,8 @@ class Layer:
             self.k_idx = gen._randn((B, self.Nc, cfg.D_I), g, dev, 1.0 / math.sqrt(cfg.D_I), torch.bfloat16)
 
     def inputs(self):
-        names = ["kv", "gate", "q"] + (["q_idx", "w", "k_idx"] if self.kind == "csa" else [])
+        names = (["kv", "q"] if self.kind == "swa" else ["kv", "gate", "q"]) + (
+            ["q_idx", "w", "k_idx"] if self.kind == "csa" else [])
         return {n: getattr(self, n) for n in names}
 
 
@@ -199,9 +200,13 @@ class StackRunner:
                                                                    workspace=self.ws, idx_out=self.idx))
             self._call(li, "csa_sparse_attn", lambda: lc.csa_sparse_attn(
                 L.q, L.ckv, self.idx, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
-        else:
+        elif L.kind == "hca":
             self._call(li, "hca_compress", lambda: lc.hca_compress(L.kv, L.gate, L.m, out=L.ckv))
             self._call(li, "hca_dense_attn", lambda: lc.hca_dense_attn(
+                L.q, L.ckv, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
+        else:
+            # pure sliding-window layer: the core attention with an empty entry cache (window + sink)
+            self._call(li, "swa_attn", lambda: lc.hca_dense_attn(
                 L.q, L.ckv, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
 
     def step(self):
@@ -268,7 +273,10 @@ def oracle_sample(cfg, n_rows, seed):
         q = (torch.randn(len(rows), H, D, generator=g) / math.sqrt(D)).to(torch.bfloat16).double().numpy()
         sink = torch.randn(H, generator=g).double().numpy()
         t0 = time.perf_counter()
-        ckv = (O.csa_compress(kv, gate, m) if kind == "csa" else O.hca_compress(kv, gate, m))
+        if kind == "swa":                   # sliding window only: no compressed entries
+            ckv = np.zeros((0, D))
+        else:
+            ckv = (O.csa_compress(kv, gate, m) if kind == "csa" else O.hca_compress(kv, gate, m))
         t_comp = time.perf_counter() - t0
         t_rows = 0.0
         if kind == "csa":
@@ -362,6 +370,7 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     f_csa = cfg.B * attn_flops(cfg.T, cfg.m, Nc4, cfg.W, cfg.k)
     f_hca = cfg.B * attn_flops(cfg.T, cfg.m_hca, Nc128, cfg.W)
     f_idx = cfg.B * indexer_flops(cfg.T, cfg.m, Nc4)
+    f_swa = cfg.B * attn_flops(cfg.T, cfg.m_hca, 0, cfg.W)
     kern = {}
     for (li, name), v in sorted(per_call.items()):
         avg = statistics.mean(v)
@@ -378,6 +387,8 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
             e["tflops"] = round(f_hca / avg / 1e9, 1)
         elif name == "indexer_topk":
             e["tflops"] = round(f_idx / avg / 1e9, 1)
+        elif name == "swa_attn":
+            e["tflops"] = round(f_swa / avg / 1e9, 1)
         elif name.endswith("compress"):
             m = cfg.m if name.startswith("csa") else cfg.m_hca
             byts = cfg.B * (2 * cfg.T * cfg.D * 2 + (cfg.T // m) * cfg.D * 2)
@@ -390,7 +401,8 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
 
     # roofline of the dominant kernel (largest share of the step)
     dom = max(summary, key=lambda n: summary[n]["ms_avg"] * summary[n]["calls_per_step"])
-    dom_flops = {"csa_sparse_attn": f_csa, "hca_dense_attn": f_hca, "indexer_topk": f_idx}.get(dom)
+    dom_flops = {"csa_sparse_attn": f_csa, "hca_dense_attn": f_hca, "indexer_topk": f_idx,
+                 "swa_attn": f_swa}.get(dom)
     avg_ms = summary[dom]["ms_avg"]
     peak = peaks["bf16_tflops_sustained"]
     achieved = dom_flops / avg_ms / 1e9 if dom_flops else None
@@ -474,7 +486,7 @@ def run_e2e(args, cfg, runner, layers, units, world):
     memory every step and the final output read back."""
     try:
         hosts = {}
-        for kind in ("csa", "hca"):
+        for kind in dict.fromkeys(L.kind for L in layers):     # one set of host inputs per layer kind
             L = next(L for L in layers if L.kind == kind)
             hosts[kind] = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t, non_blocking=False)
                            for n, t in L.inputs().items()}

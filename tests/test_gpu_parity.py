@@ -372,6 +372,19 @@ def _sink(x):
     return None if x["sink"] is None else np64(x["sink"])
 
 
+@pytest.mark.parametrize("Tq,q_pos0,W", [(300, 0, 128), (77, 5000, 128), (40, 1000, 100)])
+def test_sliding_window_only_layer(lcsa, Tq, q_pos0, W):
+    """A pure sliding-window layer (the first two V4-Flash layers): the core
+    attention with an empty entry cache, i.e. window + sink only."""
+    B, H, D, R = 2, 64, 512, 64
+    Tkv = q_pos0 + Tq
+    x = _attn_case(B, Tq, H, D, 0, Tkv, "bf16", seed=55)
+    assert x["ckv"].shape == (B, 0, D)
+    out = lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q_pos0, 0, 128, W, R)
+    ref, _ = O.hca_dense_attn(np64(x["q"]), np64(x["ckv"]), np64(x["kv"]), q_pos0, 0, 128, W, _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+
+
 @pytest.mark.parametrize("dtype,H,D,R,m,W,k,Tq,Nc,q_pos0,unit", [
     ("fp32", 4, 64, 32, 4, 64, 64, 200, 256, 824, True),       # tiny layer: rows near the end of T=1024
     ("fp32", 4, 64, 32, 4, 64, 64, 64, 256, 0, True),          # first rows: no entries / short window

@@ -61,6 +61,13 @@ CONFIGS = {
     # Alternating four-layer stack CSA->HCA->CSA->HCA, B=2, T=131072.
     "stack_4layer_128k": WorkloadConfig(name="stack_4layer_128k", dtype="bf16", B=2, T=131072, seed=5,
                                         layers=("csa", "hca", "csa", "hca")),
+    # Layer mixes of the two model sizes (first two layers differ, the rest
+    # alternate CSA / HCA): V4-Flash opens with two pure sliding-window layers,
+    # V4-Pro with two HCA layers.  Six layers, B=2, T=131072.
+    "stack_flash_6layer_128k": WorkloadConfig(name="stack_flash_6layer_128k", dtype="bf16", B=2, T=131072, seed=9,
+                                              layers=("swa", "swa", "csa", "hca", "csa", "hca")),
+    "stack_pro_6layer_128k": WorkloadConfig(name="stack_pro_6layer_128k", dtype="bf16", B=2, T=131072, seed=10,
+                                            layers=("hca", "hca", "csa", "hca", "csa", "hca")),
 }
 
 
