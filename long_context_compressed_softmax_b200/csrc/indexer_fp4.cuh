@@ -15,13 +15,15 @@
 //              query rows (E4M3 queries prepared by indexer_q8_kernel), K = 128
 //   accumulators  512 TMEM columns split into 2-8 slots (64 x query rows
 //              columns each), so the MMA runs up to 8 tiles ahead of the epilogue
-//   epilogue   8 warps: ReLU, head weights (with the query factors folded
-//              in) and the entry factor 2^(Xref - 6), one score per lane;
+//   epilogue   8 warps: w relu(x) formed as (w/2) x + (w/2) |x| on the FMA
+//              pipe (the prepared head weights carry the query factors and
+//              the 1/2), times the entry factor 2^(Xref - 6), one score per lane;
 //              with 3-4 query rows each warp scores 2 rows of every tile,
 //              with 1-2 rows the two warps of a lane quarter take alternate
 //              tiles (one accumulator each).
 // Warp roles (576 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
-// 2-9 epilogue, 10-17 dequantisers.  Every wait is bounded (tc::mbar_wait);
+// 2-9 epilogue, 10-17 dequantisers.  Every wait is bounded (tc::mbar_wait, or
+// the non-suspending tc::mbar_wait_spin for the single-thread MMA issuer);
 // on expiry the CTA stops, records LCSA_DEV_TIMEOUT, drains its in-flight
 // copies and frees TMEM.
 #pragma once
