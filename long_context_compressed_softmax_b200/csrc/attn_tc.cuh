@@ -857,11 +857,22 @@ static AtPlan attn_tc_plan(const lcsa_attn_args* a, int sparse) {
     max_c = nv < a->Nc ? nv : a->Nc;
   }
   const int max_tiles = (int)((max_c + kAtKT - 1) / kAtKT + (a->W + kAtKT - 1) / kAtKT + 1);
+  // Few rows (decode): split each row's key range.  The split count s (>= 4
+  // tiles per split) minimises, in units of one 64-key tile (~1.4 us), the
+  // persistent CTAs' rounds x (tiles per item + ~1 tile of per-item cost)
+  // plus the partial-output traffic of the combine (s x rows x 256 KB written
+  // and read at ~6 TB/s).
   int splits = 1;
-  if (rows < 2 * 148) {
-    splits = (int)((2 * 148 + rows - 1) / rows);
-    const int cap = max_tiles / 4 > 1 ? max_tiles / 4 : 1;        // >= 4 tiles per split
-    splits = splits < cap ? splits : cap;
+  const int sms = sm_count();
+  if (rows < 2 * sms) {
+    const int cap = max_tiles / 4 > 1 ? max_tiles / 4 : 1;
+    double best = -1.0;
+    for (int s = 1; s <= cap; ++s) {
+      const long long rounds = (rows * s + sms - 1) / sms;
+      const double cost = (double)rounds * (double)((max_tiles + s - 1) / s + 1) +
+                          (s > 1 ? (double)s * (double)rows * 262144.0 / 6.0e6 / 1.4 : 0.0);
+      if (best < 0.0 || cost < best) { best = cost; splits = s; }
+    }
   }
   // An item stages at most kAtMaxIdx selected entries: larger k needs more key-range splits.
   if (sparse && a->k > kAtMaxIdx) {

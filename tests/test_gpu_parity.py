@@ -426,15 +426,31 @@ def test_hca_dense_attn_parity(lcsa, dtype, H, D, R, m, W, Tq, Nc, q_pos0, unit,
     np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
 
 
-def test_hca_key_range_splits_with_empty_items(lcsa):
-    """290 query rows (< 2 x 148: key ranges split in two) at positions 0..289
-    with m = 1: the first rows have a single key tile, so their second split
-    has no keys and the persistent kernel's empty-item path writes them (zero
-    partial output, -inf partial max) before the combine."""
+def test_hca_causal_rows_from_position_zero(lcsa):
+    """290 query rows at positions 0..289 with m = 1: every row a different
+    number of visible entries, from none to 289."""
     B, H, D, R, m, W, Tq, Nc, q0 = 1, 64, 512, 64, 1, 128, 290, 290, 0
     x = _attn_case(B, Tq, H, D, Nc, q0 + Tq, "bf16", seed=63)
     out, lse = lcsa.hca_dense_attn(x["q"], x["ckv"], x["kv"], x["sink"], q0, 0, m, W, R, return_lse=True)
     ref, ref_lse = O.hca_dense_attn(np64(x["q"]), np64(x["ckv"]), np64(x["kv"]), q0, 0, m, W, _sink(x), R)
+    assert_attn_close(np64(out).reshape(ref.shape), ref)
+    np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
+    assert lcsa.get_device_status() == 0
+
+
+def test_csa_key_range_splits_with_empty_items(lcsa):
+    """40 early rows (positions 0..39, at most 9 visible entries) with k = 2048:
+    the key range of k + window tiles is split three ways (few rows, long
+    ranges), so most split items hold no keys and the persistent kernel's
+    empty-item path writes them (zero partial output, -inf partial max) before
+    the combine."""
+    B, H, D, R, m, W, k, Tq, Nc, q0 = 1, 64, 512, 64, 4, 128, 2048, 40, 700, 0
+    x = _attn_case(B, Tq, H, D, Nc, q0 + Tq, "bf16", seed=64)
+    nv = [O.n_visible(q0 + i, m, Nc) for i in range(Tq)]
+    idx = gen.make_topk_idx(B, Tq, k, nv, seed=65, device=DEV)
+    out, lse = lcsa.csa_sparse_attn(x["q"], x["ckv"], idx, x["kv"], x["sink"], q0, 0, m, W, R, return_lse=True)
+    ref, ref_lse = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), q0, 0, m, W,
+                                     _sink(x), R)
     assert_attn_close(np64(out).reshape(ref.shape), ref)
     np.testing.assert_allclose(np64(lse).reshape(ref_lse.shape), ref_lse, atol=2e-3)
     assert lcsa.get_device_status() == 0
