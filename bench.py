@@ -5,12 +5,18 @@ stack CSA -> HCA -> CSA -> HCA, prefill of B=2 sequences of T=131072 tokens,
 64 heads x 512 dims (last 64 rotary), indexer 64 x 128, m=4 / m'=128,
 top-k 2048, window 128, per-head sink, independent seeded inputs per layer.
 CSA layer = csa_compress -> indexer_topk -> csa_sparse_attn; HCA layer =
-hca_compress -> hca_dense_attn.  Metric: prefill tokens/s through the stack.
-A second object reports the CSA decode workload at 1M context (64 sequences,
-one query each, queries/s).
+hca_compress -> hca_dense_attn; a pure sliding-window layer (the first layers
+of V4-Flash) = hca_dense_attn with no entries.  Metric: prefill tokens/s through
+the stack.  Further objects on the same line: the CSA decode workload at 1M
+context (64 sequences, one query each, queries/s; BF16 and MXFP4 indexer keys),
+the end-to-end run from host memory, the grouped output projection of the
+stack's output, and the oracle's CPU baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lcsa|reference]
-                    [--workload stack_4layer_128k|csa_prefill_32k|hca_prefill_128k|csa_decode_1m]
+                    [--workload stack_4layer_128k|csa_prefill_32k|hca_prefill_128k|csa_decode_1m|
+                                stack_flash_6layer_128k|stack_pro_6layer_128k|csa_prefill_8k|
+                                hca_prefill_16k|csa_decode_8seq]
+                    [--no-e2e] [--no-decode] [--no-cpu-baseline] [--no-out-proj]
 
 N > 1 runs under torchrun, one rank per GPU; every rank runs the same
 per-GPU workload on its own seeds (weak scaling, no data-path collective) and
