@@ -39,7 +39,9 @@ Readings of points the pages leave open:
     the exact dequantised values.
   * grouped output projection: g groups of consecutive heads, each projected
     to d_g, concatenated and projected to d; the intermediate is stored in
-    BF16 (the pages give neither g nor d_g).
+    BF16 (the pages give neither g nor d_g);
+  * FP8 entry cache: E4M3 for the non-rotary dims with one power-of-two scale
+    per entry (largest magnitude mapped to at most 448), rotary dims in BF16.
 
 Parity pins: every function here is checked in tests/test_oracle_pins.py
 against closed forms, a library attention routine, brute force and values the
@@ -412,3 +414,68 @@ def _round_bf16(x):
     _, e = np.frexp(np.where(x == 0, 1.0, x))          # |x| = f * 2^e, f in [0.5, 1)
     ulp_exp = np.maximum(e - 8, -133)                    # 8 significant bits; BF16 subnormal spacing 2^-133
     return np.ldexp(np.rint(np.ldexp(x, -ulp_exp)), ulp_exp)
+
+
+# ----------------------------------------------------------------------------
+# FP8 entry cache  ([p4] "KV Cache优化细节": mixed storage, the rotary dims in
+# BF16 and the rest in FP8)
+#
+# Reading (the pages give no FP8 variant or scale): FP8 E4M3 (bias 7, no
+# infinities, largest finite 448, subnormals m * 2^-9) for the first D - R dims
+# of every entry, with one power-of-two scale per entry 2^X, X the smallest
+# integer with max|x| / 2^X <= 448 (stored as the byte X + 127; an all-zero
+# entry takes X = -127), values rounded to nearest even and saturated at 448;
+# the last R (rotary) dims stay BF16.  A power-of-two scale keeps E4M3 * 2^X
+# exact in BF16, so the cache can be expanded for BF16 tensor cores losslessly.
+# ----------------------------------------------------------------------------
+def e4m3_value(code):
+    """Value of an 8-bit E4M3 code from its fields (sign bit 7, exponent bits
+    6-3 with bias 7, mantissa bits 2-0); exponent 0 is subnormal; 0x7F and
+    0xFF are NaN."""
+    code = int(code)
+    sgn = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 0xF, code & 7
+    if e == 15 and m == 7:
+        return float("nan")
+    mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return sgn * mag
+
+
+E4M3_POS = np.array([e4m3_value(c) for c in range(0x7F)])     # codes 0x00..0x7E, increasing
+
+
+def e4m3_codes(y):
+    """E4M3 codes of the values nearest to y (array): round to nearest, ties to
+    the code with an even mantissa (code bit 0), magnitudes above 448 saturate
+    to 448; bit 7 is the sign of y."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.minimum(np.abs(y), 448.0)
+    hi = np.clip(np.searchsorted(E4M3_POS, a, side="left"), 0, len(E4M3_POS) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - E4M3_POS[lo], E4M3_POS[hi] - a
+    c = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    c = np.where(a == E4M3_POS[hi], hi, c)
+    return (c | np.where(y < 0, 0x80, 0)).astype(np.uint8)
+
+
+def quantize_entries_fp8(ckv, R):
+    """Entries [..., D] -> (codes uint8 [..., D-R] E4M3, scales uint8 [...]
+    (X + 127), rope BF16 values [..., R] as FP64)."""
+    x = np.asarray(ckv, dtype=np.float64)
+    D = x.shape[-1]
+    body, rope = x[..., :D - R], x[..., D - R:]
+    amax = np.abs(body).max(axis=-1)
+    # smallest X with amax <= 448 * 2^X: with amax = f 2^e (f in [0.5, 1)) and
+    # 448 = 0.875 * 2^9, X = e - 9 if f <= 0.875 else e - 8 (exact comparisons)
+    f, e = np.frexp(np.where(amax > 0, amax, 1.0))
+    X = np.where(f <= 0.875, e - 9, e - 8)
+    X = np.where(amax > 0, np.clip(X, -127, 127), -127).astype(np.int64)
+    codes = e4m3_codes(np.ldexp(body, -X[..., None]))
+    return codes, (X + 127).astype(np.uint8), _round_bf16(rope)
+
+
+def dequantize_entries_fp8(codes, scales, rope):
+    """Exact FP64 entries from the FP8 cache: E4M3 value * 2^X, rotary dims as stored."""
+    vals = np.vectorize(e4m3_value, otypes=[np.float64])(np.asarray(codes))
+    X = np.asarray(scales, dtype=np.float64) - 127.0
+    return np.concatenate([vals * np.exp2(X)[..., None], np.asarray(rope, dtype=np.float64)], axis=-1)

@@ -499,3 +499,68 @@ def test_grouped_out_proj_group_permutation():
     cp = np.concatenate([np.arange(j * d_g, (j + 1) * d_g) for j in p])
     np.testing.assert_allclose(O.grouped_out_proj(o[:, hp], w1[p], w2[:, cp], round_mid=False),
                                O.grouped_out_proj(o, w1, w2, round_mid=False), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 entry cache
+def test_e4m3_codes_bruteforce_over_all_codes():
+    # nearest of the 254 finite codes of the same sign, ties to an even mantissa,
+    # saturation at 448; values on a fine grid around every binade
+    cands = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    vals = {c: O.e4m3_value(c) for c in cands}
+    ys = [s * m * 2.0 ** k for s in (1, -1) for k in range(-12, 10) for m in np.arange(1, 2, 1 / 64)]
+    ys += [0.0, 448.0, 460.0, 1e6, -1e6]
+    got = O.e4m3_codes(np.array(ys))
+    for y, c in zip(ys, got):
+        same = [cc for cc in cands if (cc >> 7) == (1 if y < 0 else 0)]
+        a = min(abs(y), 448.0)
+        best = min(abs(a - abs(vals[cc])) for cc in same)
+        near = [cc for cc in same if abs(a - abs(vals[cc])) == best]
+        want = near[0] if len(near) == 1 else [cc for cc in near if cc % 2 == 0][0]
+        assert int(c) == want, y
+
+
+def test_e4m3_values_closed_forms():
+    assert O.e4m3_value(0x7E) == 448.0 and O.e4m3_value(0x01) == 2.0 ** -9 and O.e4m3_value(0x38) == 1.0
+    assert O.e4m3_value(0xB8) == -1.0 and np.isnan(O.e4m3_value(0x7F)) and np.isnan(O.e4m3_value(0xFF))
+    assert (np.diff(O.E4M3_POS) > 0).all()
+
+
+def test_fp8_entry_scale_rule_and_rope_passthrough():
+    r = _rng(41)
+    D, R = 512, 64
+    x = r.standard_normal((6, D)) * np.exp2(r.integers(-12, 12, (6, 1)))
+    x[1, :D - R] = 0.0                          # all-zero body
+    x[2, 7] = 448.0 * 2.0 ** -3                 # amax exactly 448 * 2^-3 -> X = -3
+    x[2, :D - R] = np.clip(x[2, :D - R], -56.0, 56.0)
+    codes, sc, rope = O.quantize_entries_fp8(x, R)
+    X = sc.astype(np.int64) - 127
+    amax = np.abs(x[:, :D - R]).max(axis=1)
+    for i in range(6):
+        if amax[i] == 0:
+            assert X[i] == -127 and not codes[i].any()
+        else:
+            assert amax[i] <= 448.0 * 2.0 ** X[i] and amax[i] > 448.0 * 2.0 ** (X[i] - 1)
+    assert X[2] == -3
+    np.testing.assert_array_equal(rope, O._round_bf16(x[:, D - R:]))
+    d = O.dequantize_entries_fp8(codes, sc, rope)
+    np.testing.assert_array_equal(d[:, D - R:], rope)
+    # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 on normals, absolute <= 2^-10 * 2^X below
+    err = np.abs(d[:, :D - R] - x[:, :D - R])
+    bound = np.maximum(np.abs(x[:, :D - R]) * 2.0 ** -4, 2.0 ** -10 * np.exp2(X)[:, None])
+    assert (err <= bound + 1e-300).all()
+
+
+def test_fp8_entry_roundtrip_of_representable_entries():
+    # entries already on the scaled E4M3 grid with the saturating code present come back unchanged
+    r = _rng(42)
+    codes = r.integers(0, 0x7F, (4, 448)).astype(np.uint8)
+    codes = np.where((codes & 0x7F) == 0x7F, 0x7E, codes).astype(np.uint8)
+    codes[:, 0] = 0x7E                          # every entry holds +448 * 2^X
+    codes |= (r.integers(0, 2, (4, 448)) << 7).astype(np.uint8)
+    codes[:, 0] &= 0x7F
+    sc = r.integers(100, 130, 4).astype(np.uint8)
+    rope = O._round_bf16(r.standard_normal((4, 64)))
+    x = O.dequantize_entries_fp8(codes, sc, rope)
+    c2, s2, r2 = O.quantize_entries_fp8(x, 64)
+    np.testing.assert_array_equal(s2, sc)
+    np.testing.assert_array_equal(O.dequantize_entries_fp8(c2, s2, r2), x)
