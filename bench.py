@@ -45,6 +45,10 @@ from workloads import gen  # noqa: E402
 from workloads.scaling import max_over_ranks, rank_seed, weak_scaling_throughput  # noqa: E402
 
 METRIC = "CSA/HCA prefill tokens/s and 1M-ctx decode queries/s; % of roofline"
+# Nominal B200 figures (dense BF16 tensor peak, HBM3e bandwidth), reported next
+# to the fractions of the measured peaks.
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 7700.0
 
 # DRAM traffic per launch of the dominant kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
@@ -317,6 +321,20 @@ def _blas_threads():
     return os.cpu_count()
 
 
+def config_obj(cfg, world):
+    """The line's `config` (identical for the library arm and the reference arm)."""
+    c = {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.T, "parallelism": f"dp{world}"}
+    if cfg.decode:
+        c.update({"query_position": cfg.T, "entries": cfg.T // cfg.m, "heads": cfg.H, "head_dim": cfg.D,
+                  "indexer": f"{cfg.H_I}x{cfg.D_I}", "topk": cfg.k, "window": cfg.W})
+        return c
+    layers = list(cfg.layers) if cfg.layers else ["csa" if cfg.name.startswith("csa") else "hca"]
+    c.update({"layers": layers, "heads": cfg.H, "head_dim": cfg.D, "rope_dims": cfg.R,
+              "indexer": f"{cfg.H_I}x{cfg.D_I}", "m": cfg.m, "m_hca": cfg.m_hca, "topk": cfg.k, "window": cfg.W,
+              "out_dtype": "bf16", "l2": "inputs larger than L2 (GBs per layer); no flush"})
+    return c
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, cfg, world, rank):
     if rank != 0:
@@ -333,12 +351,16 @@ def run_reference(args, cfg, world, rank):
     full = statistics.mean(fulls)
     value = units / full
     unit = "queries/s" if cfg.decode else "tokens/s"
+    # A step is one bounded sample (measured wall time); the throughput is the
+    # sample's per-row cost extrapolated to the whole workload.
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * full,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1)-scaled, BF16-rounded)",
-            "config": {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.T,
-                       "parallelism": f"dp{world}"},
+            "config": config_obj(cfg, world),
+            "extrapolated": {"ms_per_full_step": 1e3 * full,
+                             "how": "value = workload units / (sample time extrapolated by per-row cost); "
+                                    "ms_per_step is the measured time of one sample"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": _blas_threads(), "kind": "oracle",
                              "sample": desc + f"; {statistics.mean(times):.1f} s of CPU work per step"},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -416,6 +438,8 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     traffic = tr["bytes_per_launch"] if tr and tr.get("src") == _src_hash(tr["file"]) else None
     roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
+                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                "frac_vs_spec_peak": round(achieved / SPEC_BF16_TFLOPS, 4),
                 "peak_source": f"bf16_tflops_sustained of {peaks['source']}",
                 "flops_per_launch": dom_flops,
                 "note": "launch = one library call (rotary pre-pass + attention kernel); "
@@ -442,11 +466,7 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)-scaled BF16 inputs, independent per layer and rank)",
-            "config": {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.T,
-                       "parallelism": f"dp{world}", "layers": list(cfg.layers), "heads": cfg.H, "head_dim": cfg.D,
-                       "rope_dims": cfg.R, "indexer": f"{cfg.H_I}x{cfg.D_I}", "m": cfg.m, "m_hca": cfg.m_hca,
-                       "topk": cfg.k, "window": cfg.W, "out_dtype": "bf16",
-                       "l2": "inputs larger than L2 (GBs per layer); no flush"},
+            "config": config_obj(cfg, world),
             "layer_ms": layer_ms, "kernels": summary, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
     if out_proj is not None:
@@ -590,6 +610,7 @@ def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
            "ms_per_step": ms, "indexer_topk_ms": ix_ms, "csa_sparse_attn_ms": at_ms,
            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                        "frac_vs_spec_peak": round(gbs / SPEC_HBM_GBS, 4),
                         "bytes_per_step": byts, "peak_source": f"hbm_gbs of {peaks['source']}",
                         "note": "whole decode step (indexer keys + gathered rows + window + q/out)"},
            "gpu_launches": int(launches), "clocks": clocks,
@@ -669,8 +690,20 @@ def run_single(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     kind = "csa" if cfg.name.startswith("csa") else "hca"
     cfg1 = cfg.__class__(**{**cfg.__dict__, "layers": (kind,)})
     line = run_stack(args, cfg1, lcsa, dev, world, rank, bus_id, peaks)
-    line["config"]["workload"] = cfg.name
+    line["config"] = config_obj(cfg, world)
     return line
+
+
+def launch_ranks(n):
+    """`--gpus N` without a launcher: start N ranks (one per GPU) under
+    torch.distributed.run on this node and return its exit status."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -690,6 +723,12 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(launch_ranks(args.gpus))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU "
+              f"(torchrun --nproc-per-node {args.gpus}) or pass --gpus {world}", file=sys.stderr)
+        sys.exit(2)
     cfg = get_config(args.workload)
 
     if args.impl == "reference":
@@ -714,8 +753,7 @@ def main():
             line = run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world)
             line = {"metric": METRIC, **line, "n_gpus": world, "steps": args.steps * 4, "warmup": args.warmup,
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                    "data": "synthetic", "config": {"workload": cfg.name, "global_batch": cfg.B * world,
-                                                    "seq_len": cfg.T, "parallelism": f"dp{world}"}}
+                    "data": "synthetic", "config": config_obj(cfg, world)}
         elif cfg.layers:
             line = run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks)
             if not args.no_decode:

@@ -291,13 +291,22 @@ lcsa_status lcsa_grouped_out_proj(const lcsa_out_proj_args* a, void* workspace, 
  * held by every GPU that loads the library until the process exits; large
  * problems are processed in row chunks that fit it.  Nothing is allocated and
  * nothing needs clearing (each chunk writes the scratch it reads).
- *   - Returns LCSA_ERR_WORKSPACE when a single score row does not fit, i.e.
- *     when Nc * 4 bytes (rounded up to 256) + 256 exceeds 32 MiB
- *     (Nc > 8,388,544).
- *   - The first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before capturing any stream into a CUDA graph.
- *   - All calls on a device share the one array: calls that overlap on the
+ *   - Argument errors are those of lcsa_indexer_topk, checked first.
+ *   - Returns LCSA_ERR_WORKSPACE when what one query row needs does not fit
+ *     32 MiB: its Nc FP32 scores (rounded up to 256 bytes), its 256-byte
+ *     count and, for rows longer than 32768 columns that take the two-phase
+ *     top-k, 3 x (ceil(Nc/32768) x k x 4 bytes, rounded up to 256) + 256.
+ *     Nc > 8,388,544 never fits; with a two-phase row the limit is lower
+ *     (e.g. about 8.34 M columns at k = 64).
+ *   - The scratch array's device address belongs to the current context: it
+ *     differs between contexts and changes after cudaDeviceReset.  Every call
+ *     made while its stream is not being captured looks the address up in the
+ *     current context (cudaGetSymbolAddress) and remembers it for that
+ *     context; a call made during stream capture uses the remembered address
+ *     and returns LCSA_ERR_CUDA when the current context has none.  So make
+ *     one call outside capture in each context, and again after a reset,
+ *     before capturing a call into a CUDA graph.
+ *   - All calls in a context share the one array: calls that overlap on the
  *     GPU (different streams, or concurrent host threads without ordering)
  *     race on it.  Order them on one stream.
  * ------------------------------------------------------------------------ */

@@ -201,6 +201,15 @@ lcsa_status indexer_by_chunks(int B, int Tq, int Nc, int k, long long q_pos0, in
 
 }  // namespace
 
+// Shared with noalloc.cu (same library, not exported): the argument checks of
+// lcsa_indexer_topk, and the workspace that one query row needs.
+__attribute__((visibility("hidden"))) lcsa_status lcsa_internal_check_indexer(const lcsa_indexer_args* a) {
+  return check_indexer(a);
+}
+__attribute__((visibility("hidden"))) size_t lcsa_internal_indexer_one_row_bytes(const lcsa_indexer_args* a) {
+  return indexer_ws_need(1, a->Nc, a->k, 0);
+}
+
 extern "C" {
 
 const char* lcsa_version(void) { return "lcsa 0.1 (sm_100a)"; }

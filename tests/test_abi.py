@@ -172,3 +172,27 @@ def test_workspace_queries(lcsa):
     q = torch.empty((1, 4096, 64, 128), dtype=torch.bfloat16)
     k = torch.empty((1, 1024, 128), dtype=torch.bfloat16)
     assert lcsa.indexer_workspace_bytes(q, k, 2048) >= 4096 * 1024 * 4
+
+
+def test_noalloc_validates_like_the_workspace_call(lcsa):
+    """lcsa_indexer_topk_noalloc runs lcsa_indexer_topk's argument checks first,
+    so a bad argument gives the same status through both entry points, before
+    anything touches a device."""
+    L = lcsa.lib
+    ptrs = dict(q_idx=0x1000, w=0x2000, k_idx=0x3000, idx_out=0x4000)
+    base = dict(B=1, Tq=4, Nc=8, H_I=64, D_I=128, dtype=lcsa.LCSA_BF16, q_pos0=0, m=4, k=8)
+    cases = [dict(Nc=-1), dict(m=0), dict(k=0), dict(q_pos0=-5), dict(idx_out=0x4004), dict(w=0)]
+    for c in cases:
+        a = lcsa.IndexerArgs(**{**ptrs, **base, **c})
+        assert L.lcsa_indexer_topk(ctypes.byref(a), None, 0, None) == 1, c
+        assert L.lcsa_indexer_topk_noalloc(ctypes.byref(a), None) == 1, c
+    # 8,388,544 scores of one row fill the 32 MiB scratch exactly: with k = 2048 the row
+    # takes the single-phase top-k (more than 16 chunks of 32768) and fits; with k = 64
+    # its two-phase top-k scratch (256 chunks x 64 winners) does not; one more column never fits
+    a = lcsa.IndexerArgs(**{**ptrs, **base, "Nc": 8388544, "k": 64})
+    assert L.lcsa_indexer_topk_noalloc(ctypes.byref(a), None) == 3
+    a.k, a.Nc = 2048, 8388545
+    assert L.lcsa_indexer_topk_noalloc(ctypes.byref(a), None) == 3
+    if not torch.cuda.is_available():
+        a.Nc = 8388544
+        assert L.lcsa_indexer_topk_noalloc(ctypes.byref(a), None) == 4     # fits; no device: no CPU path

@@ -130,3 +130,32 @@ def make_topk_idx(B, Tq, k, n_vis, seed=0, device="cpu"):
                 sel = torch.sort(torch.randperm(nv, generator=g)[:k]).values
             out[b, t, :sel.numel()] = sel.to(torch.int32)
     return out.to(device)
+
+
+def make_layer_inputs(cfg, device="cpu", unit_scale=False):
+    """Every input of one CSA + HCA layer of workload `cfg`, drawn from one
+    generator seeded with cfg.seed in a fixed order (kv, gate, q, indexer q,
+    indexer weights, indexer keys, sink):
+
+      kv    [B,T,D]        N(0,1)/sqrt(D)      (unit_scale: N(0,1))
+      gate  [B,T,D]        N(0,1), or N(0,1)/sqrt(D) when cfg.gate_scale_by_dim
+      q     [B,T,H,D]      N(0,1)/sqrt(D)      (unit_scale: N(0,1))
+      q_idx [B,T,H_I,D_I]  N(0,1)/sqrt(D_I)
+      w     [B,T,H_I]      N(0,1)/sqrt(H_I)    (FP32)
+      k_idx [B,T//m,D_I]   N(0,1)/sqrt(D_I)    (one indexer key per CSA entry)
+      sink  [H]            N(0,1)              (FP32)
+
+    Float inputs are stored in cfg.dtype."""
+    g = _gen(cfg.seed, device)
+    dt = _DT[cfg.dtype]
+    B, T, H, D, H_I, D_I = cfg.B, cfg.T, cfg.H, cfg.D, cfg.H_I, cfg.D_I
+    s = 1.0 if unit_scale else 1.0 / math.sqrt(D)
+    return {
+        "kv": _randn((B, T, D), g, device, s, dt),
+        "gate": _randn((B, T, D), g, device, 1.0 / math.sqrt(D) if cfg.gate_scale_by_dim else 1.0, dt),
+        "q": _randn((B, T, H, D), g, device, s, dt),
+        "q_idx": _randn((B, T, H_I, D_I), g, device, 1.0 / math.sqrt(D_I), dt),
+        "w": _randn((B, T, H_I), g, device, 1.0 / math.sqrt(H_I)),
+        "k_idx": _randn((B, T // cfg.m, D_I), g, device, 1.0 / math.sqrt(D_I), dt),
+        "sink": _randn((H,), g, device),
+    }
