@@ -15,7 +15,7 @@ stack's output, and the oracle's CPU baseline.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lcsa|reference]
                     [--workload stack_4layer_128k|csa_prefill_32k|hca_prefill_128k|csa_decode_1m|
                                 stack_flash_6layer_128k|stack_pro_6layer_128k|csa_prefill_8k|
-                                hca_prefill_16k|csa_decode_8seq]
+                                hca_prefill_16k|csa_decode_8seq|compress_128k]
                     [--no-e2e] [--no-decode] [--no-cpu-baseline] [--no-out-proj]
 
 N > 1 runs under torchrun, one rank per GPU; every rank runs the same
@@ -327,6 +327,10 @@ def config_obj(cfg, world):
     if cfg.decode:
         c.update({"query_position": cfg.T, "entries": cfg.T // cfg.m, "heads": cfg.H, "head_dim": cfg.D,
                   "indexer": f"{cfg.H_I}x{cfg.D_I}", "topk": cfg.k, "window": cfg.W})
+        return c
+    if cfg.name.startswith("compress"):
+        c.update({"calls": ["csa_compress", "hca_compress"], "head_dim": cfg.D, "m": cfg.m, "m_hca": cfg.m_hca,
+                  "gate": "per channel", "l2": "inputs larger than L2; no flush"})
         return c
     layers = list(cfg.layers) if cfg.layers else ["csa" if cfg.name.startswith("csa") else "hca"]
     c.update({"layers": layers, "heads": cfg.H, "head_dim": cfg.D, "rope_dims": cfg.R,
@@ -685,6 +689,42 @@ def append_cost(lcsa, cfg, B, ckv, t, g, dev, reps=20):
     return res
 
 
+def run_compress(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
+    """The two compressors alone on one layer's kv and gate (per-channel
+    gates), each timed with CUDA events; bytes = kv + gate read once plus the
+    entries written."""
+    B, T, D = cfg.B, cfg.T, cfg.D
+    g = gen._gen(rank_seed(cfg.seed, rank), dev)
+    kv = gen._randn((B, T, D), g, dev, 1.0 / math.sqrt(D), torch.bfloat16)
+    gate = gen._randn((B, T, D), g, dev, 1.0, torch.bfloat16)
+    res = {}
+    for name, m, fn in (("csa_compress", cfg.m, lcsa.csa_compress), ("hca_compress", cfg.m_hca, lcsa.hca_compress)):
+        out = torch.empty((B, T // m, D), dtype=torch.bfloat16, device=dev)
+        n0 = lcsa.kernel_launches()
+        fn(kv, gate, m, out=out)
+        torch.cuda.synchronize()
+        launches = lcsa.kernel_launches() - n0
+        ms, clocks = timed(lambda: fn(kv, gate, m, out=out), args.steps * 10, args.warmup, bus_id)
+        ms = max_over_ranks(ms)
+        byts = B * (2 * T * D * 2 + (T // m) * D * 2)
+        gbs = byts / (ms / 1e3) / 1e9
+        res[name] = {"ms": round(ms, 4), "bytes_per_launch": byts, "gbs": round(gbs, 1),
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                  "frac_vs_spec_peak": round(gbs / SPEC_HBM_GBS, 4),
+                                  "peak_source": f"hbm_gbs of {peaks['source']}"},
+                     "gpu_launches": int(launches), "clocks": clocks}
+    units = B * T
+    ms_step = res["csa_compress"]["ms"] + res["hca_compress"]["ms"]
+    return {"metric": METRIC, "value": weak_scaling_throughput(units, ms_step / 1e3, world), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps * 10, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_obj(cfg, world), "kernels": res,
+            "roofline": res["csa_compress"]["roofline"] | {"kernel": "csa_compress", "traffic": None},
+            "gpu_launches": res["csa_compress"]["gpu_launches"] + res["hca_compress"]["gpu_launches"],
+            "note": "one step = csa_compress + hca_compress of one layer's inputs"}
+
+
 def run_single(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     """One layer workload (csa_prefill_32k or hca_prefill_128k)."""
     kind = "csa" if cfg.name.startswith("csa") else "hca"
@@ -754,6 +794,8 @@ def main():
             line = {"metric": METRIC, **line, "n_gpus": world, "steps": args.steps * 4, "warmup": args.warmup,
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                     "data": "synthetic", "config": config_obj(cfg, world)}
+        elif cfg.name.startswith("compress"):
+            line = run_compress(args, cfg, lcsa, dev, world, rank, bus_id, peaks)
         elif cfg.layers:
             line = run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks)
             if not args.no_decode:

@@ -58,6 +58,10 @@ CONFIGS = {
     # CSA decode at 1M context: 64 sequences, one query each at position 2^20.
     "csa_decode_1m": WorkloadConfig(name="csa_decode_1m", dtype="bf16", B=64, T=1 << 20, seed=3,
                                     decode=True, boost_frac=0.01),
+    # The compressors alone on one layer's kv and gate of the stack (B=2,
+    # T=131072, 512 MB of inputs, larger than L2): profiling-sized case of the
+    # CSA and HCA compress kernels.
+    "compress_128k": WorkloadConfig(name="compress_128k", dtype="bf16", B=2, T=131072, seed=11),
     # Alternating four-layer stack CSA->HCA->CSA->HCA, B=2, T=131072.
     "stack_4layer_128k": WorkloadConfig(name="stack_4layer_128k", dtype="bf16", B=2, T=131072, seed=5,
                                         layers=("csa", "hca", "csa", "hca")),
