@@ -25,6 +25,14 @@ inline unsigned long long& launch_counter() {
 }
 inline void count_launch(int n = 1) { __atomic_fetch_add(&launch_counter(), (unsigned long long)n, __ATOMIC_RELAXED); }
 
+// Streaming multiprocessors of the current device.
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
 // ---------------------------------------------------------------------------
 // Element load / store helpers (BF16 storage, FP32 arithmetic).
 // ---------------------------------------------------------------------------

@@ -194,13 +194,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_consta
   }
 }
 
-static int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 // Entry-range splits per query group when there are few groups (decode): the
 // split count s (at most tiles / 8, so a CTA keeps >= 8 tiles) that minimises
 // the waves of one-CTA-per-SM launches times the tiles per CTA, with a
