@@ -423,10 +423,12 @@ def _round_bf16(x):
 # Reading (the pages give no FP8 variant or scale): FP8 E4M3 (bias 7, no
 # infinities, largest finite 448, subnormals m * 2^-9) for the first D - R dims
 # of every entry, with one power-of-two scale per entry 2^X, X the smallest
-# integer with max|x| / 2^X <= 448 (stored as the byte X + 127; an all-zero
-# entry takes X = -127), values rounded to nearest even and saturated at 448;
-# the last R (rotary) dims stay BF16.  A power-of-two scale keeps E4M3 * 2^X
-# exact in BF16, so the cache can be expanded for BF16 tensor cores losslessly.
+# integer with max|x| / 2^X <= 448, raised to at least -124 (stored as the
+# byte X + 127; an all-zero entry takes X = -124), values rounded to nearest
+# even and saturated at 448; the last R (rotary) dims stay BF16.  E4M3 values
+# are multiples of 2^-9, so with X >= -124 every E4M3 * 2^X is a multiple of
+# 2^-133 (the smallest BF16 subnormal) with at most 4 significant bits: exact
+# in BF16, so the cache expands for BF16 tensor cores losslessly.
 # ----------------------------------------------------------------------------
 def e4m3_value(code):
     """Value of an 8-bit E4M3 code from its fields (sign bit 7, exponent bits
@@ -469,7 +471,7 @@ def quantize_entries_fp8(ckv, R):
     # 448 = 0.875 * 2^9, X = e - 9 if f <= 0.875 else e - 8 (exact comparisons)
     f, e = np.frexp(np.where(amax > 0, amax, 1.0))
     X = np.where(f <= 0.875, e - 9, e - 8)
-    X = np.where(amax > 0, np.clip(X, -127, 127), -127).astype(np.int64)
+    X = np.where(amax > 0, np.clip(X, -124, 127), -124).astype(np.int64)
     codes = e4m3_codes(np.ldexp(body, -X[..., None]))
     return codes, (X + 127).astype(np.uint8), _round_bf16(rope)
 

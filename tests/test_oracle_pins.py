@@ -537,7 +537,7 @@ def test_fp8_entry_scale_rule_and_rope_passthrough():
     amax = np.abs(x[:, :D - R]).max(axis=1)
     for i in range(6):
         if amax[i] == 0:
-            assert X[i] == -127 and not codes[i].any()
+            assert X[i] == -124 and not codes[i].any()
         else:
             assert amax[i] <= 448.0 * 2.0 ** X[i] and amax[i] > 448.0 * 2.0 ** (X[i] - 1)
     assert X[2] == -3
@@ -564,3 +564,28 @@ def test_fp8_entry_roundtrip_of_representable_entries():
     c2, s2, r2 = O.quantize_entries_fp8(x, 64)
     np.testing.assert_array_equal(s2, sc)
     np.testing.assert_array_equal(O.dequantize_entries_fp8(c2, s2, r2), x)
+
+
+def test_fp8_entry_tiny_magnitudes_stay_exact_in_bf16():
+    # entries far below 448 * 2^-124 take the floor scale X = -124: their codes
+    # are E4M3 subnormals or zero, and every dequantised value is a BF16 number
+    # (multiples of 2^-133), checked against an independent BF16 rounding
+    r = _rng(43)
+    D, R = 512, 64
+    x = r.standard_normal((3, D))
+    x[0, :D - R] *= 2.0 ** -128                   # amax ~ 2^-126: normal FP64, far below the floor
+    x[1, :D - R] *= 2.0 ** -130
+    x[2, :D - R] = 0.0
+    x[2, 5] = 2.0 ** -133                         # one BF16-subnormal-sized value
+    codes, sc, rope = O.quantize_entries_fp8(x, R)
+    assert (sc.astype(np.int64) - 127 == -124).all()
+    d = O.dequantize_entries_fp8(codes, sc, rope)
+    body = d[:, :D - R]
+    np.testing.assert_array_equal(body, O._round_bf16(body))
+    assert (np.abs(np.rint(body * 2.0 ** 133) - body * 2.0 ** 133) == 0).all()
+    # the one value of row 2 is the E4M3 code 2^-9 times 2^-124
+    assert codes[2, 5] == 0x01 and d[2, 5] == 2.0 ** -133
+    # E4M3 error bound at the floor scale: 2^-4 relative on normals, half the
+    # subnormal spacing (2^-10 * 2^-124) below
+    err = np.abs(body - x[:, :D - R])
+    assert (err <= np.maximum(np.abs(x[:, :D - R]) * 2.0 ** -4, 2.0 ** -134)).all()
