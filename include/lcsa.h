@@ -12,7 +12,8 @@
  *   [p3] untitled classical-Chinese paraphrase page: the "Partial RoPE",
  *        "Attention sink", "第一步/第二步/第三步" step sentences, and the
  *        strict-causality, HCA-no-overlap and sliding-window sentences
- *   [p4] "DeepSeek V4 技术架构深度解析", section "二、CSA + HCA"
+ *   [p4] "DeepSeek V4 技术架构深度解析", section "二、CSA + HCA" (with
+ *        "KV Cache优化细节")
  *
  * Conventions shared by every call
  *   - Every tensor argument is a DEVICE pointer, allocated and owned by the
@@ -361,6 +362,47 @@ lcsa_status lcsa_csa_sparse_attn(const lcsa_attn_args* a, void* workspace,
 lcsa_status lcsa_hca_dense_attn(const lcsa_attn_args* a, void* workspace,
                                 size_t workspace_bytes, void* stream);
 int lcsa_attn_uses_tensor_cores(const lcsa_attn_args* a);
+
+/* ------------------------------------------------------------------------
+ * FP8 entry cache ([p4] "二、CSA + HCA" / "KV Cache优化细节": the compressed
+ * KV cache keeps the RoPE dims in BF16 and the rest in FP8).  The pages give
+ * no FP8 variant or scale; this library's format, per entry row x[0..D):
+ *   - body x[0..D-R): one E4M3 byte per value (bias 7, no infinities,
+ *     largest finite 448, subnormals m * 2^-9), the value nearest to
+ *     x / 2^X (ties to even, magnitudes above 448 saturate, a zero of either
+ *     sign coded +0), with one scale per entry: X the smallest integer with
+ *     max|body| <= 448 * 2^X, raised to at least -124 (-124 for an all-zero
+ *     body), stored as the byte X + 127;
+ *   - rotary dims x[D-R..D): BF16 (round to nearest even).
+ * Every E4M3 * 2^X with X >= -124 is a BF16 number, so the attention calls
+ * expand entries to BF16 exactly.  Bytes per entry at D=512, R=64:
+ * 448 + 1 + 128 = 577 against 1024.
+ *
+ *   x      [rows, D] dtype (BF16 or FP32), device, aligned to its element size
+ *   codes  [rows, D-R] uint8        scales [rows] uint8
+ *   rope   [rows, R] BF16
+ * R must be even and less than D; codes, scales and rope are a pure function
+ * of x (bit-exact with any other exact implementation of the rule above).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const uint8_t* codes;   /* [B,Nc,D-R] E4M3, 16-byte aligned                  */
+  const uint8_t* scales;  /* [B,Nc] X + 127                                    */
+  const void* rope;       /* [B,Nc,R] BF16, 16-byte aligned                    */
+} lcsa_fp8_entries;
+
+lcsa_status lcsa_quantize_entries_fp8(const void* x, int64_t rows, int D, int R, lcsa_dtype dtype,
+                                      uint8_t* codes, uint8_t* scales, void* rope, void* stream);
+
+/* Core attention (as lcsa_csa_sparse_attn / lcsa_hca_dense_attn) over
+ * entries held in the FP8 cache `e` instead of a->ckv (not read; may be
+ * NULL).  Every other argument, the workspace (lcsa_attn_workspace) and the
+ * results are those of the BF16 calls on the expanded entries.  Only the
+ * tensor-core shapes (BF16 q/kv, H=64, D=512, R=64); LCSA_ERR_UNSUPPORTED
+ * otherwise. */
+lcsa_status lcsa_csa_sparse_attn_fp8(const lcsa_attn_args* a, const lcsa_fp8_entries* e, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+lcsa_status lcsa_hca_dense_attn_fp8(const lcsa_attn_args* a, const lcsa_fp8_entries* e, void* workspace,
+                                    size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

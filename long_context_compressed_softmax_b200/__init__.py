@@ -34,6 +34,7 @@ EXPORTED = [
     "lcsa_quantize_mxfp4", "lcsa_indexer_topk_mxfp4_workspace", "lcsa_indexer_topk_mxfp4",
     "lcsa_grouped_out_proj_workspace", "lcsa_grouped_out_proj",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
+    "lcsa_quantize_entries_fp8", "lcsa_csa_sparse_attn_fp8", "lcsa_hca_dense_attn_fp8",
 ]
 
 
@@ -82,6 +83,10 @@ class AttnArgs(ctypes.Structure):
     ]
 
 
+class Fp8Entries(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rope", ctypes.c_void_p)]
+
+
 _vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 _sig = {
     "lcsa_version": (ctypes.c_char_p, []),
@@ -107,6 +112,9 @@ _sig = {
     "lcsa_csa_sparse_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_attn_uses_tensor_cores": (_i, [ctypes.POINTER(AttnArgs)]),
+    "lcsa_quantize_entries_fp8": (_i, [_vp, _i64, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "lcsa_csa_sparse_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
+    "lcsa_hca_dense_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -390,3 +398,61 @@ def hca_dense_attn(q, ckv, kv, sink, q_pos0, kv_pos0, m=128, W=128, R=64, softma
     """HCA core attention over every visible entry plus the window and sink."""
     return _attn(_lib.lcsa_hca_dense_attn, "hca_dense_attn", 0, q, ckv, None, kv, sink, q_pos0, kv_pos0, m, W, R,
                  softmax_scale, rope_base, out_dtype, return_lse, workspace, out)
+
+
+# ----------------------------------------------------------------- FP8 entry cache
+def quantize_entries_fp8(ckv, R=64, codes=None, scales=None, rope=None):
+    """FP8 entry cache of ckv [..., D] (BF16 or FP32): E4M3 codes of the first
+    D-R dims with one power-of-two scale per entry, the last R dims in BF16
+    -> (codes uint8 [..., D-R], scales uint8 [...], rope BF16 [..., R])."""
+    _need_contig(ckv)
+    D = ckv.shape[-1]
+    rows = ckv.numel() // D if D else 0
+    lead = ckv.shape[:-1]
+    if codes is None:
+        codes = torch.empty(lead + (D - R,), dtype=torch.uint8, device=ckv.device)
+    if scales is None:
+        scales = torch.empty(lead, dtype=torch.uint8, device=ckv.device)
+    if rope is None:
+        rope = torch.empty(lead + (R,), dtype=torch.bfloat16, device=ckv.device)
+    st = _lib.lcsa_quantize_entries_fp8(_p(ckv), rows, D, R, _dt(ckv), _p(codes), _p(scales), _p(rope),
+                                        _stream(ckv.device))
+    _check(st, "quantize_entries_fp8")
+    return codes, scales, rope
+
+
+def _attn_fp8(fn, name, sparse, q, cache, idx, kv, sink, q_pos0, kv_pos0, m, W, R, softmax_scale, rope_base,
+              out_dtype, return_lse, workspace, out):
+    codes, scales, rope = cache
+    _need_contig(q, codes, scales, rope, idx, kv, sink)
+    B, Tq, H, D = q.shape
+    Nc = codes.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Tq, H, D), dtype=out_dtype, device=dev)
+    lse = torch.empty((B, Tq, H), dtype=torch.float32, device=dev) if return_lse else None
+    k = idx.shape[2] if idx is not None else 0
+    a = AttnArgs(_p(q), None, _p(idx), _p(kv), _p(sink), B, Tq, H, D, R, Nc, k, kv.shape[1], int(q_pos0),
+                 int(kv_pos0), m, W, float(softmax_scale), float(rope_base), _dt(q), _p(out), _dt(out), _p(lse))
+    e = Fp8Entries(_p(codes), _p(scales), _p(rope))
+    need = int(_lib.lcsa_attn_workspace(ctypes.byref(a), sparse))
+    if need > 0 and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_n = 0 if workspace is None else workspace.numel()
+    st = fn(ctypes.byref(a), ctypes.byref(e), _p(workspace), ws_n, _stream(dev))
+    _check(st, name)
+    return (out, lse) if return_lse else out
+
+
+def csa_sparse_attn_fp8(q, cache, idx, kv, sink, q_pos0, kv_pos0, m=4, W=128, R=64, softmax_scale=0.0,
+                        rope_base=10000.0, out_dtype=torch.float32, return_lse=False, workspace=None, out=None):
+    """CSA core attention with the entries in the FP8 cache (codes, scales, rope)."""
+    return _attn_fp8(_lib.lcsa_csa_sparse_attn_fp8, "csa_sparse_attn_fp8", 1, q, cache, idx, kv, sink, q_pos0,
+                     kv_pos0, m, W, R, softmax_scale, rope_base, out_dtype, return_lse, workspace, out)
+
+
+def hca_dense_attn_fp8(q, cache, kv, sink, q_pos0, kv_pos0, m=128, W=128, R=64, softmax_scale=0.0,
+                       rope_base=10000.0, out_dtype=torch.float32, return_lse=False, workspace=None, out=None):
+    """HCA core attention with the entries in the FP8 cache (codes, scales, rope)."""
+    return _attn_fp8(_lib.lcsa_hca_dense_attn_fp8, "hca_dense_attn_fp8", 0, q, cache, None, kv, sink, q_pos0,
+                     kv_pos0, m, W, R, softmax_scale, rope_base, out_dtype, return_lse, workspace, out)

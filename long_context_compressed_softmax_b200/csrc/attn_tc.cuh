@@ -36,6 +36,7 @@
 #pragma once
 #include "tc_ptx.cuh"
 #include "rope.cuh"
+#include "fp8cache.cuh"
 
 namespace lcsa {
 
@@ -59,9 +60,13 @@ constexpr uint32_t kAtOffTab = kAtOffP + 2 * kAtPBytes;
 constexpr uint32_t kAtOffIdx = kAtOffTab + kAtStages * kAtKT * 2 * 8;
 constexpr uint32_t kAtOffCs = kAtOffIdx + kAtMaxIdx * 4;               // [kAtStages] per stage, [2] per item
 constexpr uint32_t kAtOffStats = kAtOffCs + (kAtStages + 2) * kAtCsBytes;   // [2][64] (row max, row sum)
-constexpr uint32_t kAtOffBar = kAtOffStats + 2 * 64 * 8;
+constexpr uint32_t kAtOffScl = kAtOffStats + 2 * 64 * 8;             // [kAtStages][64] FP8 entry scales
+constexpr uint32_t kAtOffKm = kAtOffScl + kAtStages * kAtKT * 4;        // [kAtStages][2] valid-row masks
+constexpr uint32_t kAtOffBar = kAtOffKm + 32;
 constexpr int kAtBars = 21;
 constexpr size_t kAtSmem = 1024 + kAtOffBar + kAtBars * 8;
+static_assert(kAtSmem <= 232448, "attention shared memory exceeds 227 KB");
+constexpr int kAtCodeBytes = 448;               // FP8 entry cache: E4M3 bytes of dims 0..447 per entry
 constexpr float kLog2e = 1.4426950408889634f;
 // TMEM map: lanes 0-15 of each sub-partition hold S[0] (cols 0-63), S[1]
 // (64-127) and Q (128-383, the A operand of S = Q K^T); lanes 16-31 hold O
@@ -81,10 +86,13 @@ struct AtGeom {
   int out_bf16;
   int out_v8;          // the output (or split partials) is 32-byte aligned: 32-byte stores
   int n_items;         // rows * splits
+  int fp8;             // entries come from the FP8 cache (codes + scales + BF16 rotary slices)
 };
 
 struct AtPtrs {
   const __nv_bfloat16* ckv;
+  const uint8_t* c8;            // FP8 entry cache: codes [B*Nc][448] (else null)
+  const uint8_t* c8s;           // FP8 entry cache: scale bytes X + 127 [B*Nc]
   const int32_t* idx;
   const int32_t* nc;            // sparse: number of valid selected entries of each query row
   const float2* cs;             // [Tq][32] (cos, sin) at each query position
@@ -330,6 +338,8 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
   float2* s_cs = reinterpret_cast<float2*>(smem + kAtOffCs);                  // [stage][32] with the Q pseudo-tile
   float2* s_cs_item = s_cs + kAtStages * 32;                                  // [2][32] for the epilogue
   float2* s_stats = reinterpret_cast<float2*>(smem + kAtOffStats);            // [2][64] softmax -> epilogue
+  float* s_scl = reinterpret_cast<float*>(smem + kAtOffScl);                  // [stage][64] FP8 entry scales
+  uint32_t* s_km = reinterpret_cast<uint32_t*>(smem + kAtOffKm);              // [stage][2] rows read (gathered tiles)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAtOffBar);
   uint64_t* q_ready = bars + 0;                 // transition warps (4): Q of the item is in TMEM
   uint64_t* kv_full = bars + 1;                 // [kAtStages] producers (one arrival each; TMA bytes)
@@ -393,6 +403,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       tc::prefetch_tmap(&tm_rotw);
     }
     const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.cs);
+    // Entry tiles that every producer fills (gathered rows, FP8 expansion)
+    // make the producers leave only together, at named barrier 1.
+    const bool coll = g.sparse || g.fp8;
     bool bad = false;
     int slot = 0, ni = 0;
     int nc_next = at_item_nc(g, P, blockIdx.x);
@@ -408,7 +421,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         const int st = slot % kAtStages;
         if (slot >= kAtStages && !tc::mbar_wait_backoff(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
         if (*abort_flag) bad = true;
-        if (bad && !g.sparse) break;
+        if (bad && !coll) break;
         if (tid == 0) {
           uint64_t* qf = q_full + (ni & 1);
           if (!bad) {
@@ -452,9 +465,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         if (*abort_flag) bad = true;
         const int gt = x.t0 + n;                    // tile index in the query's key list
         uint8_t* stage = s_k + st * kAtKBytes;
-        if (gt >= x.ks.tiles_c || !g.sparse) {
+        if (gt >= x.ks.tiles_c || !coll) {
           // ---- contiguous rows: TMA boxes
-          if (g.sparse) {
+          if (coll) {
             if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
           } else if (bad) {
             break;
@@ -479,27 +492,79 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           }
           continue;
         }
-        // ---- gathered rows (CSA): per-tile row table, then 16-byte cp.async pieces
+        // ---- gathered rows (CSA) or FP8 entry rows: per-tile row table first
         const uint8_t** tab = s_tab + st * kAtKT * 2;
         if (tid < kAtKT) {
           const int kk = tid;
           const uint8_t* rm = nullptr;
           const uint8_t* rr = nullptr;
+          float scl = 0.f;
           const int sl = gt * kAtKT + kk;
           if (sl < x.ks.n_c) {
-            const int j = s_idx[sl - slot0];
+            const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
             if (j >= 0 && j < g.Nc) {
-              rm = reinterpret_cast<const uint8_t*>(P.ckv + ((long long)x.b * g.Nc + j) * 512);
-              rr = reinterpret_cast<const uint8_t*>(
-                  P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : ((long long)x.b * g.Nc + j)) * 64);
+              const long long e = (long long)x.b * g.Nc + j;
+              rm = g.fp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
+              rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
+              if (g.fp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
             } else {
               report(LCSA_DEV_BAD_INDEX);
             }
           }
           tab[2 * kk] = rm;
           tab[2 * kk + 1] = rr;
+          s_scl[st * kAtKT + kk] = scl;
+          // keys whose row is read: a bad index is skipped, not a zero key
+          const uint32_t vm = __ballot_sync(0xffffffffu, rm != nullptr);
+          if ((kk & 31) == 0) s_km[st * 2 + (kk >> 5)] = vm;
         }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
+        if (g.fp8) {
+          // FP8 entry rows: every 16-byte load (codes and rotary slices) is
+          // issued before the first conversion; codes expand to BF16 with the
+          // entry's power-of-two scale (exact) and land at the swizzled
+          // addresses; absent rows are zeros.  Generic-proxy stores, so a
+          // proxy fence precedes this thread's arrival.
+          constexpr int kCodePer = kAtKT * (kAtCodeBytes / 16) / kAtProdThreads;   // 7
+          constexpr int kRopePer = kAtKT * 8 / kAtProdThreads;                     // 2
+          static_assert(kCodePer * kAtProdThreads == kAtKT * (kAtCodeBytes / 16), "code pieces per thread");
+          static_assert(kRopePer * kAtProdThreads == kAtKT * 8, "rotary pieces per thread");
+          uint4 cv[kCodePer], rv[kRopePer];
+#pragma unroll
+          for (int u = 0; u < kCodePer; ++u) {
+            const int q = tid + u * kAtProdThreads;
+            const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
+            const uint8_t* base = tab[2 * kk];
+            cv[u] = base ? __ldg(reinterpret_cast<const uint4*>(base + p * 16)) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < kRopePer; ++u) {
+            const int q = tid + u * kAtProdThreads;
+            const int kk = q >> 3, c16 = q & 7;
+            const uint8_t* base = tab[2 * kk + 1];
+            rv[u] = base ? __ldg(reinterpret_cast<const uint4*>(base + c16 * 16)) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < kCodePer; ++u) {
+            const int q = tid + u * kAtProdThreads;
+            const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
+            uint4 lo, hi;
+            e4m3x16_to_bf16(cv[u], s_scl[st * kAtKT + kk], lo, hi);
+            uint8_t* row = stage + (p >> 2) * kAtRegion + kk * 128;   // 16 codes = dims 16p .. 16p+15
+            const int c0 = (p & 3) * 2;
+            *reinterpret_cast<uint4*>(row + ((c0 ^ (kk & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (kk & 7)) << 4)) = hi;
+          }
+#pragma unroll
+          for (int u = 0; u < kRopePer; ++u) {
+            const int q = tid + u * kAtProdThreads;
+            const int kk = q >> 3, c16 = q & 7;
+            *reinterpret_cast<uint4*>(stage + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4)) = rv[u];
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(kv_full + st);
+          continue;
+        }
         // 16-byte piece q = tid + u * kAtProdThreads of the 64 x 1 KB tile:
         // key q / 64, piece q % 64 of its row (region = 64-dim block).
         const uint32_t sbase = tc::smem_u32(stage);
@@ -637,10 +702,19 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         const int gt = x.t0 + n;
         int nvalid = gt < x.ks.tiles_c ? x.ks.n_c - gt * kAtKT : x.ks.n_w - (gt - x.ks.tiles_c) * kAtKT;
         nvalid = (nvalid < kAtKT ? nvalid : kAtKT) - 32 * half;   // valid keys among this thread's 32
+        uint32_t km = nvalid >= 32 ? 0xffffffffu : (nvalid <= 0 ? 0u : (1u << nvalid) - 1u);
+        if (g.sparse && gt < x.ks.tiles_c) {
+          // gathered tile: the producers' row mask of its stage (slot = ga + ni + 1, one Q
+          // slot per item before its tiles); the stage's fill completed before S, so this
+          // wait returns at once and orders the mask's reads after the producers' writes
+          const int sl = ga + ni + 1;
+          if (!tc::mbar_wait(kv_full + sl % kAtStages, (sl / kAtStages) & 1)) ok = false;
+          km &= s_km[(sl % kAtStages) * 2 + half];
+        }
         float tmax = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float s = j < nvalid ? __uint_as_float(v[j]) : -INFINITY;
+          const float s = (km >> j) & 1u ? __uint_as_float(v[j]) : -INFINITY;
           v[j] = __float_as_uint(s);
           tmax = fmaxf(tmax, s);
         }
@@ -676,7 +750,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         {
           float psum = 0.f;
           uint8_t* prow = s_p + sb * kAtPBytes + h * 128;
-          const float neg_m = -m_run;
+          const float neg_m = m_run == -INFINITY ? 0.f : -m_run;   // no valid key yet: every p is 0
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[4];
@@ -901,7 +975,9 @@ static AtPlan attn_tc_plan(const lcsa_attn_args* a, int sparse) {
 
 static size_t attn_tc_workspace(const lcsa_attn_args* a, int sparse) { return attn_tc_plan(a, sparse).total; }
 
-static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws, cudaStream_t st) {
+// f8 != null: the entries come from the FP8 cache (a->ckv is not read).
+static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws, cudaStream_t st,
+                                  const lcsa_fp8_entries* f8 = nullptr) {
   const AtPlan pl = attn_tc_plan(a, sparse);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   const double log_base = log(a->rope_base > 0.f ? (double)a->rope_base : 10000.0);
@@ -910,6 +986,8 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   if (rows * pl.splits * 64 > (long long)INT32_MAX - 64 * 1024) return cudaErrorInvalidValue;
   AtPtrs P;
   P.ckv = (const __nv_bfloat16*)a->ckv;
+  P.c8 = f8 ? f8->codes : nullptr;
+  P.c8s = f8 ? f8->scales : nullptr;
   P.idx = sparse ? a->idx : nullptr;
   P.nc = (const int32_t*)(w + pl.off_nc);
   P.cs = (const float2*)(w + pl.off_cs);
@@ -921,13 +999,15 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   P.o_part = (float*)(w + pl.off_opart);
   P.ml_part = (float*)(w + pl.off_ml);
   cudaError_t e;
-  // rotary slices of the keys
+  // rotary slices of the keys (from the entries, or from the FP8 cache's BF16 rotary dims)
   if (a->Nc > 0) {
+    const void* rsrc = f8 ? f8->rope : a->ckv;
+    const int rld = f8 ? kRopeR : 512;
     if (pl.rot_slot)
-      e = launch_rope_rows(a->ckv, w + pl.off_rot_c, rows * a->k, 512, 1, 0, a->m, log_base, 1, a->idx,
+      e = launch_rope_rows(rsrc, w + pl.off_rot_c, rows * a->k, rld, 1, 0, a->m, log_base, 1, a->idx,
                            (long long)a->Tq * a->k, a->Nc, st);
     else
-      e = launch_rope_rows(a->ckv, w + pl.off_rot_c, (long long)a->B * a->Nc, 512, a->Nc, 0, a->m, log_base, 0,
+      e = launch_rope_rows(rsrc, w + pl.off_rot_c, (long long)a->B * a->Nc, rld, a->Nc, 0, a->m, log_base, 0,
                            nullptr, 0, a->Nc, st);
     if (e != cudaSuccess) return e;
   }
@@ -958,6 +1038,7 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   g.out_bf16 = a->out_dtype == LCSA_BF16;
   g.out_v8 = (reinterpret_cast<uintptr_t>(pl.splits > 1 ? (const void*)P.o_part : a->out) & 31u) == 0 ? 1 : 0;
   g.n_items = (int)(rows * pl.splits);
+  g.fp8 = f8 != nullptr;
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
   if (e != cudaSuccess) return e;
   // Tensor maps (64-row boxes, 128-byte swizzle).  A map whose tensor is
@@ -969,7 +1050,7 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
     return make_tmap_bf16_2d(m, base, nrows, cols, cols, 64, 64);
   };
   bool okm = mk(&m_q, a->q, (uint64_t)rows * 64, 512) &&
-             mk(&m_ckv, a->Nc > 0 ? a->ckv : nullptr, (uint64_t)a->B * a->Nc, 512) &&
+             mk(&m_ckv, (a->Nc > 0 && !f8) ? a->ckv : nullptr, (uint64_t)a->B * a->Nc, 512) &&
              mk(&m_kv, a->Tkv > 0 ? a->kv : nullptr, (uint64_t)a->B * a->Tkv, 512) &&
              mk(&m_rotc, a->Nc > 0 ? (const void*)P.rot_c : nullptr, rows_rotc, 64) &&
              mk(&m_rotw, (a->Tkv > 0 && a->W > 0) ? (const void*)P.rot_w : nullptr, (uint64_t)a->B * a->Tkv, 64);

@@ -9,7 +9,7 @@
 // token costs one exp per element.  Consecutive entries of a block share
 // their overlapping CSA tokens through L1/L2, so DRAM reads each token once.
 #pragma once
-#include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace lcsa {
 
@@ -104,246 +104,185 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
 }
 
 // ---------------------------------------------------------------------------
-// Streaming compressor for whole sequences (window 2m or m, no RMSNorm).
+// Streaming compressor for whole sequences (per-channel gates, window 2m or m,
+// no RMSNorm): token rows reach shared memory by bulk copies.
 //
-// Each thread owns 4 channels and walks a stream of tokens 4 at a time (a
-// chunk): raw 8-byte (BF16) or 16-byte (FP32) vectors of kv and gate, the next
-// chunk's loads issued before the current chunk is reduced.  A block of m
-// tokens folds into a per-channel softmax state (running max, sum of weights,
-// weighted sum): one exp per element plus one rescale per chunk.
-//   CSA (window 2m): entry j pools blocks j-1 and j, so it is the merge of
-//     two neighbouring block states; a thread walks kCsaRun consecutive
-//     blocks (plus the block before them) and emits one entry per block.
-//   HCA (window m): the lanes of a CTA split a block's m tokens, and their
-//     states merge through shared memory.
-// A warp reads 256 contiguous bytes of a token row per load (32 threads x 8
-// bytes); the CTA covers whole rows.  The grid is persistent (two CTAs of 256
-// threads per SM) and strides over work units.
+// A CTA owns a contiguous range of blocks (m tokens each) of one sequence and
+// streams their token rows, kCmpRows at a time, through a kCmpStages-deep ring:
+// one thread issues two cp.async.bulk copies per stage (kv rows, gate rows;
+// contiguous in HBM) that complete on the stage's mbarrier, so the bytes in
+// flight do not depend on registers or occupancy.  Each thread owns two
+// channels of every row and folds the rows in order, up to 4 at a time (one
+// rescale by the chunk's maximum), into a per-channel softmax state (running
+// max, sum of weights, weighted sum):
+//   HCA (window m): the entry is the state of its block;
+//   CSA (window 2m): entry j pools blocks j-1 and j, the merge of two
+//     neighbouring block states; the range starts one block early so that its
+//     first entry has its predecessor.
+// Every wait is bounded; a CTA whose wait gave up stops at the same stage on
+// all threads (__syncthreads_and), waits (bounded) for its copies in flight
+// and leaves.
 // ---------------------------------------------------------------------------
-constexpr int kCsaRun = 16;          // CSA blocks per thread
-constexpr int kStreamThreads = 256;
+constexpr int kCmpRows = 16;       // token rows per stage
+constexpr int kCmpStages = 3;
 
-template <typename Tin> struct Raw4;                      // 4 channels of one token
-template <> struct Raw4<__nv_bfloat16> { using T = uint2; };
-template <> struct Raw4<float> { using T = float4; };
-
-// Channel v (0..3) of a raw 4-channel vector as FP32 (a BF16 value is the
-// high half of its FP32 bit pattern).
-__device__ __forceinline__ float chan(const uint2& r, int v) {
-  const uint32_t w = v < 2 ? r.x : r.y;
-  return __uint_as_float((v & 1) ? (w & 0xffff0000u) : (w << 16));
-}
-__device__ __forceinline__ float chan(const float4& r, int v) {
-  return v == 0 ? r.x : (v == 1 ? r.y : (v == 2 ? r.z : r.w));
-}
-
-struct Soft4 {                 // softmax state of 4 channels
-  float m[4], s[4], a[4];
+struct Soft2 {                     // softmax state of 2 channels
+  float m[2], s[2], a[2];
   __device__ __forceinline__ void reset() {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) { m[v] = -INFINITY; s[v] = 0.f; a[v] = 0.f; }
+    m[0] = m[1] = -INFINITY;
+    s[0] = s[1] = a[0] = a[1] = 0.f;
   }
 };
 
-// One chunk of a thread's token stream: n (<= 4) tokens from token t.
-template <typename Tin, bool kPC>
-struct Chunk4 {
-  typename Raw4<Tin>::T x[4], g[4];
-  float gs[4];                 // scalar gates (kPC = false)
-  __device__ __forceinline__ void load(const typename Raw4<Tin>::T* kvp, const typename Raw4<Tin>::T* gp,
-                                       const Tin* gsp, long long t, int n, int tpr) {
+// Two consecutive channels of a staged row as FP32.
+__device__ __forceinline__ float2 ld2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 ld2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+
+// Fold rows r .. r+n-1 (n <= 4) of a staged tile into st.
+template <typename Tin>
+__device__ __forceinline__ void fold_rows(Soft2& st, const Tin* kvs, const Tin* gs, int D, int r, int n) {
+  float2 x[4], g[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < 4; ++u)
+    if (u < n) {
+      x[u] = ld2(kvs + (r + u) * D);
+      g[u] = ld2(gs + (r + u) * D);
+    }
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    float cm = st.m[v];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) if (u < n) cm = fmaxf(cm, v ? g[u].y : g[u].x);
+    const float alpha = __expf(st.m[v] - cm);          // 0 while the state is empty
+    float a = st.a[v] * alpha, sm = st.s[v] * alpha;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
       if (u < n) {
-        x[u] = __ldg(kvp + (t + u) * tpr);
-        if constexpr (kPC) g[u] = __ldg(gp + (t + u) * tpr);
-        else gs[u] = ld_scalar(gsp + t + u);
+        const float p = __expf((v ? g[u].y : g[u].x) - cm);
+        sm += p;
+        a = fmaf(p, v ? x[u].y : x[u].x, a);
       }
-    }
-  }
-  // fold the chunk's n tokens into st: one rescale by the chunk maximum;
-  // channel by channel, each value converted where it is used
-  __device__ __forceinline__ void fold(Soft4& st, int n) const {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      float cm = st.m[v];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) if (u < n) cm = fmaxf(cm, gate_at(u, v));
-      const float alpha = __expf(st.m[v] - cm);        // 0 while the state is empty
-      float a = st.a[v] * alpha, sm = st.s[v] * alpha;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (u < n) {
-          const float p = __expf(gate_at(u, v) - cm);
-          sm += p;
-          a = fmaf(p, chan(x[u], v), a);
-        }
-      }
-      st.m[v] = cm; st.s[v] = sm; st.a[v] = a;
-    }
-  }
-  __device__ __forceinline__ float gate_at(int u, int v) const {
-    if constexpr (kPC) return chan(g[u], v);
-    else return gs[u];
-  }
-};
-
-// Pooled value of the union of two states' tokens (A may be empty).
-__device__ __forceinline__ void merge_out(const Soft4& A, const Soft4& B, float* o) {
-#pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const float M = fmaxf(A.m[v], B.m[v]);
-    const float fa = __expf(A.m[v] - M), fb = __expf(B.m[v] - M);
-    o[v] = (A.a[v] * fa + B.a[v] * fb) / (A.s[v] * fa + B.s[v] * fb);
+    st.m[v] = cm; st.s[v] = sm; st.a[v] = a;
   }
 }
 
-// Walk nb blocks of `bl` tokens starting at token t0 in chunks of 4 tokens;
-// two chunk buffers alternate, so the next chunk's loads are in flight while
-// the current one is folded.  on_block(k, state) runs after block k.
-template <typename Tin, bool kPC, typename F>
-__device__ __forceinline__ void walk_blocks(const typename Raw4<Tin>::T* kvp, const typename Raw4<Tin>::T* gp,
-                                            const Tin* gsp, int tpr, long long t0, int nb, int bl, F&& on_block) {
-  if (nb <= 0 || bl <= 0) return;
-  const int cpb = (bl + 3) >> 2;
-  const int nq = nb * cpb;
-  Chunk4<Tin, kPC> ca, cb;
-  Soft4 st;
+template <typename Tin, typename Tout, bool kCSA>
+__global__ void __launch_bounds__(1024)
+compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* __restrict__ out, int T, int D,
+                     int m, int Nc, int blocks_per_unit, int units_per_seq) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t row_bytes = (uint32_t)D * sizeof(Tin);
+  const uint32_t tile_bytes = kCmpRows * row_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCmpStages * 2 * tile_bytes);
+  const int tid = threadIdx.x;
+  const int b = blockIdx.x / units_per_seq;
+  const int unit = blockIdx.x - b * units_per_seq;
+  const int jb = unit * blocks_per_unit;                              // first entry of this CTA
+  const int je = jb + blocks_per_unit < Nc ? jb + blocks_per_unit : Nc;
+  if (jb >= je) return;                                               // uniform over the CTA
+  const int first = (kCSA && jb > 0) ? jb - 1 : jb;                   // first block streamed
+  const long long ta = (long long)first * m;                          // first token row
+  const int rows = (je - first) * m;
+  const int K = (rows + kCmpRows - 1) / kCmpRows;                     // stages
+  const Tin* kvb = kv + ((long long)b * T + ta) * D;
+  const Tin* gb = gate + ((long long)b * T + ta) * D;
+
+  if (tid == 0) {
+    for (int s = 0; s < kCmpStages; ++s) tc::mbar_init(full + s, 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int k) {                                           // stage k into slot k % kCmpStages
+    const int slot = k % kCmpStages;
+    const int r0 = k * kCmpRows;
+    const int n = rows - r0 < kCmpRows ? rows - r0 : kCmpRows;
+    uint8_t* dst = smem + slot * 2 * tile_bytes;
+    tc::mbar_arrive_expect_tx(full + slot, 2u * n * row_bytes);
+    tc::bulk_load(dst, kvb + (long long)r0 * D, n * row_bytes, full + slot);
+    tc::bulk_load(dst + tile_bytes, gb + (long long)r0 * D, n * row_bytes, full + slot);
+  };
+  if (tid == 0)
+    for (int k = 0; k < kCmpStages && k < K; ++k) issue(k);
+
+  const int c = 2 * tid;                                              // this thread's channels c, c+1
+  const bool has = c < D;
+  Soft2 st, prev;
   st.reset();
-  int k = 0, w = 0;                  // block and chunk-in-block of the chunk being folded
-  int kl = 0, wl = 0;                // ... of the next chunk to load
-  auto load = [&](Chunk4<Tin, kPC>& c) {
-    const int n = bl - 4 * wl < 4 ? bl - 4 * wl : 4;
-    c.load(kvp, gp, gsp, t0 + (long long)kl * bl + 4 * wl, n, tpr);
-    if (++wl == cpb) { wl = 0; ++kl; }
-  };
-  auto fold = [&](const Chunk4<Tin, kPC>& c) {
-    const int n = bl - 4 * w < 4 ? bl - 4 * w : 4;
-    c.fold(st, n);
-    if (++w == cpb) {
-      on_block(k, st);
-      st.reset();
-      w = 0;
-      ++k;
-    }
-  };
-  load(ca);
-  for (int q = 0; q < nq; q += 2) {
-    if (q + 1 < nq) load(cb);
-    fold(ca);
-    if (q + 1 < nq) {
-      if (q + 2 < nq) load(ca);
-      fold(cb);
-    }
-  }
-}
-
-template <typename Tin, typename Tout, bool kPC, bool kCSA>
-__global__ void __launch_bounds__(kStreamThreads, 2)
-compress_stream_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* __restrict__ out, int T, int D,
-                       int m, int Nc, int units_per_seq, long long n_units) {
-  using R = typename Raw4<Tin>::T;
-  const int tpr = D >> 2;                          // threads per token row
-  const int nl = blockDim.x / tpr;                 // lanes (token streams) per CTA
-  const int c = threadIdx.x % tpr, l = threadIdx.x / tpr;
-  extern __shared__ float s_part[];                // HCA: [nl][tpr][12] lane states
-  for (long long u = blockIdx.x; u < n_units; u += gridDim.x) {
-    const int b = (int)(u / units_per_seq);
-    const int r = (int)(u - (long long)b * units_per_seq);
-    const R* kvp = reinterpret_cast<const R*>(kv + (long long)b * T * D) + c;
-    const R* gp = kPC ? reinterpret_cast<const R*>(gate + (long long)b * T * D) + c : nullptr;
-    const Tin* gsp = kPC ? nullptr : gate + (long long)b * T;
-    Tout* ob = out + (long long)b * Nc * D + c * 4;
-    if constexpr (kCSA) {
-      if (l >= nl) continue;
-      const int jb = (r * nl + l) * kCsaRun;
-      const int je = jb + kCsaRun < Nc ? jb + kCsaRun : Nc;
-      if (jb >= je) continue;
-      const int first = jb > 0 ? jb - 1 : 0;       // the block before the run feeds entry jb
-      Soft4 prev;
-      prev.reset();
-      walk_blocks<Tin, kPC>(kvp, gp, gsp, tpr, (long long)first * m, je - first, m, [&](int k, const Soft4& st) {
-        const int j = first + k;
-        if (j >= jb) {
-          float o[4];
-          merge_out(prev, st, o);                  // entry 0: prev is empty
-          store_vec<4>(ob + (long long)j * D, o);
-        }
-        prev = st;
-      });
-    } else {
-      // block r, lanes split its m tokens
-      const int L = (m + nl - 1) / nl;
-      const int lo = l * L < m ? l * L : m;
-      const int hi = lo + L < m ? lo + L : m;
-      Soft4 part;
-      part.reset();
-      if (l < nl)
-        walk_blocks<Tin, kPC>(kvp, gp, gsp, tpr, (long long)r * m + lo, 1, hi - lo,
-                              [&](int, const Soft4& st) { part = st; });
-      if (l < nl) {
-        float* sp = s_part + ((long long)l * tpr + c) * 12;
+  prev.reset();
+  int blk = first, pos = 0;                                           // current block, rows of it folded
+  int k = 0;
+  bool ok = true;
+  for (; k < K; ++k) {
+    const int slot = k % kCmpStages;
+    ok = __syncthreads_and(tc::mbar_wait(full + slot, (k / kCmpStages) & 1));
+    if (!ok) break;
+    const Tin* kvs = reinterpret_cast<const Tin*>(smem + slot * 2 * tile_bytes) + c;
+    const Tin* gs = reinterpret_cast<const Tin*>(smem + slot * 2 * tile_bytes + tile_bytes) + c;
+    const int r1 = rows - k * kCmpRows < kCmpRows ? rows - k * kCmpRows : kCmpRows;
+    for (int r = 0; r < r1;) {
+      int n = r1 - r < 4 ? r1 - r : 4;
+      n = m - pos < n ? m - pos : n;                                  // a chunk stays inside its block
+      if (has) fold_rows<Tin>(st, kvs, gs, D, r, n);
+      r += n;
+      pos += n;
+      if (pos == m) {                                                 // block `blk` complete
+        if (has && blk >= jb) {
+          float o[2];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) { sp[v] = part.m[v]; sp[4 + v] = part.s[v]; sp[8 + v] = part.a[v]; }
-      }
-      __syncthreads();
-      if (l == 0) {
-        Soft4 acc = part;
-        for (int q = 1; q < nl; ++q) {
-          const float* sp = s_part + ((long long)q * tpr + c) * 12;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float M = fmaxf(acc.m[v], sp[v]);
-            if (M == -INFINITY) continue;          // both empty
-            const float fa = __expf(acc.m[v] - M), fb = __expf(sp[v] - M);
-            acc.s[v] = acc.s[v] * fa + sp[4 + v] * fb;
-            acc.a[v] = acc.a[v] * fa + sp[8 + v] * fb;
-            acc.m[v] = M;
+          for (int v = 0; v < 2; ++v) {
+            if (kCSA) {                                               // entry 0: prev is empty
+              const float M = fmaxf(prev.m[v], st.m[v]);
+              const float fa = __expf(prev.m[v] - M), fb = __expf(st.m[v] - M);
+              o[v] = (prev.a[v] * fa + st.a[v] * fb) / (prev.s[v] * fa + st.s[v] * fb);
+            } else {
+              o[v] = st.a[v] / st.s[v];
+            }
           }
+          Tout* op = out + ((long long)b * Nc + blk) * D + c;
+          st_scalar(op, o[0]);
+          st_scalar(op + 1, o[1]);
         }
-        float o[4];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) o[v] = acc.a[v] / acc.s[v];
-        store_vec<4>(ob + (long long)r * D, o);
+        if (kCSA) prev = st;
+        st.reset();
+        pos = 0;
+        ++blk;
       }
-      __syncthreads();                             // s_part is reused by the next unit
     }
+    __syncthreads();                                                  // every thread is done with the slot
+    if (tid == 0 && k + kCmpStages < K) issue(k + kCmpStages);
+  }
+  if (!ok && tid == 0) {
+    // copies in flight (stages k .. the last issued) land before the CTA leaves
+    const int last = K - 1 < k + kCmpStages - 1 ? K - 1 : k + kCmpStages - 1;
+    for (int q = k; q <= last; ++q) tc::mbar_wait(full + q % kCmpStages, (q / kCmpStages) & 1);
   }
 }
 
-// Whole-sequence CSA (window 2m) or HCA (window m) compression without
-// RMSNorm on the streaming kernel.  Returns false when the shape needs the
-// per-entry kernel (D not a multiple of 4 or wider than 4 x 256 channels).
+// Whole-sequence CSA (window 2m) or HCA (window m) compression with
+// per-channel gates and no RMSNorm on the bulk-copy kernel.  Returns false
+// when the shape does not fit it (odd D, more than 1024 channel pairs, or a
+// stage ring above 200 KB of shared memory).
 template <typename Tin, typename Tout>
-static bool launch_compress_stream(const void* kv, const void* gate, int per_channel, int B, int T, int D, int m,
-                                   int window, void* out, cudaStream_t st, cudaError_t* err) {
-  const int tpr = D / 4;
-  if (D % 4 != 0 || tpr > kStreamThreads || (window != m && window != 2 * m)) return false;
+static bool launch_compress_bulk(const void* kv, const void* gate, int B, int T, int D, int m, int window,
+                                 void* out, cudaStream_t st, cudaError_t* err) {
+  if ((D & 1) || D / 2 > 1024 || (window != m && window != 2 * m)) return false;
   const int Nc = T / m;
-  const int nl = kStreamThreads / tpr;
-  const bool csa = window == 2 * m;
-  const int ups = csa ? (Nc + nl * kCsaRun - 1) / (nl * kCsaRun) : Nc;
-  const long long n_units = (long long)B * ups;
-  const long long cap = 2LL * sm_count();
-  const int grid = (int)(n_units < cap ? n_units : cap);
-  const size_t smem = csa ? 0 : (size_t)nl * tpr * 12 * sizeof(float);
-  const int threads = nl * tpr;
+  // about two CTAs per SM, each a contiguous range of blocks of one sequence
+  const int want = (2 * sm_count() + B - 1) / B;
+  int ups = Nc < want ? Nc : want;
+  const int bpu = (Nc + ups - 1) / ups;
+  ups = (Nc + bpu - 1) / bpu;
+  const size_t smem = 128 + (size_t)kCmpStages * 2 * kCmpRows * D * sizeof(Tin) + kCmpStages * 8;
+  if (smem > 200 * 1024) return false;
+  int threads = ((D / 2 + 31) / 32) * 32;
+  auto kern = window == 2 * m ? compress_bulk_kernel<Tin, Tout, true> : compress_bulk_kernel<Tin, Tout, false>;
+  *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (*err != cudaSuccess) return true;
   count_launch();
-  if (csa) {
-    if (per_channel)
-      compress_stream_kernel<Tin, Tout, true, true><<<grid, threads, 0, st>>>(
-          (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, Nc, ups, n_units);
-    else
-      compress_stream_kernel<Tin, Tout, false, true><<<grid, threads, 0, st>>>(
-          (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, Nc, ups, n_units);
-  } else {
-    if (per_channel)
-      compress_stream_kernel<Tin, Tout, true, false><<<grid, threads, smem, st>>>(
-          (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, Nc, ups, n_units);
-    else
-      compress_stream_kernel<Tin, Tout, false, false><<<grid, threads, smem, st>>>(
-          (const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, Nc, ups, n_units);
-  }
+  kern<<<B * ups, threads, smem, st>>>((const Tin*)kv, (const Tin*)gate, (Tout*)out, T, D, m, Nc, bpu, ups);
   *err = cudaGetLastError();
   return true;
 }
@@ -357,9 +296,9 @@ static cudaError_t launch_compress_t(const void* kv, const void* gate, int per_c
   const int Nc = n_entries >= 0 ? n_entries : T / m;
   if (out_rows < 0) out_rows = Nc;
   if (Nc == 0 || B == 0) return cudaSuccess;
-  if (rms_w == nullptr && j0 == 0 && n_entries < 0 && kv_pos0 == 0) {
+  if (per_channel && rms_w == nullptr && j0 == 0 && n_entries < 0 && kv_pos0 == 0) {
     cudaError_t e;
-    if (launch_compress_stream<Tin, Tout>(kv, gate, per_channel, B, T, D, m, window, out, st, &e)) return e;
+    if (launch_compress_bulk<Tin, Tout>(kv, gate, B, T, D, m, window, out, st, &e)) return e;
   }
   const int tpe = D / V;
   int epb = 256 / tpe;

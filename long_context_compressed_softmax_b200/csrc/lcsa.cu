@@ -68,7 +68,8 @@ lcsa_status check_indexer(const lcsa_indexer_args* a) {
   return LCSA_OK;
 }
 
-lcsa_status check_attn(const lcsa_attn_args* a, int sparse) {
+// need_ckv = 0: the entries come from elsewhere (the FP8 cache), ckv is not read.
+lcsa_status check_attn(const lcsa_attn_args* a, int sparse, int need_ckv = 1) {
   if (!a) return LCSA_ERR_INVALID_ARG;
   if (!valid_dtype(a->dtype) || !valid_dtype(a->out_dtype)) return LCSA_ERR_INVALID_ARG;
   if (a->B < 0 || a->Tq < 0 || a->H <= 0 || a->D <= 0 || a->R < 0 || a->R > a->D || (a->R & 1) ||
@@ -79,10 +80,10 @@ lcsa_status check_attn(const lcsa_attn_args* a, int sparse) {
   if ((long long)a->B * a->Tq == 0) return LCSA_OK;
   if ((a->D * esize(a->dtype)) % 16 != 0) return LCSA_ERR_INVALID_ARG;
   if (!a->q || !a->out) return LCSA_ERR_INVALID_ARG;
-  if (a->Nc > 0 && !a->ckv) return LCSA_ERR_INVALID_ARG;
+  if (need_ckv && a->Nc > 0 && !a->ckv) return LCSA_ERR_INVALID_ARG;
   if (a->Tkv > 0 && !a->kv) return LCSA_ERR_INVALID_ARG;
   if (sparse && !a->idx) return LCSA_ERR_INVALID_ARG;
-  if (!aligned16(a->q) || !aligned16(a->out) || (a->ckv && !aligned16(a->ckv)) ||
+  if (!aligned16(a->q) || !aligned16(a->out) || (need_ckv && a->ckv && !aligned16(a->ckv)) ||
       (a->kv && !aligned16(a->kv)) || (sparse && !aligned16(a->idx)) || (a->lse && !aligned16(a->lse)) ||
       (a->sink && (reinterpret_cast<uintptr_t>(a->sink) & 3u)))
     return LCSA_ERR_INVALID_ARG;
@@ -459,6 +460,44 @@ lcsa_status lcsa_csa_sparse_attn(const lcsa_attn_args* a, void* ws, size_t ws_by
 
 lcsa_status lcsa_hca_dense_attn(const lcsa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
   return attn_common(a, 0, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------ FP8 entry cache
+lcsa_status lcsa_quantize_entries_fp8(const void* x, int64_t rows, int D, int R, lcsa_dtype dtype, uint8_t* codes,
+                                      uint8_t* scales, void* rope, void* stream) {
+  if (!valid_dtype(dtype) || rows < 0 || D <= 0 || R < 0 || R >= D || (R & 1)) return LCSA_ERR_INVALID_ARG;
+  if (rows == 0) return LCSA_OK;
+  if (!x || !codes || !scales || (R > 0 && !rope)) return LCSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) % esize(dtype) != 0 || (reinterpret_cast<uintptr_t>(rope) & 1u))
+    return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  return from_cuda(launch_quantize_entries_fp8(x, rows, D, R, dtype, codes, scales, rope, (cudaStream_t)stream));
+}
+
+static lcsa_status attn_fp8_common(const lcsa_attn_args* a, const lcsa_fp8_entries* f8, int sparse, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  lcsa_status s = check_attn(a, sparse, 0);
+  if (s != LCSA_OK) return s;
+  if (!f8) return LCSA_ERR_INVALID_ARG;
+  if (!attn_tc_supported(a)) return LCSA_ERR_UNSUPPORTED;
+  if ((long long)a->B * a->Tq == 0) return LCSA_OK;
+  if (a->Nc > 0 && (!f8->codes || !f8->scales || !f8->rope || !aligned16(f8->codes) || !aligned16(f8->rope)))
+    return LCSA_ERR_INVALID_ARG;
+  if (!have_device()) return LCSA_ERR_CUDA;
+  const size_t need = attn_tc_workspace(a, sparse);
+  if (need > 0 && (!ws || ws_bytes < need)) return LCSA_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return LCSA_ERR_INVALID_ARG;
+  return from_cuda(launch_attn_tc(a, sparse, ws, (cudaStream_t)stream, f8));
+}
+
+lcsa_status lcsa_csa_sparse_attn_fp8(const lcsa_attn_args* a, const lcsa_fp8_entries* e, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  return attn_fp8_common(a, e, 1, ws, ws_bytes, stream);
+}
+
+lcsa_status lcsa_hca_dense_attn_fp8(const lcsa_attn_args* a, const lcsa_fp8_entries* e, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  return attn_fp8_common(a, e, 0, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -46,7 +46,8 @@ def test_struct_layouts_match_header(lcsa, tmp_path):
     import subprocess
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "lcsa.h"', 'int main(void){']
     structs = (("lcsa_indexer_args", lcsa.IndexerArgs), ("lcsa_attn_args", lcsa.AttnArgs),
-               ("lcsa_indexer_mxfp4_args", lcsa.IndexerMxfp4Args), ("lcsa_out_proj_args", lcsa.OutProjArgs))
+               ("lcsa_indexer_mxfp4_args", lcsa.IndexerMxfp4Args), ("lcsa_out_proj_args", lcsa.OutProjArgs),
+               ("lcsa_fp8_entries", lcsa.Fp8Entries))
     for cname, py in structs:
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in py._fields_:
@@ -196,3 +197,28 @@ def test_noalloc_validates_like_the_workspace_call(lcsa):
     if not torch.cuda.is_available():
         a.Nc = 8388544
         assert L.lcsa_indexer_topk_noalloc(ctypes.byref(a), None) == 4     # fits; no device: no CPU path
+
+
+def test_fp8_cache_calls_check_arguments(lcsa):
+    L = lcsa.lib
+    x, c, sc, r = (ctypes.c_void_p(v) for v in (0x1000, 0x2000, 0x3000, 0x4000))
+    assert L.lcsa_quantize_entries_fp8(x, 4, 512, 63, lcsa.LCSA_BF16, c, sc, r, None) == 1     # odd R
+    assert L.lcsa_quantize_entries_fp8(x, 4, 512, 512, lcsa.LCSA_BF16, c, sc, r, None) == 1    # R = D
+    assert L.lcsa_quantize_entries_fp8(None, 4, 512, 64, lcsa.LCSA_BF16, c, sc, r, None) == 1  # null input
+    assert L.lcsa_quantize_entries_fp8(ctypes.c_void_p(0x1001), 4, 512, 64, lcsa.LCSA_BF16, c, sc, r, None) == 1
+    assert L.lcsa_quantize_entries_fp8(None, 0, 512, 64, lcsa.LCSA_BF16, None, None, None, None) == 0
+    a = lcsa.AttnArgs()
+    a.q, a.out, a.kv, a.idx = 0x10000, 0x20000, 0x30000, 0x40000
+    a.B, a.Tq, a.H, a.D, a.R, a.Nc, a.k, a.Tkv, a.m, a.W = 1, 1, 64, 512, 64, 8, 8, 8, 4, 8
+    a.dtype = a.out_dtype = lcsa.LCSA_BF16
+    e = lcsa.Fp8Entries(0x50000, 0x60000, 0x70000)
+    assert L.lcsa_csa_sparse_attn_fp8(ctypes.byref(a), None, None, 0, None) == 1          # no cache
+    e.codes = 0x50008
+    assert L.lcsa_csa_sparse_attn_fp8(ctypes.byref(a), ctypes.byref(e), None, 0, None) == 1   # misaligned codes
+    e.codes = 0x50000
+    a.H = 16
+    assert L.lcsa_hca_dense_attn_fp8(ctypes.byref(a), ctypes.byref(e), None, 0, None) == 2    # not the layer shape
+    a.H = 64
+    if not torch.cuda.is_available():
+        ws = ctypes.c_void_p(0x100000)
+        assert L.lcsa_hca_dense_attn_fp8(ctypes.byref(a), ctypes.byref(e), ws, 1 << 30, None) == 4   # no CPU path

@@ -507,3 +507,32 @@ def test_layer_shapes_use_tensor_cores(lcsa):
 def test_device_status_clean(lcsa):
     torch.cuda.synchronize()
     assert lcsa.get_device_status() == 0
+
+
+def test_bad_index_is_skipped_and_flagged(lcsa):
+    """Every use of a selected index is checked before an address is formed:
+    an index >= Nc is skipped (its slot is no key at all) and the device
+    status reports LCSA_DEV_BAD_INDEX (2), read and cleared by the host; the
+    next call on the same stream is clean.  Tensor-core shapes and the FP32
+    CUDA-core kernel, with a row whose selection is entirely bad."""
+    for dtype, H, D, R, k, Nc, q_pos0 in (("bf16", 64, 512, 64, 64, 500, 2400), ("fp32", 4, 64, 32, 16, 200, 900)):
+        B, Tq, m, W = 1, 3, 4, 16
+        x = _attn_case(B, Tq, H, D, Nc, q_pos0 + Tq, dtype, seed=96)
+        nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+        idx = gen.make_topk_idx(B, Tq, k, nv, seed=97, device=DEV)
+        assert lcsa.get_device_status() == 0
+        bad = idx.clone()
+        bad[0, 1, k - 1] = Nc + 7                      # last slot of row 1 points past the cache
+        bad[0, 2, :] = Nc                              # every slot of row 2 (window and sink remain)
+        out = lcsa.csa_sparse_attn(x["q"], x["ckv"], bad, x["kv"], x["sink"], q_pos0, 0, m, W, R)
+        assert lcsa.get_device_status() == 2
+        assert lcsa.get_device_status() == 0            # read and cleared
+        sel = bad.cpu().numpy().copy()
+        sel[sel >= Nc] = -1                             # the skipped slots are no keys
+        ref, _ = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), sel, np64(x["kv"]), q_pos0, 0, m, W, _sink(x), R)
+        assert_attn_close(np64(out).reshape(ref.shape), ref)
+        out2 = lcsa.csa_sparse_attn(x["q"], x["ckv"], idx, x["kv"], x["sink"], q_pos0, 0, m, W, R)
+        assert lcsa.get_device_status() == 0
+        ref2, _ = O.csa_sparse_attn(np64(x["q"]), np64(x["ckv"]), idx.cpu().numpy(), np64(x["kv"]), q_pos0, 0, m, W,
+                                    _sink(x), R)
+        assert_attn_close(np64(out2).reshape(ref2.shape), ref2)
