@@ -476,8 +476,11 @@ def quantize_entries_fp8(ckv, R):
     return codes, (X + 127).astype(np.uint8), _round_bf16(rope)
 
 
+E4M3_ALL = np.array([e4m3_value(c) for c in range(256)])     # value of every code, by e4m3_value
+
+
 def dequantize_entries_fp8(codes, scales, rope):
     """Exact FP64 entries from the FP8 cache: E4M3 value * 2^X, rotary dims as stored."""
-    vals = np.vectorize(e4m3_value, otypes=[np.float64])(np.asarray(codes))
+    vals = E4M3_ALL[np.asarray(codes, dtype=np.uint8)]
     X = np.asarray(scales, dtype=np.float64) - 127.0
     return np.concatenate([vals * np.exp2(X)[..., None], np.asarray(rope, dtype=np.float64)], axis=-1)
