@@ -659,7 +659,44 @@ def run_decode(args, cfg, lcsa, dev, rank, bus_id, peaks, world):
         "clocks": clocks4,
         "note": "indexer keys as MXFP4 (64 code bytes + 4 scale bytes per entry), queries quantised per head; "
                 "recall = share of the BF16-key selection kept"}
-    del ix, ckv, q, kvw, idx, out, ws_ix, ws_at, kc, ks, idx4, ws_ix4
+    # The FP8 entry cache (E4M3 body + scale byte + BF16 rotary dims per entry,
+    # written once as a cache is): the same decode step with the attention
+    # gathering FP8 rows.
+    cache = lcsa.quantize_entries_fp8(ckv, cfg.R)
+    ev8 = []
+
+    def step8(record=False):
+        a = torch.cuda.Event(enable_timing=True) if record else None
+        if a:
+            a.record()
+        lcsa.indexer_topk(ix["q_idx"], ix["w"], ix["k_idx"], t, cfg.m, cfg.k, workspace=ws_ix, idx_out=idx)
+        b = torch.cuda.Event(enable_timing=True) if record else None
+        if b:
+            b.record()
+        lcsa.csa_sparse_attn_fp8(q, cache, idx, kvw, sink, t, t - cfg.W + 1, cfg.m, cfg.W, cfg.R, out=out,
+                                 workspace=ws_at)
+        if record:
+            c = torch.cuda.Event(enable_timing=True)
+            c.record()
+            ev8.append((a, b, c))
+
+    ms8, clocks8 = timed(lambda: step8(True), args.steps * 4, args.warmup, bus_id)
+    ms8 = max_over_ranks(ms8)
+    row8 = (cfg.D - cfg.R) + 1 + cfg.R * 2
+    byts8 = byts - B * cfg.k * cfg.D * 2 + B * cfg.k * row8
+    gbs8 = byts8 / (ms8 / 1e3) / 1e9
+    at8 = statistics.mean(b.elapsed_time(c) for _, b, c in ev8)
+    res["fp8_cache"] = {
+        "value": weak_scaling_throughput(B, ms8 / 1e3, world), "unit": "queries/s", "ms_per_step": ms8,
+        "indexer_topk_ms": statistics.mean(a.elapsed_time(b) for a, b, _ in ev8), "csa_sparse_attn_ms": at8,
+        "entry_bytes": row8, "cache_bytes": int(B * Nc * row8),
+        "roofline": {"bound": "hbm", "achieved": round(gbs8, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs8 / peaks["hbm_gbs"], 4), "bytes_per_step": byts8,
+                     "peak_source": f"hbm_gbs of {peaks['source']}"},
+        "clocks": clocks8,
+        "note": "entries as FP8 E4M3 (448 B) + scale byte + BF16 rotary dims (128 B) = 577 B against 1024; "
+                "BF16 indexer keys; attention expands the gathered rows to BF16 in shared memory"}
+    del ix, ckv, q, kvw, idx, out, ws_ix, ws_at, kc, ks, idx4, ws_ix4, cache
     torch.cuda.empty_cache()
     return res
 

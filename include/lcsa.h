@@ -76,6 +76,23 @@ uint64_t lcsa_kernel_launches(void);
  * (LCSA_DEV_*) and clears it.  Returns LCSA_ERR_DEVICE when *code != 0. */
 lcsa_status lcsa_get_device_status(void* stream, int* code);
 
+/* Limit of every bounded wait (an mbarrier or a pipeline hand-off) in the
+ * library's kernels on the current device, in nanoseconds of the GPU's global
+ * timer: a wait that lasts longer gives up, the kernel records
+ * LCSA_DEV_TIMEOUT, stops issuing work, lets its copies in flight land, frees
+ * its tensor memory and returns, so the context stays usable.  Default 2 s;
+ * ns = 0 restores it.  A synchronous copy to the device: call it outside
+ * stream capture, with no library kernel running on the device. */
+lcsa_status lcsa_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook of the bounded waits: the next launch of the grouped output
+ * projection's GEMM kernel (lcsa_grouped_out_proj's first GEMM) leaves the
+ * pipeline stage of k-chunk `chunk` of its first CTA unfilled (no copy, no
+ * arrival), so every wait on that stage runs out.  The call then returns,
+ * lcsa_get_device_status reports LCSA_DEV_TIMEOUT and the output is
+ * undefined; later calls are unaffected.  chunk < 0 clears a pending hook. */
+void lcsa_test_withhold_stage(int chunk);
+
 /* ------------------------------------------------------------------------
  * KV compression ([p2] CSA Step 1: m consecutive tokens merged into one entry
  * with learned softmax weights; [p2] HCA: m' = 128 tokens per entry; [p3]

@@ -35,6 +35,7 @@ EXPORTED = [
     "lcsa_grouped_out_proj_workspace", "lcsa_grouped_out_proj",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
     "lcsa_quantize_entries_fp8", "lcsa_csa_sparse_attn_fp8", "lcsa_hca_dense_attn_fp8",
+    "lcsa_set_wait_limit_ns", "lcsa_test_withhold_stage",
 ]
 
 
@@ -113,6 +114,8 @@ _sig = {
     "lcsa_hca_dense_attn": (_i, [ctypes.POINTER(AttnArgs), _vp, _sz, _vp]),
     "lcsa_attn_uses_tensor_cores": (_i, [ctypes.POINTER(AttnArgs)]),
     "lcsa_quantize_entries_fp8": (_i, [_vp, _i64, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "lcsa_set_wait_limit_ns": (_i, [ctypes.c_uint64]),
+    "lcsa_test_withhold_stage": (None, [_i]),
     "lcsa_csa_sparse_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
 }
@@ -162,6 +165,11 @@ def version() -> str:
 def kernel_launches() -> int:
     """Kernels the library has launched in this process so far."""
     return int(_lib.lcsa_kernel_launches())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit of the kernels' bounded waits on the current device (0 = the 2 s default)."""
+    _check(_lib.lcsa_set_wait_limit_ns(int(ns)), "set_wait_limit_ns")
 
 
 def get_device_status() -> int:

@@ -657,7 +657,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           } else {
             const uint64_t now = tc::globaltimer();
             if (t_idle == 0) t_idle = now;
-            else if (now - t_idle > tc::kWaitLimitNs) { report(LCSA_DEV_TIMEOUT); ok = false; break; }
+            else if (now - t_idle > tc::wait_limit()) { report(LCSA_DEV_TIMEOUT); ok = false; break; }
           }
         }
         slot += x.n_tiles;

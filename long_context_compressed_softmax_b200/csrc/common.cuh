@@ -16,6 +16,11 @@ namespace lcsa {
 // ---------------------------------------------------------------------------
 __device__ int g_status;
 
+// Limit of every bounded wait in the library's kernels (ns of %globaltimer);
+// lcsa_set_wait_limit_ns changes it per device.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;   // 2 s
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
 __device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
 
 // Host-side count of kernel launches issued by the library.

@@ -17,6 +17,8 @@
 // tile accumulates.  Every wait is bounded; on expiry the CTA stops, records
 // LCSA_DEV_TIMEOUT, drains its copies and frees TMEM.
 #pragma once
+#include <atomic>
+
 #include "tc_ptx.cuh"
 
 namespace lcsa {
@@ -28,11 +30,19 @@ constexpr uint32_t kGmABytes = kGmBM * kGmBK * 2;   // 16 KB
 constexpr uint32_t kGmBBytes = kGmBN * kGmBK * 2;   // 32 KB
 constexpr size_t kGmSmem = 1024 + kGmStages * (kGmABytes + kGmBBytes) + 128;
 
+// Test hook: the next launch's producer in CTA 0 skips the stage fill of this
+// k-chunk (no copy, no arrival), so every wait on it runs out (-1 = off).
+inline std::atomic<int>& gemm_withhold_next() {
+  static std::atomic<int> v{-1};
+  return v;
+}
+
 struct GmGeom {
   int M, N, K;          // per group
   int groups;
   int m_tiles, n_tiles;
   long long ldc;        // C row stride (elements)
+  int withhold;         // test hook: k-chunk whose stage CTA 0 never fills (-1 = none)
 };
 
 __global__ void __launch_bounds__(kGmThreads, 1)
@@ -47,6 +57,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
   uint64_t* empty = full + kGmStages;
   uint64_t* acc_full = empty + kGmStages;
   uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drained = acc_empty + 2;            // MMA issuer: its MMAs have completed (abort path)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -56,6 +67,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGmStages; ++s) { tc::mbar_init(full + s, 1); tc::mbar_init(empty + s, 1); }
     for (int a = 0; a < 2; ++a) { tc::mbar_init(acc_full + a, 1); tc::mbar_init(acc_empty + a, 4); }
+    tc::mbar_init(drained, 1);
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -89,6 +101,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
           const long long r = it / kGmStages;
           if (r > 0 && !tc::mbar_wait(empty + s, (uint32_t)((r - 1) & 1))) { ok = false; break; }
           if (*abort_flag) { ok = false; break; }
+          if (it == g.withhold && blockIdx.x == 0) continue;     // test hook: this stage never fills
           tc::mbar_arrive_expect_tx(full + s, kGmABytes + kGmBBytes);
           tc::tma_load_2d(s_a + s * kGmABytes, &a_map, full + s, grp * g.K + kc * kGmBK, mt * kGmBM);
           tc::tma_load_2d(s_b + s * kGmBBytes, &b_map, full + s, kc * kGmBK, grp * g.N + nt * kGmBN);
@@ -127,7 +140,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
         if (!ok) break;
         tc::mma_commit(acc_full + a);
       }
-      if (!ok) *abort_flag = 1;
+      if (!ok) {
+        *abort_flag = 1;
+        // the MMAs already issued finish before TMEM is freed
+        tc::mma_commit(drained);
+        tc::mbar_wait(drained, 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5)
@@ -191,6 +209,7 @@ static cudaError_t launch_gemm_bf16(const void* A, long long lda, const void* B,
   g.m_tiles = (M + kGmBM - 1) / kGmBM;
   g.n_tiles = (N + kGmBN - 1) / kGmBN;
   g.ldc = ldc;
+  g.withhold = gemm_withhold_next().exchange(-1);
   const long long tiles = (long long)groups * g.m_tiles * g.n_tiles;
   const int grid = (int)(tiles < sms ? tiles : sms);
   cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGmSmem);

@@ -242,6 +242,14 @@ lcsa_status lcsa_get_device_status(void* stream, int* code) {
   return v == 0 ? LCSA_OK : LCSA_ERR_DEVICE;
 }
 
+lcsa_status lcsa_set_wait_limit_ns(uint64_t ns) {
+  if (!have_device()) return LCSA_ERR_CUDA;
+  const unsigned long long v = ns ? (unsigned long long)ns : kDefaultWaitLimitNs;
+  return from_cuda(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+}
+
+void lcsa_test_withhold_stage(int chunk) { gemm_withhold_next().store(chunk < 0 ? -1 : chunk); }
+
 lcsa_status lcsa_csa_compress(const void* kv, const void* gate, int gate_per_channel, int B, int T, int D, int m,
                               lcsa_dtype dtype, const float* rms_weight, float rms_eps, void* out,
                               lcsa_dtype out_dtype, void* stream) {

@@ -50,9 +50,10 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up after ~kWaitLimitNs, records LCSA_DEV_TIMEOUT and
+// Bounded wait: gives up after the device's wait limit (g_wait_limit_ns, 2 s
+// unless lcsa_set_wait_limit_ns changed it), records LCSA_DEV_TIMEOUT and
 // returns false.  Callers then stop issuing work and leave the kernel.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+__device__ __forceinline__ uint64_t wait_limit() { return *(volatile unsigned long long*)&g_wait_limit_ns; }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -60,7 +61,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > wait_limit()) {
       report(LCSA_DEV_TIMEOUT);
       return false;
     }
@@ -89,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_test_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > wait_limit()) {
       report(LCSA_DEV_TIMEOUT);
       return false;
     }
@@ -104,7 +105,7 @@ __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity
   while (true) {
     __nanosleep(128);
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > wait_limit()) {
       report(LCSA_DEV_TIMEOUT);
       return false;
     }
