@@ -408,6 +408,22 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     const bool coll = g.sparse || g.fp8;
     bool bad = false;
     int slot = 0, ni = 0;
+    // CSA: the selected entries of the next item, loaded into registers while
+    // the current item's tiles are gathered (its first gather then starts as
+    // soon as a stage frees, without a dependent index load in front of it).
+    constexpr int kPer = (kAtMaxIdx + kAtProdThreads - 1) / kAtProdThreads;
+    int32_t e_pre[kPer];
+    int pre_it = -1;
+    auto load_idx = [&](const AtItem& y, int32_t* e_v) {
+      const int s0 = y.t0 * kAtKT;
+      const int32_t* idx_row = P.idx + y.row * g.k + s0;
+      const int hi = y.ks.n_c < (y.t0 + y.n_tiles) * kAtKT ? y.ks.n_c : (y.t0 + y.n_tiles) * kAtKT;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int e = tid + u * kAtProdThreads;
+        e_v[u] = e < hi - s0 ? __ldg(idx_row + e) : 0;
+      }
+    };
     int nc_next = at_item_nc(g, P, blockIdx.x);
     for (int it = blockIdx.x; it < g.n_items; it += G) {
       const int nc_cur = nc_next;
@@ -441,21 +457,30 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       const int slot0 = x.t0 * kAtKT;
       if (g.sparse) {
         // Every read of the previous item's s_idx precedes the barrier of its
-        // last gathered tile, which all producers have passed.
-        // All loads are issued before the first store: one memory round trip.
-        const int32_t* idx_row = P.idx + x.row * g.k + slot0;
+        // last gathered tile, which all producers have passed.  The entries
+        // come from the registers filled during the previous item (all loads
+        // issued before the first store when they were not prefetched).
         const int hi = x.ks.n_c < (x.t0 + x.n_tiles) * kAtKT ? x.ks.n_c : (x.t0 + x.n_tiles) * kAtKT;
-        constexpr int kPer = (kAtMaxIdx + kAtProdThreads - 1) / kAtProdThreads;
         int32_t e_v[kPer];
+        if (pre_it == it) {
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int e = tid + u * kAtProdThreads;
-          e_v[u] = e < hi - slot0 ? __ldg(idx_row + e) : 0;
+          for (int u = 0; u < kPer; ++u) e_v[u] = e_pre[u];
+        } else {
+          load_idx(x, e_v);
         }
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
           const int e = tid + u * kAtProdThreads;
           if (e < hi - slot0) s_idx[e] = e_v[u];
+        }
+        // the next item's entries, in flight during this item's gathers
+        pre_it = -1;
+        if (it + G < g.n_items) {
+          const AtItem y = at_item(g, it + G, nc_next);
+          if (y.n_tiles > 0) {
+            load_idx(y, e_pre);
+            pre_it = it + G;
+          }
         }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
       }

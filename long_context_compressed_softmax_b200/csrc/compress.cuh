@@ -107,8 +107,9 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
 // Streaming compressor for whole sequences (per-channel gates, window 2m or m,
 // no RMSNorm): token rows reach shared memory by bulk copies.
 //
-// A CTA owns a contiguous range of blocks (m tokens each) of one sequence and
-// streams their token rows, kCmpRows at a time, through a kCmpStages-deep ring:
+// A CTA (about four per SM) owns a contiguous range of blocks (m tokens each)
+// of one sequence and streams their token rows, kCmpRows at a time, through a
+// kCmpStages-deep ring:
 // one thread issues two cp.async.bulk copies per stage (kv rows, gate rows;
 // contiguous in HBM) that complete on the stage's mbarrier, so the bytes in
 // flight do not depend on registers or occupancy.  Each thread owns two
@@ -123,8 +124,8 @@ compress_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* 
 // all threads (__syncthreads_and), waits (bounded) for its copies in flight
 // and leaves.
 // ---------------------------------------------------------------------------
-constexpr int kCmpRows = 16;       // token rows per stage
-constexpr int kCmpStages = 3;
+constexpr int kCmpRows = 8;        // token rows per stage
+constexpr int kCmpStages = 3;      // 48 KB per CTA at D = 512: four CTAs per SM
 
 struct Soft2 {                     // softmax state of 2 channels
   float m[2], s[2], a[2];
@@ -166,6 +167,50 @@ __device__ __forceinline__ void fold_rows(Soft2& st, const Tin* kvs, const Tin* 
       }
     st.m[v] = cm; st.s[v] = sm; st.a[v] = a;
   }
+}
+
+// Fold rows r .. r+3 of a staged BF16 tile into st: the common chunk (4 rows
+// of one block).  The chunk maximum of both channels is one packed BF16 max
+// tree (exact), the weights are exp2(g log2e - m log2e) with one FFMA each.
+__device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
+                                           int r) {
+  __nv_bfloat162 x[4], g[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    x[u] = *reinterpret_cast<const __nv_bfloat162*>(kvs + (r + u) * D);
+    g[u] = *reinterpret_cast<const __nv_bfloat162*>(gs + (r + u) * D);
+  }
+  const float2 gm = __bfloat1622float2(__hmax2(__hmax2(g[0], g[1]), __hmax2(g[2], g[3])));
+  constexpr float kL2e = 1.4426950408889634f;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const float cm = fmaxf(st.m[v], v ? gm.y : gm.x);
+    const float ncml = -cm * kL2e;
+    const float alpha = exp2f(fmaf(st.m[v], kL2e, ncml));     // 0 while the state is empty
+    float p[4], xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 gf = __bfloat1622float2(g[u]);
+      const float2 xf = __bfloat1622float2(x[u]);
+      p[u] = exp2f(fmaf(v ? gf.y : gf.x, kL2e, ncml));
+      xv[u] = v ? xf.y : xf.x;
+    }
+    st.s[v] = fmaf(st.s[v], alpha, (p[0] + p[1]) + (p[2] + p[3]));
+    st.a[v] = fmaf(st.a[v], alpha, fmaf(p[0], xv[0], p[1] * xv[1]) + fmaf(p[2], xv[2], p[3] * xv[3]));
+    st.m[v] = cm;
+  }
+}
+__device__ __forceinline__ void fold4(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D, int r) {
+  fold4_bf16(st, kvs, gs, D, r);
+}
+__device__ __forceinline__ void fold4(Soft2& st, const float* kvs, const float* gs, int D, int r) {
+  fold_rows<float>(st, kvs, gs, D, r, 4);
+}
+
+// Two output channels in one store.
+__device__ __forceinline__ void st_pair(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+__device__ __forceinline__ void st_pair(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
 template <typename Tin, typename Tout, bool kCSA>
@@ -225,7 +270,10 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
     for (int r = 0; r < r1;) {
       int n = r1 - r < 4 ? r1 - r : 4;
       n = m - pos < n ? m - pos : n;                                  // a chunk stays inside its block
-      if (has) fold_rows<Tin>(st, kvs, gs, D, r, n);
+      if (has) {
+        if (n == 4) fold4(st, kvs, gs, D, r);
+        else fold_rows<Tin>(st, kvs, gs, D, r, n);
+      }
       r += n;
       pos += n;
       if (pos == m) {                                                 // block `blk` complete
@@ -241,9 +289,7 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
               o[v] = st.a[v] / st.s[v];
             }
           }
-          Tout* op = out + ((long long)b * Nc + blk) * D + c;
-          st_scalar(op, o[0]);
-          st_scalar(op + 1, o[1]);
+          st_pair(out + ((long long)b * Nc + blk) * D + c, o[0], o[1]);
         }
         if (kCSA) prev = st;
         st.reset();
@@ -270,8 +316,8 @@ static bool launch_compress_bulk(const void* kv, const void* gate, int B, int T,
                                  void* out, cudaStream_t st, cudaError_t* err) {
   if ((D & 1) || D / 2 > 1024 || (window != m && window != 2 * m)) return false;
   const int Nc = T / m;
-  // about two CTAs per SM, each a contiguous range of blocks of one sequence
-  const int want = (2 * sm_count() + B - 1) / B;
+  // about four CTAs per SM, each a contiguous range of blocks of one sequence
+  const int want = (4 * sm_count() + B - 1) / B;
   int ups = Nc < want ? Nc : want;
   const int bpu = (Nc + ups - 1) / ups;
   ups = (Nc + bpu - 1) / bpu;
