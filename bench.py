@@ -170,10 +170,21 @@ class Layer:
 
 
 class StackRunner:
-    """Runs the layers through the library with per-call CUDA events."""
+    """Runs the layers through the library with per-call CUDA events.
+    fp8_entries: CSA layers quantise their entries to the FP8 cache (one call
+    after the compression) and attend over it."""
 
-    def __init__(self, lcsa, cfg, layers, dev):
+    def __init__(self, lcsa, cfg, layers, dev, fp8_entries=False):
         self.lcsa, self.cfg, self.layers = lcsa, cfg, layers
+        self.fp8 = fp8_entries
+        self.cache = {}
+        if fp8_entries:
+            for L in layers:
+                if L.kind == "csa":
+                    B, Nc = L.ckv.shape[:2]
+                    self.cache[id(L)] = (torch.empty((B, Nc, cfg.D - cfg.R), dtype=torch.uint8, device=dev),
+                                         torch.empty((B, Nc), dtype=torch.uint8, device=dev),
+                                         torch.empty((B, Nc, cfg.R), dtype=torch.bfloat16, device=dev))
         B, T = cfg.B, cfg.T
         self.out = torch.empty((B, T, cfg.H, cfg.D), dtype=torch.bfloat16, device=dev)
         self.idx = torch.empty((B, T, cfg.k), dtype=torch.int32, device=dev) if any(
@@ -208,8 +219,14 @@ class StackRunner:
             self._call(li, "csa_compress", lambda: lc.csa_compress(L.kv, L.gate, L.m, out=L.ckv))
             self._call(li, "indexer_topk", lambda: lc.indexer_topk(L.q_idx, L.w, L.k_idx, 0, L.m, c.k,
                                                                    workspace=self.ws, idx_out=self.idx))
-            self._call(li, "csa_sparse_attn", lambda: lc.csa_sparse_attn(
-                L.q, L.ckv, self.idx, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
+            if self.fp8:
+                cc = self.cache[id(L)]
+                self._call(li, "quantize_entries_fp8", lambda: lc.quantize_entries_fp8(L.ckv, c.R, *cc))
+                self._call(li, "csa_sparse_attn", lambda: lc.csa_sparse_attn_fp8(
+                    L.q, cc, self.idx, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
+            else:
+                self._call(li, "csa_sparse_attn", lambda: lc.csa_sparse_attn(
+                    L.q, L.ckv, self.idx, L.kv, L.sink, 0, 0, L.m, c.W, c.R, out=self.out, workspace=self.ws))
         elif L.kind == "hca":
             self._call(li, "hca_compress", lambda: lc.hca_compress(L.kv, L.gate, L.m, out=L.ckv))
             self._call(li, "hca_dense_attn", lambda: lc.hca_dense_attn(
@@ -374,7 +391,7 @@ def run_reference(args, cfg, world, rank):
 # ----------------------------------------------------------------------------- GPU arm
 def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     layers = [Layer(kind, cfg, rank_seed(cfg.seed * 10 + li, rank), dev) for li, kind in enumerate(cfg.layers)]
-    runner = StackRunner(lcsa, cfg, layers, dev)
+    runner = StackRunner(lcsa, cfg, layers, dev, fp8_entries=args.fp8_entries)
     n0 = lcsa.kernel_launches()
     runner.step()
     torch.cuda.synchronize()
@@ -470,7 +487,7 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)-scaled BF16 inputs, independent per layer and rank)",
-            "config": config_obj(cfg, world),
+            "config": config_obj(cfg, world) | ({"csa_entries": "fp8 cache"} if args.fp8_entries else {}),
             "layer_ms": layer_ms, "kernels": summary, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
     if out_proj is not None:
@@ -794,6 +811,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-out-proj", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-entries", action="store_true",
+                    help="CSA layers attend over the FP8 entry cache (quantised after compression, in the step)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
