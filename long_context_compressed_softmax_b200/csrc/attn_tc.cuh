@@ -63,7 +63,7 @@ constexpr uint32_t kAtOffStats = kAtOffCs + (kAtStages + 2) * kAtCsBytes;   // [
 constexpr uint32_t kAtOffScl = kAtOffStats + 2 * 64 * 8;             // [kAtStages][64] FP8 entry scales
 constexpr uint32_t kAtOffKm = kAtOffScl + kAtStages * kAtKT * 4;        // [kAtStages][2] valid-row masks
 constexpr uint32_t kAtOffBar = kAtOffKm + 32;
-constexpr int kAtBars = 21;
+constexpr int kAtBars = 22;
 constexpr size_t kAtSmem = 1024 + kAtOffBar + kAtBars * 8;
 static_assert(kAtSmem <= 232448, "attention shared memory exceeds 227 KB");
 constexpr int kAtCodeBytes = 448;               // FP8 entry cache: E4M3 bytes of dims 0..447 per entry
@@ -251,15 +251,32 @@ __device__ __forceinline__ void store32_v8(__nv_bfloat16* p, const float* o) {
   }
 }
 
+// 16 consecutive FP32 values given as bit patterns, as 32-byte stores (p 32-byte aligned).
+__device__ __forceinline__ void store16_v8_bits(float* p, const uint32_t* v) {
+  st_v8(p, v);
+  st_v8(p + 8, v + 8);
+}
+__device__ __forceinline__ void store16_v8_bits(__nv_bfloat16* p, const uint32_t* v) {
+  uint32_t w[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+    w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  st_v8(p, w);
+}
+
 // Epilogue of one item, executed by the 128 transition threads.  Row
 // statistics come from the softmax warps through shared memory; O -> sink,
 // normalisation, -t rotation of the rotary block -> output (or split
-// partials) straight from registers.  Chunk k covers dims 64k .. 64k+63:
-// thread (h % 16) takes dims 64k .. +31 and thread (h % 16) + 16 dims
-// 64k+32 .. +63 (16x32bx2 with a 32-column offset), so each warp store
-// instruction writes 16 rows x 2 adjacent 16-byte pieces.  The o_free
-// arrival follows the last TMEM read.
-__device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done, uint64_t* o_free,
+// partials) straight from registers.  Piece k covers dims 32k .. 32k+31:
+// thread (h % 16) takes dims 32k .. +15 and thread (h % 16) + 16 dims
+// 32k+16 .. +31 (16x32bx2 with a 16-column offset), so each warp store
+// instruction writes 16 rows x 2 adjacent 32-byte pieces (BF16).  The TMEM
+// read of piece k+1 is in flight while piece k is scaled and stored;
+// o_free[0] (dims 0-255, the first PV half of the next item) is arrived on
+// after piece 7's read, o_free[1] after piece 15's.
+__device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done, uint64_t* o_free /*[2]*/,
                             uint64_t* stats_full, const float2* stats, int item, const float2* cs, long long row,
                             int split, int last, uint32_t tmem, uint32_t lane_base, int h, int half, int xt, bool ok) {
   const int lane = xt & 31;
@@ -291,35 +308,45 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
                              : (g.out_bf16 ? nullptr : reinterpret_cast<float*>(P.out) + orow * 512);
   __nv_bfloat16* obf = (g.splits == 1 && g.out_bf16) ? reinterpret_cast<__nv_bfloat16*>(P.out) + orow * 512 : nullptr;
   const uint32_t taddr = tmem + lane_base + kTmO;
-#pragma unroll 1
-  for (int k = 0; k < 8; ++k) {
-    uint32_t v[32];
-    tc::tmem_ld_16x32bx2_x32<32>(taddr + k * 64, v);
-    tc::tmem_wait_ld();
-    if (k == 7) {
+  // piece k (0..15) = O columns 32k .. 32k+31: thread (h % 16) dims 32k .. +15,
+  // thread (h % 16) + 16 dims 32k+16 .. +31 (16x32bx2 with a 16-column offset)
+  uint32_t buf[2][16];
+  tc::tmem_ld_16x32bx2_x16<16>(taddr, buf[0]);
+#pragma unroll 2
+  for (int k = 0; k < 16; ++k) {
+    uint32_t* v = buf[k & 1];
+    tc::tmem_wait_ld_regs16(v);
+    if (k + 1 < 16) tc::tmem_ld_16x32bx2_x16<16>(taddr + (k + 1) * 32, buf[(k + 1) & 1]);
+    if (k == 7 || k == 15) {
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(o_free);          // O may be overwritten by the next item's PV
+      if (lane == 0) tc::mbar_arrive(o_free + (k == 15 ? 1 : 0));  // that half of O may be overwritten
     }
-    const int d0 = k * 64 + half * 32;                 // first output dim of this thread's piece
-    float o[32];
+    const int d0 = k * 32 + half * 16;                 // first output dim of this thread's piece
+    // scaled in place (FP32 bit patterns in v)
 #pragma unroll
-    for (int q2 = 0; q2 < 32; ++q2) o[q2] = __uint_as_float(v[q2]) * scale_out;
-    if (k == 7 && g.splits == 1) {
+    for (int q2 = 0; q2 < 16; ++q2) v[q2] = __float_as_uint(__uint_as_float(v[q2]) * scale_out);
+    if (k >= 14 && g.splits == 1) {
 #pragma unroll
-      for (int q2 = 0; q2 < 32; q2 += 2) {
-        const float2 e = cs[half * 16 + (q2 >> 1)];    // rotate by -t: (cos, -sin)
-        const float a0 = o[q2], a1 = o[q2 + 1];
-        o[q2] = a0 * e.x + a1 * e.y;
-        o[q2 + 1] = -a0 * e.y + a1 * e.x;
+      for (int q2 = 0; q2 < 16; q2 += 2) {
+        const float2 e = cs[(d0 - 448 + q2) >> 1];      // rotate by -t: (cos, -sin)
+        const float a0 = __uint_as_float(v[q2]), a1 = __uint_as_float(v[q2 + 1]);
+        v[q2] = __float_as_uint(a0 * e.x + a1 * e.y);
+        v[q2 + 1] = __float_as_uint(-a0 * e.y + a1 * e.x);
       }
     }
     if (g.out_v8) {
-      if (obf) store32_v8(obf + d0, o);
-      else store32_v8(of32 + d0, o);
+      if (obf) store16_v8_bits(obf + d0, v);
+      else store16_v8_bits(of32 + d0, v);
     } else {
-      if (obf) store_vec<32>(obf + d0, o);
-      else store_vec<32>(of32 + d0, o);
+#pragma unroll
+      for (int j = 0; j < 16; j += 8) {
+        float o[8];
+#pragma unroll
+        for (int q2 = 0; q2 < 8; ++q2) o[q2] = __uint_as_float(v[j + q2]);
+        if (obf) store_vec<8>(obf + d0 + j, o);
+        else store_vec<8>(of32 + d0 + j, o);
+      }
     }
   }
   return ok;
@@ -348,8 +375,8 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
   uint64_t* s_free = s_full + 2;                // [2] softmax warps (4)
   uint64_t* p_full = s_free + 2;                // [2] softmax warps (4)
   uint64_t* pv_done = p_full + 2;               // [2] MMA commit
-  uint64_t* o_free = pv_done + 2;               // transition warps (4): the epilogue has read O
-  uint64_t* stats_full = o_free + 1;            // [2] by item parity, softmax warps (4): row statistics
+  uint64_t* o_free = pv_done + 2;               // [2] transition warps (4): the epilogue has read O dims 0-255 / 256-511
+  uint64_t* stats_full = o_free + 2;            // [2] by item parity, softmax warps (4): row statistics
   uint64_t* q_full = stats_full + 2;            // [2] by item parity, TMA bytes: Q and its (cos, sin) row
   uint64_t* s_done = q_full + 2;                // MMA commit after the last S of each item
   // Waiters that skip phases (the transition warps watch one event per item)
@@ -373,6 +400,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       tc::mbar_init(pv_done + s, 1);
     }
     tc::mbar_init(o_free, 4);
+    tc::mbar_init(o_free + 1, 4);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(stats_full + s, 4);
       tc::mbar_init(q_full + s, 1);
@@ -629,6 +657,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         if (!tc::mbar_wait(q_ready, ni & 1)) { ok = false; break; }
         tc::tc_fence_after();
         int next_s = 0, next_pv = 0;
+        int pv_half = 0;                            // halves of PV(next_pv) already issued
         uint64_t t_idle = 0;
         while (next_pv < x.n_tiles) {
           bool did = false;
@@ -652,15 +681,20 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
             }
           }
           if (next_pv < next_s) {
+            // PV(n): O[:, 256 half .. +255] += P V for both halves.  The first PV
+            // of an item overwrites O, so each half waits for the previous
+            // item's epilogue to have read that half (o_free[half]).
             const int gp = tcount + next_pv, sp = slot + next_pv;
             const int st = sp % kAtStages, sb = gp & 1;
-            if (tc::mbar_try_wait(p_full + sb, (gp >> 1) & 1) &&
-                (next_pv > 0 || ni == 0 || tc::mbar_try_wait(o_free, (ni - 1) & 1))) {
+            const bool first = next_pv == 0 && ni > 0;
+            if ((pv_half > 0 || tc::mbar_try_wait(p_full + sb, (gp >> 1) & 1)) &&
+                (!first || tc::mbar_try_wait(o_free + pv_half, (ni - 1) & 1))) {
               tc::tc_fence_after();
               const uint32_t pb = tc::smem_u32(s_p + sb * kAtPBytes);
               const uint32_t kb = tc::smem_u32(s_k + st * kAtKBytes);
-#pragma unroll
-              for (int half = 0; half < 2; ++half) {
+              const int h_end = first && pv_half == 0 ? 1 : 2;   // a first PV goes one half at a time
+#pragma unroll 1
+              for (int half = pv_half; half < h_end; ++half) {
 #pragma unroll
                 for (int kstep = 0; kstep < kAtKT / 16; ++kstep) {
                   const uint64_t ad = tc::sdesc_sw128(pb + kstep * 32, 16, 1024);
@@ -668,9 +702,13 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
                   tc::mma_bf16_ss(tmem + kTmO + half * 256, ad, bd, idesc_o, (next_pv > 0 || kstep > 0) ? 1u : 0u);
                 }
               }
-              tc::mma_commit(kv_empty + st);
-              tc::mma_commit(pv_done + sb);
-              ++next_pv;
+              pv_half = h_end;
+              if (pv_half == 2) {
+                tc::mma_commit(kv_empty + st);
+                tc::mma_commit(pv_done + sb);
+                ++next_pv;
+                pv_half = 0;
+              }
               did = true;
             }
           }

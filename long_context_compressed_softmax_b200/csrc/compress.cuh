@@ -169,34 +169,45 @@ __device__ __forceinline__ void fold_rows(Soft2& st, const Tin* kvs, const Tin* 
   }
 }
 
+// 2^x on the MUFU (flushes results below 2^-126 to zero: such weights are
+// negligible next to the chunk maximum's weight of 1).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
 // Fold rows r .. r+3 of a staged BF16 tile into st: the common chunk (4 rows
 // of one block).  The chunk maximum of both channels is one packed BF16 max
-// tree (exact), the weights are exp2(g log2e - m log2e) with one FFMA each.
+// tree (exact); each weight is exp2(g log2e - m log2e): one FFMA and one MUFU.
 __device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
                                            int r) {
-  __nv_bfloat162 x[4], g[4];
+  uint32_t x[4], g[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    x[u] = *reinterpret_cast<const __nv_bfloat162*>(kvs + (r + u) * D);
-    g[u] = *reinterpret_cast<const __nv_bfloat162*>(gs + (r + u) * D);
+    x[u] = *reinterpret_cast<const uint32_t*>(kvs + (r + u) * D);
+    g[u] = *reinterpret_cast<const uint32_t*>(gs + (r + u) * D);
   }
-  const float2 gm = __bfloat1622float2(__hmax2(__hmax2(g[0], g[1]), __hmax2(g[2], g[3])));
+  const __nv_bfloat162 m2 = __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[0]),
+                                            *reinterpret_cast<const __nv_bfloat162*>(&g[1])),
+                                    __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[2]),
+                                            *reinterpret_cast<const __nv_bfloat162*>(&g[3])));
+  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m2);
   constexpr float kL2e = 1.4426950408889634f;
 #pragma unroll
   for (int v = 0; v < 2; ++v) {
-    const float cm = fmaxf(st.m[v], v ? gm.y : gm.x);
+    const float cm = fmaxf(st.m[v], v ? bf_hi(mw) : bf_lo(mw));
     const float ncml = -cm * kL2e;
-    const float alpha = exp2f(fmaf(st.m[v], kL2e, ncml));     // 0 while the state is empty
-    float p[4], xv[4];
+    const float alpha = ex2(fmaf(st.m[v], kL2e, ncml));       // 0 while the state is empty (m = -inf)
+    float p[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 gf = __bfloat1622float2(g[u]);
-      const float2 xf = __bfloat1622float2(x[u]);
-      p[u] = exp2f(fmaf(v ? gf.y : gf.x, kL2e, ncml));
-      xv[u] = v ? xf.y : xf.x;
-    }
+    for (int u = 0; u < 4; ++u) p[u] = ex2(fmaf(v ? bf_hi(g[u]) : bf_lo(g[u]), kL2e, ncml));
+    const float xv0 = v ? bf_hi(x[0]) : bf_lo(x[0]), xv1 = v ? bf_hi(x[1]) : bf_lo(x[1]);
+    const float xv2 = v ? bf_hi(x[2]) : bf_lo(x[2]), xv3 = v ? bf_hi(x[3]) : bf_lo(x[3]);
     st.s[v] = fmaf(st.s[v], alpha, (p[0] + p[1]) + (p[2] + p[3]));
-    st.a[v] = fmaf(st.a[v], alpha, fmaf(p[0], xv[0], p[1] * xv[1]) + fmaf(p[2], xv[2], p[3] * xv[3]));
+    st.a[v] = fmaf(st.a[v], alpha, fmaf(p[0], xv0, p[1] * xv1) + fmaf(p[2], xv2, p[3] * xv3));
     st.m[v] = cm;
   }
 }
@@ -213,8 +224,14 @@ __device__ __forceinline__ void st_pair(__nv_bfloat16* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
+// Warp roles: warps 0 .. nw-1 fold (one channel pair per thread), warp nw
+// issues the bulk copies.  Stage k lives in slot k % kCmpStages; `full` of a
+// slot completes when its copies land, `empty` when every folding warp has
+// arrived (one arrival per warp) after reading it.
+constexpr int kCmpMaxThreads = 256 + 32;   // D <= 512: up to 8 folding warps and the copy warp
+
 template <typename Tin, typename Tout, bool kCSA>
-__global__ void __launch_bounds__(1024)
+__global__ void __launch_bounds__(kCmpMaxThreads, 4)
 compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, Tout* __restrict__ out, int T, int D,
                      int m, int Nc, int blocks_per_unit, int units_per_seq) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -222,7 +239,9 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
   const uint32_t row_bytes = (uint32_t)D * sizeof(Tin);
   const uint32_t tile_bytes = kCmpRows * row_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCmpStages * 2 * tile_bytes);
-  const int tid = threadIdx.x;
+  uint64_t* empty = full + kCmpStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nw = (int)(blockDim.x >> 5) - 1;                          // folding warps
   const int b = blockIdx.x / units_per_seq;
   const int unit = blockIdx.x - b * units_per_seq;
   const int jb = unit * blocks_per_unit;                              // first entry of this CTA
@@ -232,38 +251,48 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
   const long long ta = (long long)first * m;                          // first token row
   const int rows = (je - first) * m;
   const int K = (rows + kCmpRows - 1) / kCmpRows;                     // stages
-  const Tin* kvb = kv + ((long long)b * T + ta) * D;
-  const Tin* gb = gate + ((long long)b * T + ta) * D;
-
   if (tid == 0) {
-    for (int s = 0; s < kCmpStages; ++s) tc::mbar_init(full + s, 1);
+    for (int s = 0; s < kCmpStages; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, nw);
+    }
     tc::fence_barrier_init();
   }
   __syncthreads();
-  auto issue = [&](int k) {                                           // stage k into slot k % kCmpStages
-    const int slot = k % kCmpStages;
-    const int r0 = k * kCmpRows;
-    const int n = rows - r0 < kCmpRows ? rows - r0 : kCmpRows;
-    uint8_t* dst = smem + slot * 2 * tile_bytes;
-    tc::mbar_arrive_expect_tx(full + slot, 2u * n * row_bytes);
-    tc::bulk_load(dst, kvb + (long long)r0 * D, n * row_bytes, full + slot);
-    tc::bulk_load(dst + tile_bytes, gb + (long long)r0 * D, n * row_bytes, full + slot);
-  };
-  if (tid == 0)
-    for (int k = 0; k < kCmpStages && k < K; ++k) issue(k);
 
+  if (warp == nw) {
+    // ---------------------------------------------------------------- copies
+    if (lane == 0) {
+      const Tin* kvb = kv + ((long long)b * T + ta) * D;
+      const Tin* gb = gate + ((long long)b * T + ta) * D;
+      int k = 0;
+      for (; k < K; ++k) {
+        const int slot = k % kCmpStages;
+        if (k >= kCmpStages && !tc::mbar_wait(empty + slot, ((k / kCmpStages) - 1) & 1)) break;
+        const int r0 = k * kCmpRows;
+        const int n = rows - r0 < kCmpRows ? rows - r0 : kCmpRows;
+        uint8_t* dst = smem + slot * 2 * tile_bytes;
+        tc::mbar_arrive_expect_tx(full + slot, 2u * n * row_bytes);
+        tc::bulk_load(dst, kvb + (long long)r0 * D, n * row_bytes, full + slot);
+        tc::bulk_load(dst + tile_bytes, gb + (long long)r0 * D, n * row_bytes, full + slot);
+      }
+      // every copy issued lands before the CTA may leave
+      for (int q = k - kCmpStages > 0 ? k - kCmpStages : 0; q < k; ++q)
+        tc::mbar_wait(full + q % kCmpStages, (q / kCmpStages) & 1);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ folding
   const int c = 2 * tid;                                              // this thread's channels c, c+1
   const bool has = c < D;
   Soft2 st, prev;
   st.reset();
   prev.reset();
   int blk = first, pos = 0;                                           // current block, rows of it folded
-  int k = 0;
-  bool ok = true;
-  for (; k < K; ++k) {
+  for (int k = 0; k < K; ++k) {
     const int slot = k % kCmpStages;
-    ok = __syncthreads_and(tc::mbar_wait(full + slot, (k / kCmpStages) & 1));
-    if (!ok) break;
+    if (!__all_sync(0xffffffffu, tc::mbar_wait(full + slot, (k / kCmpStages) & 1))) break;
     const Tin* kvs = reinterpret_cast<const Tin*>(smem + slot * 2 * tile_bytes) + c;
     const Tin* gs = reinterpret_cast<const Tin*>(smem + slot * 2 * tile_bytes + tile_bytes) + c;
     const int r1 = rows - k * kCmpRows < kCmpRows ? rows - k * kCmpRows : kCmpRows;
@@ -278,15 +307,16 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
       pos += n;
       if (pos == m) {                                                 // block `blk` complete
         if (has && blk >= jb) {
+          constexpr float kL2e = 1.4426950408889634f;
           float o[2];
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
             if (kCSA) {                                               // entry 0: prev is empty
               const float M = fmaxf(prev.m[v], st.m[v]);
-              const float fa = __expf(prev.m[v] - M), fb = __expf(st.m[v] - M);
-              o[v] = (prev.a[v] * fa + st.a[v] * fb) / (prev.s[v] * fa + st.s[v] * fb);
+              const float fa = ex2((prev.m[v] - M) * kL2e), fb = ex2((st.m[v] - M) * kL2e);
+              o[v] = __fdividef(prev.a[v] * fa + st.a[v] * fb, prev.s[v] * fa + st.s[v] * fb);
             } else {
-              o[v] = st.a[v] / st.s[v];
+              o[v] = __fdividef(st.a[v], st.s[v]);
             }
           }
           st_pair(out + ((long long)b * Nc + blk) * D + c, o[0], o[1]);
@@ -297,33 +327,28 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
         ++blk;
       }
     }
-    __syncthreads();                                                  // every thread is done with the slot
-    if (tid == 0 && k + kCmpStages < K) issue(k + kCmpStages);
-  }
-  if (!ok && tid == 0) {
-    // copies in flight (stages k .. the last issued) land before the CTA leaves
-    const int last = K - 1 < k + kCmpStages - 1 ? K - 1 : k + kCmpStages - 1;
-    for (int q = k; q <= last; ++q) tc::mbar_wait(full + q % kCmpStages, (q / kCmpStages) & 1);
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(empty + slot);                     // this warp is done with the slot
   }
 }
 
 // Whole-sequence CSA (window 2m) or HCA (window m) compression with
 // per-channel gates and no RMSNorm on the bulk-copy kernel.  Returns false
-// when the shape does not fit it (odd D, more than 1024 channel pairs, or a
-// stage ring above 200 KB of shared memory).
+// when the shape does not fit it (odd D, D > 512, or a stage ring above
+// 200 KB of shared memory).
 template <typename Tin, typename Tout>
 static bool launch_compress_bulk(const void* kv, const void* gate, int B, int T, int D, int m, int window,
                                  void* out, cudaStream_t st, cudaError_t* err) {
-  if ((D & 1) || D / 2 > 1024 || (window != m && window != 2 * m)) return false;
+  if ((D & 1) || D / 2 + 32 > kCmpMaxThreads || (window != m && window != 2 * m)) return false;
   const int Nc = T / m;
   // about four CTAs per SM, each a contiguous range of blocks of one sequence
   const int want = (4 * sm_count() + B - 1) / B;
   int ups = Nc < want ? Nc : want;
   const int bpu = (Nc + ups - 1) / ups;
   ups = (Nc + bpu - 1) / bpu;
-  const size_t smem = 128 + (size_t)kCmpStages * 2 * kCmpRows * D * sizeof(Tin) + kCmpStages * 8;
+  const size_t smem = 128 + (size_t)kCmpStages * 2 * kCmpRows * D * sizeof(Tin) + kCmpStages * 16;
   if (smem > 200 * 1024) return false;
-  int threads = ((D / 2 + 31) / 32) * 32;
+  const int threads = ((D / 2 + 31) / 32) * 32 + 32;                  // folding warps + the copy warp
   auto kern = window == 2 * m ? compress_bulk_kernel<Tin, Tout, true> : compress_bulk_kernel<Tin, Tout, false>;
   *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (*err != cudaSuccess) return true;
