@@ -390,7 +390,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
   if (threadIdx.x == 0) {
     tc::mbar_init(q_ready, 4);
     for (int s = 0; s < kAtStages; ++s) {
-      tc::mbar_init(kv_full + s, kAtProdThreads);
+      // every producer arrives where all of them fill tiles (gathered rows, FP8
+      // expansion); otherwise thread 0 alone fills by TMA and arrives
+      tc::mbar_init(kv_full + s, (g.sparse || g.fp8) ? kAtProdThreads : 1);
       tc::mbar_init(kv_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -434,6 +436,11 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     // Entry tiles that every producer fills (gathered rows, FP8 expansion)
     // make the producers leave only together, at named barrier 1.
     const bool coll = g.sparse || g.fp8;
+    // The threads that need a free stage wait for it (without sleeping):
+    // thread 0, which issues every TMA copy, and the 64 threads that build a
+    // gathered tile's row table; the others are released by named barrier 1
+    // after them.  Without gathered tiles the other producers have no work.
+    const bool waits = tid == 0 || (coll && tid < kAtKT);
     bool bad = false;
     int slot = 0, ni = 0;
     // CSA: the selected entries of the next item, loaded into registers while
@@ -453,7 +460,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       }
     };
     int nc_next = at_item_nc(g, P, blockIdx.x);
-    for (int it = blockIdx.x; it < g.n_items; it += G) {
+    for (int it = (coll || tid == 0) ? blockIdx.x : g.n_items; it < g.n_items; it += G) {
       const int nc_cur = nc_next;
       nc_next = at_item_nc(g, P, it + G);
       const AtItem x = at_item(g, it, nc_cur);
@@ -463,7 +470,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         // phase completes at once (nobody waits on it) to keep the ring's
         // phase count one per slot.
         const int st = slot % kAtStages;
-        if (slot >= kAtStages && !tc::mbar_wait_backoff(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
+        if (slot >= kAtStages && tid == 0 && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
         if (*abort_flag) bad = true;
         if (bad && !coll) break;
         if (tid == 0) {
@@ -514,7 +521,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       }
       for (int n = 0; n < x.n_tiles; ++n, ++slot) {
         const int st = slot % kAtStages;
-        if (slot >= kAtStages && !tc::mbar_wait_backoff(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
+        if (slot >= kAtStages && waits && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
         if (*abort_flag) bad = true;
         const int gt = x.t0 + n;                    // tile index in the query's key list
         uint8_t* stage = s_k + st * kAtKBytes;
