@@ -211,8 +211,43 @@ __device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, 
     st.m[v] = cm;
   }
 }
+// A whole block of 4 rows into an empty state (m = 4): no rescale.
+__device__ __forceinline__ void block4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
+                                            int r) {
+  uint32_t x[4], g[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    x[u] = *reinterpret_cast<const uint32_t*>(kvs + (r + u) * D);
+    g[u] = *reinterpret_cast<const uint32_t*>(gs + (r + u) * D);
+  }
+  const __nv_bfloat162 m2 = __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[0]),
+                                            *reinterpret_cast<const __nv_bfloat162*>(&g[1])),
+                                    __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[2]),
+                                            *reinterpret_cast<const __nv_bfloat162*>(&g[3])));
+  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m2);
+  constexpr float kL2e = 1.4426950408889634f;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const float cm = v ? bf_hi(mw) : bf_lo(mw);
+    const float ncml = -cm * kL2e;
+    float p[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) p[u] = ex2(fmaf(v ? bf_hi(g[u]) : bf_lo(g[u]), kL2e, ncml));
+    const float xv0 = v ? bf_hi(x[0]) : bf_lo(x[0]), xv1 = v ? bf_hi(x[1]) : bf_lo(x[1]);
+    const float xv2 = v ? bf_hi(x[2]) : bf_lo(x[2]), xv3 = v ? bf_hi(x[3]) : bf_lo(x[3]);
+    st.s[v] = (p[0] + p[1]) + (p[2] + p[3]);
+    st.a[v] = fmaf(p[0], xv0, p[1] * xv1) + fmaf(p[2], xv2, p[3] * xv3);
+    st.m[v] = cm;
+  }
+}
 __device__ __forceinline__ void fold4(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D, int r) {
   fold4_bf16(st, kvs, gs, D, r);
+}
+__device__ __forceinline__ void block4(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D, int r) {
+  block4_bf16(st, kvs, gs, D, r);
+}
+__device__ __forceinline__ void block4(Soft2& st, const float* kvs, const float* gs, int D, int r) {
+  fold_rows<float>(st, kvs, gs, D, r, 4);
 }
 __device__ __forceinline__ void fold4(Soft2& st, const float* kvs, const float* gs, int D, int r) {
   fold_rows<float>(st, kvs, gs, D, r, 4);
@@ -300,8 +335,12 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
       int n = r1 - r < 4 ? r1 - r : 4;
       n = m - pos < n ? m - pos : n;                                  // a chunk stays inside its block
       if (has) {
-        if (n == 4) fold4(st, kvs, gs, D, r);
-        else fold_rows<Tin>(st, kvs, gs, D, r, n);
+        if (n == 4) {
+          if (pos == 0 && m == 4) block4(st, kvs, gs, D, r);          // the state is empty
+          else fold4(st, kvs, gs, D, r);
+        } else {
+          fold_rows<Tin>(st, kvs, gs, D, r, n);
+        }
       }
       r += n;
       pos += n;
@@ -312,9 +351,12 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
             if (kCSA) {                                               // entry 0: prev is empty
-              const float M = fmaxf(prev.m[v], st.m[v]);
-              const float fa = ex2((prev.m[v] - M) * kL2e), fb = ex2((st.m[v] - M) * kL2e);
-              o[v] = __fdividef(prev.a[v] * fa + st.a[v] * fb, prev.s[v] * fa + st.s[v] * fb);
+              // one weight is 1 (the block with the larger max), the other exp2(-|dm| log2e)
+              const float d = (prev.m[v] - st.m[v]) * kL2e;
+              const float f = ex2(-fabsf(d));                         // 0 when prev is empty
+              const bool pa = d > 0.f;
+              const float fa = pa ? 1.f : f, fb = pa ? f : 1.f;
+              o[v] = __fdividef(fmaf(prev.a[v], fa, st.a[v] * fb), fmaf(prev.s[v], fa, st.s[v] * fb));
             } else {
               o[v] = __fdividef(st.a[v], st.s[v]);
             }
