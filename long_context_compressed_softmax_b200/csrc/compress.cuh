@@ -179,12 +179,53 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Fold rows r .. r+3 of a staged BF16 tile into st: the common chunk (4 rows
-// of one block).  The chunk maximum of both channels is one packed BF16 max
-// tree (exact); each weight is exp2(g log2e - m log2e): one FFMA and one MUFU.
-__device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
-                                           int r) {
-  uint32_t x[4], g[4];
+// Packed FP32 pairs (the two channels of a thread): sm_100 executes add,
+// mul and fma on two FP32 lanes of a 64-bit register in one instruction.
+typedef unsigned long long f2x;
+__device__ __forceinline__ f2x pk2(float a, float b) {
+  f2x r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 upk2(f2x r) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+  return f;
+}
+__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
+  f2x r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f2x add2(f2x a, f2x b) {
+  f2x r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
+  f2x r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// a BF16 pair (channel c in the low half) as a packed FP32 pair
+__device__ __forceinline__ f2x bf2f2(uint32_t w) { return pk2(bf_lo(w), bf_hi(w)); }
+
+// Weights of 4 rows against the chunk reference -m log2e (ncml2) folded into
+// (s2, a2): p = exp2(g log2e - m log2e), s += p, a += p x.
+__device__ __forceinline__ void fold4_core(const uint32_t* x, const uint32_t* g, f2x ncml2, f2x& s2, f2x& a2) {
+  constexpr float kL2e = 1.4426950408889634f;
+  const f2x l2e2 = pk2(kL2e, kL2e);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 t = upk2(fma2(bf2f2(g[u]), l2e2, ncml2));
+    const f2x p2 = pk2(ex2(t.x), ex2(t.y));
+    s2 = add2(s2, p2);
+    a2 = fma2(p2, bf2f2(x[u]), a2);
+  }
+}
+
+__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D, int r,
+                                           uint32_t* x, uint32_t* g, uint32_t* mw) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     x[u] = *reinterpret_cast<const uint32_t*>(kvs + (r + u) * D);
@@ -194,51 +235,39 @@ __device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, 
                                             *reinterpret_cast<const __nv_bfloat162*>(&g[1])),
                                     __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[2]),
                                             *reinterpret_cast<const __nv_bfloat162*>(&g[3])));
-  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m2);
-  constexpr float kL2e = 1.4426950408889634f;
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const float cm = fmaxf(st.m[v], v ? bf_hi(mw) : bf_lo(mw));
-    const float ncml = -cm * kL2e;
-    const float alpha = ex2(fmaf(st.m[v], kL2e, ncml));       // 0 while the state is empty (m = -inf)
-    float p[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) p[u] = ex2(fmaf(v ? bf_hi(g[u]) : bf_lo(g[u]), kL2e, ncml));
-    const float xv0 = v ? bf_hi(x[0]) : bf_lo(x[0]), xv1 = v ? bf_hi(x[1]) : bf_lo(x[1]);
-    const float xv2 = v ? bf_hi(x[2]) : bf_lo(x[2]), xv3 = v ? bf_hi(x[3]) : bf_lo(x[3]);
-    st.s[v] = fmaf(st.s[v], alpha, (p[0] + p[1]) + (p[2] + p[3]));
-    st.a[v] = fmaf(st.a[v], alpha, fmaf(p[0], xv0, p[1] * xv1) + fmaf(p[2], xv2, p[3] * xv3));
-    st.m[v] = cm;
-  }
+  *mw = *reinterpret_cast<const uint32_t*>(&m2);
 }
+
+// Fold rows r .. r+3 of a staged BF16 tile into st: the common chunk (4 rows
+// of one block).  The chunk maximum of both channels is one packed BF16 max
+// tree (exact); each weight is exp2(g log2e - m log2e).
+__device__ __forceinline__ void fold4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
+                                           int r) {
+  uint32_t x[4], g[4], mw;
+  load4_bf16(kvs, gs, D, r, x, g, &mw);
+  constexpr float kL2e = 1.4426950408889634f;
+  const float cm0 = fmaxf(st.m[0], bf_lo(mw)), cm1 = fmaxf(st.m[1], bf_hi(mw));
+  // 0 while the state is empty (m = -inf)
+  const f2x al2 = pk2(ex2((st.m[0] - cm0) * kL2e), ex2((st.m[1] - cm1) * kL2e));
+  f2x s2 = mul2(pk2(st.s[0], st.s[1]), al2), a2 = mul2(pk2(st.a[0], st.a[1]), al2);
+  fold4_core(x, g, pk2(-cm0 * kL2e, -cm1 * kL2e), s2, a2);
+  const float2 sf = upk2(s2), af = upk2(a2);
+  st.s[0] = sf.x; st.s[1] = sf.y; st.a[0] = af.x; st.a[1] = af.y;
+  st.m[0] = cm0; st.m[1] = cm1;
+}
+
 // A whole block of 4 rows into an empty state (m = 4): no rescale.
 __device__ __forceinline__ void block4_bf16(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
                                             int r) {
-  uint32_t x[4], g[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    x[u] = *reinterpret_cast<const uint32_t*>(kvs + (r + u) * D);
-    g[u] = *reinterpret_cast<const uint32_t*>(gs + (r + u) * D);
-  }
-  const __nv_bfloat162 m2 = __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[0]),
-                                            *reinterpret_cast<const __nv_bfloat162*>(&g[1])),
-                                    __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&g[2]),
-                                            *reinterpret_cast<const __nv_bfloat162*>(&g[3])));
-  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m2);
+  uint32_t x[4], g[4], mw;
+  load4_bf16(kvs, gs, D, r, x, g, &mw);
   constexpr float kL2e = 1.4426950408889634f;
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const float cm = v ? bf_hi(mw) : bf_lo(mw);
-    const float ncml = -cm * kL2e;
-    float p[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) p[u] = ex2(fmaf(v ? bf_hi(g[u]) : bf_lo(g[u]), kL2e, ncml));
-    const float xv0 = v ? bf_hi(x[0]) : bf_lo(x[0]), xv1 = v ? bf_hi(x[1]) : bf_lo(x[1]);
-    const float xv2 = v ? bf_hi(x[2]) : bf_lo(x[2]), xv3 = v ? bf_hi(x[3]) : bf_lo(x[3]);
-    st.s[v] = (p[0] + p[1]) + (p[2] + p[3]);
-    st.a[v] = fmaf(p[0], xv0, p[1] * xv1) + fmaf(p[2], xv2, p[3] * xv3);
-    st.m[v] = cm;
-  }
+  const float cm0 = bf_lo(mw), cm1 = bf_hi(mw);
+  f2x s2 = 0ull, a2 = 0ull;                                         // +0.0 in both lanes
+  fold4_core(x, g, pk2(-cm0 * kL2e, -cm1 * kL2e), s2, a2);
+  const float2 sf = upk2(s2), af = upk2(a2);
+  st.s[0] = sf.x; st.s[1] = sf.y; st.a[0] = af.x; st.a[1] = af.y;
+  st.m[0] = cm0; st.m[1] = cm1;
 }
 __device__ __forceinline__ void fold4(Soft2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D, int r) {
   fold4_bf16(st, kvs, gs, D, r);
