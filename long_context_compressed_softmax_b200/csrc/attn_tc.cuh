@@ -67,6 +67,10 @@ constexpr int kAtBars = 22;
 constexpr size_t kAtSmem = 1024 + kAtOffBar + kAtBars * 8;
 static_assert(kAtSmem <= 232448, "attention shared memory exceeds 227 KB");
 constexpr int kAtCodeBytes = 448;               // FP8 entry cache: E4M3 bytes of dims 0..447 per entry
+// FP8 entry tiles stage their raw codes (64 x 448 B) in the upper part of
+// regions 3-6 of their own stage, below the rotary region 7.
+constexpr uint32_t kAtCodeStage = 7 * kAtRegion - kAtKT * kAtCodeBytes;
+static_assert(kAtCodeStage % 16 == 0 && kAtCodeStage >= 3 * kAtRegion, "FP8 code staging");
 constexpr float kLog2e = 1.4426950408889634f;
 // TMEM map: lanes 0-15 of each sub-partition hold S[0] (cols 0-63), S[1]
 // (64-127) and Q (128-383, the A operand of S = Q K^T); lanes 16-31 hold O
@@ -118,6 +122,9 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// all but this thread's most recent cp.async group have landed
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // Key-set geometry of one query: n_c compressed entries (selected or
 // visible), then the window of raw tokens.
@@ -442,6 +449,47 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     // after them.  Without gathered tiles the other producers have no work.
     const bool waits = tid == 0 || (coll && tid < kAtKT);
     bool bad = false;
+    // FP8 entry tiles are expanded one tile behind their copies: the stage of
+    // the tile whose codes are in flight or landed but not yet expanded.
+    int pend = -1;
+    constexpr int kCodePer = kAtKT * (kAtCodeBytes / 16) / kAtProdThreads;   // 7
+    constexpr int kRopePer = kAtKT * 8 / kAtProdThreads;                     // 2
+    static_assert(kCodePer * kAtProdThreads == kAtKT * (kAtCodeBytes / 16), "code pieces per thread");
+    static_assert(kRopePer * kAtProdThreads == kAtKT * 8, "rotary pieces per thread");
+    // Expand the pending tile: its copies land (keep_newest: this thread's
+    // latest group, the next tile's, may stay in flight), every producer has
+    // read its codes before any BF16 row is written over them, then a proxy
+    // fence and this thread's arrival on the tile's full barrier.  Collective
+    // over the producers; false when one of them gave up.
+    auto expand_pending = [&](bool keep_newest) -> bool {
+      if (pend < 0) return true;
+      if (keep_newest) cp_async_wait_prev();
+      else cp_async_wait_all();
+      if (!tc::bar_and(1, kAtProdThreads, !bad)) return false;
+      uint8_t* stg = s_k + pend * kAtKBytes;
+      uint4 cv[kCodePer];
+#pragma unroll
+      for (int u = 0; u < kCodePer; ++u) {
+        const int q = tid + u * kAtProdThreads;                 // 16-code piece q % 28 of row q / 28
+        cv[u] = *reinterpret_cast<const uint4*>(stg + kAtCodeStage + q * 16);
+      }
+      if (!tc::bar_and(1, kAtProdThreads, true)) return false;
+#pragma unroll
+      for (int u = 0; u < kCodePer; ++u) {
+        const int q = tid + u * kAtProdThreads;
+        const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
+        uint4 lo, hi;
+        e4m3x16_to_bf16(cv[u], s_scl[pend * kAtKT + kk], lo, hi);
+        uint8_t* row = stg + (p >> 2) * kAtRegion + kk * 128;   // 16 codes = dims 16p .. 16p+15
+        const int c0 = (p & 3) * 2;
+        *reinterpret_cast<uint4*>(row + ((c0 ^ (kk & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (kk & 7)) << 4)) = hi;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(kv_full + pend);
+      pend = -1;
+      return true;
+    };
     int slot = 0, ni = 0;
     // CSA: the selected entries of the next item, loaded into registers while
     // the current item's tiles are gathered (its first gather then starts as
@@ -527,6 +575,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         uint8_t* stage = s_k + st * kAtKBytes;
         if (gt >= x.ks.tiles_c || !coll) {
           // ---- contiguous rows: TMA boxes
+          if (pend >= 0 && !expand_pending(false)) { bad = true; break; }
           if (coll) {
             if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
           } else if (bad) {
@@ -580,49 +629,29 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
         if (g.fp8) {
-          // FP8 entry rows: every 16-byte load (codes and rotary slices) is
-          // issued before the first conversion; codes expand to BF16 with the
-          // entry's power-of-two scale (exact) and land at the swizzled
-          // addresses; absent rows are zeros.  Generic-proxy stores, so a
-          // proxy fence precedes this thread's arrival.
-          constexpr int kCodePer = kAtKT * (kAtCodeBytes / 16) / kAtProdThreads;   // 7
-          constexpr int kRopePer = kAtKT * 8 / kAtProdThreads;                     // 2
-          static_assert(kCodePer * kAtProdThreads == kAtKT * (kAtCodeBytes / 16), "code pieces per thread");
-          static_assert(kRopePer * kAtProdThreads == kAtKT * 8, "rotary pieces per thread");
-          uint4 cv[kCodePer], rv[kRopePer];
+          // FP8 entry rows: the 448 code bytes of each row land by 16-byte
+          // cp.async in the stage's code staging area, the BF16 rotary rows at
+          // their swizzled addresses in region 7 (absent rows: zeros); then
+          // the previous FP8 tile is expanded while these copies are in flight.
+          const uint32_t sb = tc::smem_u32(stage);
 #pragma unroll
           for (int u = 0; u < kCodePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
             const uint8_t* base = tab[2 * kk];
-            cv[u] = base ? __ldg(reinterpret_cast<const uint4*>(base + p * 16)) : make_uint4(0, 0, 0, 0);
+            cp_async16(sb + kAtCodeStage + q * 16, base ? base + p * 16 : dummy, base ? 16u : 0u);
           }
 #pragma unroll
           for (int u = 0; u < kRopePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q >> 3, c16 = q & 7;
             const uint8_t* base = tab[2 * kk + 1];
-            rv[u] = base ? __ldg(reinterpret_cast<const uint4*>(base + c16 * 16)) : make_uint4(0, 0, 0, 0);
+            cp_async16(sb + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4), base ? base + c16 * 16 : dummy,
+                       base ? 16u : 0u);
           }
-#pragma unroll
-          for (int u = 0; u < kCodePer; ++u) {
-            const int q = tid + u * kAtProdThreads;
-            const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
-            uint4 lo, hi;
-            e4m3x16_to_bf16(cv[u], s_scl[st * kAtKT + kk], lo, hi);
-            uint8_t* row = stage + (p >> 2) * kAtRegion + kk * 128;   // 16 codes = dims 16p .. 16p+15
-            const int c0 = (p & 3) * 2;
-            *reinterpret_cast<uint4*>(row + ((c0 ^ (kk & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (kk & 7)) << 4)) = hi;
-          }
-#pragma unroll
-          for (int u = 0; u < kRopePer; ++u) {
-            const int q = tid + u * kAtProdThreads;
-            const int kk = q >> 3, c16 = q & 7;
-            *reinterpret_cast<uint4*>(stage + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4)) = rv[u];
-          }
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(kv_full + st);
+          cp_async_commit();
+          if (pend >= 0 && !expand_pending(true)) { bad = true; break; }
+          pend = st;
           continue;
         }
         // 16-byte piece q = tid + u * kAtProdThreads of the 64 x 1 KB tile:
@@ -642,6 +671,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         }
         cp_async_arrive_noinc(kv_full + st);
       }
+      if (!bad && pend >= 0 && !expand_pending(false)) bad = true;   // no FP8 tile stays pending across items
       if (bad) break;
     }
     cp_async_wait_all();                            // nothing may land after the CTA exits
