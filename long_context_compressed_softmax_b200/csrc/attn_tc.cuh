@@ -680,6 +680,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     // ============================================================ MMA issuer
     // S(n+1) and PV(n) are independent: whichever is ready is issued first.
     if (tc::elect_one()) {
+      const uint64_t limit_ns = tc::wait_limit();                  // read once: the loop below polls
       const uint32_t idesc_s = tc::idesc_bf16(64, kAtKT, 0, 0);    // A (TMEM) K-major, B K-major
       const uint32_t idesc_o = tc::idesc_bf16(64, 256, 0, 1);      // A K-major, B MN-major
       bool ok = true;
@@ -757,7 +758,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           } else {
             const uint64_t now = tc::globaltimer();
             if (t_idle == 0) t_idle = now;
-            else if (now - t_idle > tc::wait_limit()) { report(LCSA_DEV_TIMEOUT); ok = false; break; }
+            else if (now - t_idle > limit_ns) { report(LCSA_DEV_TIMEOUT); ok = false; break; }
           }
         }
         slot += x.n_tiles;
