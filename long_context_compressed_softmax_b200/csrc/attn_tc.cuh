@@ -359,6 +359,9 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
   return ok;
 }
 
+// kFp8: the entries come from the FP8 cache (a separate instantiation, so the
+// BF16 kernel carries none of the expansion code).
+template <bool kFp8>
 __global__ void __launch_bounds__(kAtThreads, 1)
 attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ckv,
                const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rotc,
@@ -399,7 +402,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     for (int s = 0; s < kAtStages; ++s) {
       // every producer arrives where all of them fill tiles (gathered rows, FP8
       // expansion); otherwise thread 0 alone fills by TMA and arrives
-      tc::mbar_init(kv_full + s, (g.sparse || g.fp8) ? kAtProdThreads : 1);
+      tc::mbar_init(kv_full + s, (g.sparse || kFp8) ? kAtProdThreads : 1);
       tc::mbar_init(kv_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -442,7 +445,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.cs);
     // Entry tiles that every producer fills (gathered rows, FP8 expansion)
     // make the producers leave only together, at named barrier 1.
-    const bool coll = g.sparse || g.fp8;
+    const bool coll = g.sparse || kFp8;
     // The threads that need a free stage wait for it (without sleeping):
     // thread 0, which issues every TMA copy, and the 64 threads that build a
     // gathered tile's row table; the others are released by named barrier 1
@@ -613,9 +616,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
             const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
             if (j >= 0 && j < g.Nc) {
               const long long e = (long long)x.b * g.Nc + j;
-              rm = g.fp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
+              rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
               rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
-              if (g.fp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
+              if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
             } else {
               report(LCSA_DEV_BAD_INDEX);
             }
@@ -628,7 +631,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           if ((kk & 31) == 0) s_km[st * 2 + (kk >> 5)] = vm;
         }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
-        if (g.fp8) {
+        if (kFp8) {
           // FP8 entry rows: the 448 code bytes of each row land by 16-byte
           // cp.async in the stage's code staging area, the BF16 rotary rows at
           // their swizzled addresses in region 7 (absent rows: zeros); then
@@ -1140,7 +1143,8 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   g.out_v8 = (reinterpret_cast<uintptr_t>(pl.splits > 1 ? (const void*)P.o_part : a->out) & 31u) == 0 ? 1 : 0;
   g.n_items = (int)(rows * pl.splits);
   g.fp8 = f8 != nullptr;
-  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
+  auto kern = g.fp8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
   if (e != cudaSuccess) return e;
   // Tensor maps (64-row boxes, 128-byte swizzle).  A map whose tensor is
   // absent is never read; it points at q instead.
@@ -1157,7 +1161,7 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
              mk(&m_rotw, (a->Tkv > 0 && a->W > 0) ? (const void*)P.rot_w : nullptr, (uint64_t)a->B * a->Tkv, 64);
   if (!okm) return cudaErrorInvalidValue;
   const int grid = g.n_items < sm_count() ? g.n_items : sm_count();
-  attn_tc_kernel<<<grid, kAtThreads, kAtSmem, st>>>(P, g, m_q, m_ckv, m_kv, m_rotc, m_rotw);
+  kern<<<grid, kAtThreads, kAtSmem, st>>>(P, g, m_q, m_ckv, m_kv, m_rotc, m_rotw);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;

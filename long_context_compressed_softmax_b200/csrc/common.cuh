@@ -19,7 +19,7 @@ __device__ int g_status;
 // Limit of every bounded wait in the library's kernels (ns of %globaltimer);
 // lcsa_set_wait_limit_ns changes it per device.
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;   // 2 s
-__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+__constant__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;   // constant cache: cheap to poll
 
 __device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
 

@@ -53,7 +53,7 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // Bounded wait: gives up after the device's wait limit (g_wait_limit_ns, 2 s
 // unless lcsa_set_wait_limit_ns changed it), records LCSA_DEV_TIMEOUT and
 // returns false.  Callers then stop issuing work and leave the kernel.
-__device__ __forceinline__ uint64_t wait_limit() { return *(volatile unsigned long long*)&g_wait_limit_ns; }
+__device__ __forceinline__ uint64_t wait_limit() { return g_wait_limit_ns; }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
