@@ -54,11 +54,11 @@ SPEC_HBM_GBS = 7700.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # kernel source it was taken on; a changed source reports null.
 NCU_TRAFFIC = {
-    # csa_prefill_8k capture (8192 queries): 585.4 MB read + 493.3 MB written =
+    # csa_prefill_8k capture (8192 queries): 584.8 MB read + 493.9 MB written =
     # 131.7 KB per query (Q in, BF16 output out; entry rows hit L2), scaled to
     # the stack's CSA launch of 2 x 131072 queries.
     "csa_sparse_attn": {"bytes_per_launch": 34.52e9, "file": "long_context_compressed_softmax_b200/csrc/attn_tc.cuh",
-                        "src": "f37a1d5cc82fb240"},
+                        "src": "230cf93a763e5194"},
 }
 
 def _src_hash(rel):
@@ -391,6 +391,7 @@ def run_reference(args, cfg, world, rank):
 # ----------------------------------------------------------------------------- GPU arm
 def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
     layers = [Layer(kind, cfg, rank_seed(cfg.seed * 10 + li, rank), dev) for li, kind in enumerate(cfg.layers)]
+    lcsa.set_attn_gather(1 if args.attn_gather == "tma" else 0)
     runner = StackRunner(lcsa, cfg, layers, dev, fp8_entries=args.fp8_entries)
     n0 = lcsa.kernel_launches()
     runner.step()
@@ -487,7 +488,8 @@ def run_stack(args, cfg, lcsa, dev, world, rank, bus_id, peaks):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)-scaled BF16 inputs, independent per layer and rank)",
-            "config": config_obj(cfg, world) | ({"csa_entries": "fp8 cache"} if args.fp8_entries else {}),
+            "config": config_obj(cfg, world) | ({"csa_entries": "fp8 cache"} if args.fp8_entries else {})
+                      | ({"csa_row_staging": "tma gather4"} if args.attn_gather == "tma" else {}),
             "layer_ms": layer_ms, "kernels": summary, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
     if out_proj is not None:
@@ -813,6 +815,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8-entries", action="store_true",
                     help="CSA layers attend over the FP8 entry cache (quantised after compression, in the step)")
+    ap.add_argument("--attn-gather", default="cp.async", choices=["cp.async", "tma"],
+                    help="how CSA attention stages its selected BF16 rows (16-byte cp.async, or TMA tile::gather4)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -93,6 +93,16 @@ lcsa_status lcsa_set_wait_limit_ns(uint64_t ns);
  * undefined; later calls are unaffected.  chunk < 0 clears a pending hook. */
 void lcsa_test_withhold_stage(int chunk);
 
+/* How CSA sparse attention on BF16 entries stages its selected rows (the
+ * entries chosen by top-k, [p2] CSA Step 3; the pages leave the copy
+ * mechanism open): mode 0 (default) gathers each 64-row tile with 16-byte
+ * cp.async copies from all producer warps; mode 1 uses TMA tile::gather4
+ * (four 128-byte rows per copy, 128 copies per tile, issued by the same
+ * warps).  Both give identical results; mode 0 is the faster on B200 and
+ * mode 1 is kept for measurement.  Process-wide; applies to calls issued
+ * after it.  Any other value: LCSA_ERR_INVALID_ARG. */
+lcsa_status lcsa_set_attn_gather(int mode);
+
 /* ------------------------------------------------------------------------
  * KV compression ([p2] CSA Step 1: m consecutive tokens merged into one entry
  * with learned softmax weights; [p2] HCA: m' = 128 tokens per entry; [p3]

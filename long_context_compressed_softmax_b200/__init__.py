@@ -35,7 +35,7 @@ EXPORTED = [
     "lcsa_grouped_out_proj_workspace", "lcsa_grouped_out_proj",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
     "lcsa_quantize_entries_fp8", "lcsa_csa_sparse_attn_fp8", "lcsa_hca_dense_attn_fp8",
-    "lcsa_set_wait_limit_ns", "lcsa_test_withhold_stage",
+    "lcsa_set_wait_limit_ns", "lcsa_test_withhold_stage", "lcsa_set_attn_gather",
 ]
 
 
@@ -116,6 +116,7 @@ _sig = {
     "lcsa_quantize_entries_fp8": (_i, [_vp, _i64, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "lcsa_set_wait_limit_ns": (_i, [ctypes.c_uint64]),
     "lcsa_test_withhold_stage": (None, [_i]),
+    "lcsa_set_attn_gather": (_i, [_i]),
     "lcsa_csa_sparse_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
 }
@@ -170,6 +171,11 @@ def kernel_launches() -> int:
 def set_wait_limit_ns(ns: int) -> None:
     """Limit of the kernels' bounded waits on the current device (0 = the 2 s default)."""
     _check(_lib.lcsa_set_wait_limit_ns(int(ns)), "set_wait_limit_ns")
+
+
+def set_attn_gather(mode: int) -> None:
+    """CSA row staging on BF16 entries: 0 = cp.async (default), 1 = TMA tile::gather4."""
+    _check(_lib.lcsa_set_attn_gather(int(mode)), "set_attn_gather")
 
 
 def get_device_status() -> int:

@@ -34,6 +34,8 @@
 // bounded; abort decisions among threads that share a named barrier are
 // taken collectively at that barrier.
 #pragma once
+#include <atomic>
+
 #include "tc_ptx.cuh"
 #include "rope.cuh"
 #include "fp8cache.cuh"
@@ -360,8 +362,10 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
 }
 
 // kFp8: the entries come from the FP8 cache (a separate instantiation, so the
-// BF16 kernel carries none of the expansion code).
-template <bool kFp8>
+// BF16 kernel carries none of the expansion code).  kG4: BF16 selected rows
+// arrive by TMA tile::gather4 instead of 16-byte cp.async (the measured
+// alternative; cp.async is the default).
+template <bool kFp8, bool kG4>
 __global__ void __launch_bounds__(kAtThreads, 1)
 attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ckv,
                const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rotc,
@@ -402,7 +406,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     for (int s = 0; s < kAtStages; ++s) {
       // every producer arrives where all of them fill tiles (gathered rows, FP8
       // expansion); otherwise thread 0 alone fills by TMA and arrives
-      tc::mbar_init(kv_full + s, (g.sparse || kFp8) ? kAtProdThreads : 1);
+      tc::mbar_init(kv_full + s, ((g.sparse && !kG4) || kFp8) ? kAtProdThreads : 1);
       tc::mbar_init(kv_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -432,8 +436,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     // ============================================================ producers
     // Q and contiguous key tiles (every HCA entry tile and every window tile)
     // arrive as eight 2D TMA boxes of 64 rows x 64 dims; CSA's selected rows
-    // are gathered 16 bytes at a time with cp.async by all producer warps.  In
-    // CSA the producers share named barrier 1, so they leave only together.
+    // are gathered 16 bytes at a time with cp.async by all producer warps
+    // (which share named barrier 1 and leave only together), or with kG4 by
+    // TMA gather, four rows per copy, warp w filling column block w.
     const int tid = threadIdx.x;                    // 0..kAtProdThreads-1
     if (tid == 0) {
       tc::prefetch_tmap(&tm_q);
@@ -445,13 +450,27 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
     const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.cs);
     // Entry tiles that every producer fills (gathered rows, FP8 expansion)
     // make the producers leave only together, at named barrier 1.
-    const bool coll = g.sparse || kFp8;
+    const bool coll = (g.sparse && !kG4) || kFp8;
+    // TMA-gathered rows: every producer warp gathers; the lanes of a warp
+    // share its abort decisions by warp votes.
+    const bool gw = kG4 && g.sparse;
     // The threads that need a free stage wait for it (without sleeping):
-    // thread 0, which issues every TMA copy, and the 64 threads that build a
-    // gathered tile's row table; the others are released by named barrier 1
-    // after them.  Without gathered tiles the other producers have no work.
-    const bool waits = tid == 0 || (coll && tid < kAtKT);
+    // thread 0, which issues every TMA copy, the 64 threads that build a
+    // gathered tile's row table (the others are released by named barrier 1
+    // after them) and the TMA-gathering warps.  Otherwise the other producers
+    // have no work.
+    const bool waits = tid == 0 || (coll && tid < kAtKT) || gw;
     bool bad = false;
+    // The slot of the latest TMA fill of each stage and of each Q buffer
+    // (thread 0), so that an abort waits for the copies still in flight
+    // (registers: a run-time index into an array would put it on the stack).
+    static_assert(kAtStages == 3, "one fill record per stage");
+    int tx0 = -1, tx1 = -1, tx2 = -1, txq0 = -1, txq1 = -1;
+    auto set_tx = [&](int st, int v) {
+      if (st == 0) tx0 = v;
+      else if (st == 1) tx1 = v;
+      else tx2 = v;
+    };
     // FP8 entry tiles are expanded one tile behind their copies: the stage of
     // the tile whose codes are in flight or landed but not yet expanded.
     int pend = -1;
@@ -511,7 +530,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       }
     };
     int nc_next = at_item_nc(g, P, blockIdx.x);
-    for (int it = (coll || tid == 0) ? blockIdx.x : g.n_items; it < g.n_items; it += G) {
+    for (int it = (coll || tid == 0 || gw) ? blockIdx.x : g.n_items; it < g.n_items; it += G) {
       const int nc_cur = nc_next;
       nc_next = at_item_nc(g, P, it + G);
       const AtItem x = at_item(g, it, nc_cur);
@@ -523,10 +542,13 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         const int st = slot % kAtStages;
         if (slot >= kAtStages && tid == 0 && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
         if (*abort_flag) bad = true;
+        if (gw) bad = __any_sync(0xffffffffu, bad);
         if (bad && !coll) break;
         if (tid == 0) {
           uint64_t* qf = q_full + (ni & 1);
           if (!bad) {
+            set_tx(st, -1);                         // the stage's previous fill was consumed
+            if (ni & 1) txq1 = ni; else txq0 = ni;
             tc::mbar_arrive_expect_tx(qf, kAtKBytes + kAtCsBytes);
 #pragma unroll
             for (int reg = 0; reg < 8; ++reg)
@@ -536,12 +558,12 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
             tc::mbar_arrive(qf);
           }
         }
-        tc::mbar_arrive(kv_full + st);
+        if (coll || tid == 0) tc::mbar_arrive(kv_full + st);
         ++slot;
         ++ni;
       }
       const int slot0 = x.t0 * kAtKT;
-      if (g.sparse) {
+      if (g.sparse && coll) {
         // Every read of the previous item's s_idx precedes the barrier of its
         // last gathered tile, which all producers have passed.  The entries
         // come from the registers filled during the previous item (all loads
@@ -572,10 +594,69 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       }
       for (int n = 0; n < x.n_tiles; ++n, ++slot) {
         const int st = slot % kAtStages;
+        const int gt = x.t0 + n;                    // tile index in the query's key list
+        // TMA-gathered tile: lane l of each warp reads the entries of keys
+        // 4 (l % 16) .. +3, the four-row group its copy fills, before the
+        // stage wait
+        const bool gath = gw && gt < x.ks.tiles_c;
+        int32_t ev[4];
+        if (gath) {
+          const int sl0 = gt * kAtKT + 4 * (lane & 15);
+          const int32_t* idx_row = P.idx + x.row * g.k;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ev[j] = sl0 + j < x.ks.n_c ? __ldg(idx_row + sl0 + j) : -1;
+        }
         if (slot >= kAtStages && waits && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
         if (*abort_flag) bad = true;
-        const int gt = x.t0 + n;                    // tile index in the query's key list
+        if (gw) bad = __any_sync(0xffffffffu, bad);
         uint8_t* stage = s_k + st * kAtKBytes;
+        if (gath) {
+          // ---- selected rows by TMA gather: warp w < 7 fills entry column
+          // block w, warp 7 the rotated slice, lanes 0-15 one four-row group
+          // each; absent rows and bad indices take a row past the tensor's
+          // end (zeros) and leave the tile's row mask.  Thread 0 arms the
+          // stage for all 64 KB; a copy of another warp may land first (the
+          // pending byte count goes below zero until then).
+          if (bad) break;
+          const int grp = lane & 15;
+          const int oob_c = (int)((long long)g.B * g.Nc);
+          const int oob_r = g.rot_slot ? (int)(g.rows * g.k) : oob_c;
+          int yc[4], yr[4];
+          uint32_t v = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int sl = gt * kAtKT + 4 * grp + j;
+            yc[j] = oob_c;
+            yr[j] = oob_r;
+            if (sl < x.ks.n_c) {
+              if (ev[j] >= 0 && ev[j] < g.Nc) {
+                yc[j] = (int)((long long)x.b * g.Nc + ev[j]);
+                yr[j] = g.rot_slot ? (int)(x.row * g.k + sl) : yc[j];
+                v |= 1u << j;
+              } else if (tid < 16) {                // warp 0 reports
+                report(LCSA_DEV_BAD_INDEX);
+              }
+            }
+          }
+          if (warp == 0) {
+            const uint32_t km_lo = __reduce_or_sync(0xffffffffu, grp < 8 ? v << (4 * grp) : 0u);
+            const uint32_t km_hi = __reduce_or_sync(0xffffffffu, grp >= 8 ? v << (4 * (grp - 8)) : 0u);
+            if (tid == 0) {
+              s_km[st * 2] = km_lo;
+              s_km[st * 2 + 1] = km_hi;
+              set_tx(st, slot);
+              tc::mbar_arrive_expect_tx(kv_full + st, kAtKBytes);
+            }
+          }
+          if (lane < 16) {
+            uint8_t* dst = stage + warp * kAtRegion + grp * 4 * 128;
+            if (warp < 7)
+              tc::tma_gather4(dst, &tm_ckv, kv_full + st, warp * 64, yc[0], yc[1], yc[2], yc[3]);
+            else
+              tc::tma_gather4(dst, &tm_rotc, kv_full + st, 0, yr[0], yr[1], yr[2], yr[3]);
+          }
+          continue;
+        }
         if (gt >= x.ks.tiles_c || !coll) {
           // ---- contiguous rows: TMA boxes
           if (pend >= 0 && !expand_pending(false)) { bad = true; break; }
@@ -595,11 +676,12 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
               mm = &tm_kv; mr = &tm_rotw;
               y = (int)((long long)x.b * g.Tkv + (x.ks.wlo - g.kv_pos0) + (long long)(gt - x.ks.tiles_c) * kAtKT);
             }
+            set_tx(st, slot);
             tc::mbar_arrive_expect_tx(kv_full + st, kAtKBytes);
 #pragma unroll
             for (int reg = 0; reg < 7; ++reg) tc::tma_load_2d(stage + reg * kAtRegion, mm, kv_full + st, reg * 64, y);
             tc::tma_load_2d(stage + 7 * kAtRegion, mr, kv_full + st, 0, y);
-          } else {
+          } else if (coll) {
             tc::mbar_arrive(kv_full + st);
           }
           continue;
@@ -678,7 +760,19 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       if (bad) break;
     }
     cp_async_wait_all();                            // nothing may land after the CTA exits
-    if (bad) *abort_flag = 1;
+    if (bad) {
+      *abort_flag = 1;
+      // TMA fills still in flight land before the CTA exits (bounded waits:
+      // each of these fills was armed with its full byte count)
+      if (tid == 0) {
+        const int txs[3] = {tx0, tx1, tx2};
+#pragma unroll
+        for (int s2 = 0; s2 < kAtStages; ++s2)
+          if (txs[s2] >= 0) tc::mbar_wait(kv_full + s2, (txs[s2] / kAtStages) & 1);
+        if (txq0 >= 0) tc::mbar_wait(q_full, (txq0 >> 1) & 1);
+        if (txq1 >= 0) tc::mbar_wait(q_full + 1, (txq1 >> 1) & 1);
+      }
+    }
   } else if (warp == kAtMmaWarp) {
     // ============================================================ MMA issuer
     // S(n+1) and PV(n) are independent: whichever is ready is issued first.
@@ -1079,6 +1173,13 @@ static AtPlan attn_tc_plan(const lcsa_attn_args* a, int sparse) {
 
 static size_t attn_tc_workspace(const lcsa_attn_args* a, int sparse) { return attn_tc_plan(a, sparse).total; }
 
+// How BF16 CSA tiles gather their selected rows: 0 = 16-byte cp.async by all
+// producer warps (default), 1 = TMA tile::gather4.
+inline std::atomic<int>& attn_gather_mode() {
+  static std::atomic<int> m{0};
+  return m;
+}
+
 // f8 != null: the entries come from the FP8 cache (a->ckv is not read).
 static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws, cudaStream_t st,
                                   const lcsa_fp8_entries* f8 = nullptr) {
@@ -1088,6 +1189,11 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   const long long rows = (long long)a->B * a->Tq;
   // int32 item indices and TMA row coordinates
   if (rows * pl.splits * 64 > (long long)INT32_MAX - 64 * 1024) return cudaErrorInvalidValue;
+  const bool g4 = sparse && f8 == nullptr && attn_gather_mode().load() == 1;
+  // TMA-gathered rows: entry and rotary-slice row coordinates, and the row
+  // past the end that absent rows read, are int32
+  if (g4 && ((long long)a->B * a->Nc >= (long long)INT32_MAX || (pl.rot_slot && rows * a->k >= (long long)INT32_MAX)))
+    return cudaErrorInvalidValue;
   AtPtrs P;
   P.ckv = (const __nv_bfloat16*)a->ckv;
   P.c8 = f8 ? f8->codes : nullptr;
@@ -1143,22 +1249,25 @@ static cudaError_t launch_attn_tc(const lcsa_attn_args* a, int sparse, void* ws,
   g.out_v8 = (reinterpret_cast<uintptr_t>(pl.splits > 1 ? (const void*)P.o_part : a->out) & 31u) == 0 ? 1 : 0;
   g.n_items = (int)(rows * pl.splits);
   g.fp8 = f8 != nullptr;
-  auto kern = g.fp8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  auto kern = g.fp8 ? attn_tc_kernel<true, false> : g4 ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
   if (e != cudaSuccess) return e;
-  // Tensor maps (64-row boxes, 128-byte swizzle).  A map whose tensor is
-  // absent is never read; it points at q instead.
+  // Tensor maps (128-byte swizzle): 64-row boxes, except the entry and
+  // rotary-slice maps of TMA-gathered CSA, which read one row per box row.
+  // A map whose tensor is absent is never read; it points at q instead.
   CUtensorMap m_q, m_ckv, m_kv, m_rotc, m_rotw;
   const uint64_t rows_rotc = pl.rot_slot ? (uint64_t)rows * a->k : (uint64_t)a->B * a->Nc;
-  auto mk = [&](CUtensorMap* m, const void* base, uint64_t nrows, uint64_t cols) {
-    if (base == nullptr || nrows == 0) return make_tmap_bf16_2d(m, a->q, (uint64_t)rows * 64, 512, 512, 64, 64);
-    return make_tmap_bf16_2d(m, base, nrows, cols, cols, 64, 64);
+  const uint32_t box_c = g4 ? 1 : 64;
+  auto mk = [&](CUtensorMap* m, const void* base, uint64_t nrows, uint64_t cols, uint32_t box_rows) {
+    if (base == nullptr || nrows == 0) return make_tmap_bf16_2d(m, a->q, (uint64_t)rows * 64, 512, 512, 64, box_rows);
+    return make_tmap_bf16_2d(m, base, nrows, cols, cols, 64, box_rows);
   };
-  bool okm = mk(&m_q, a->q, (uint64_t)rows * 64, 512) &&
-             mk(&m_ckv, (a->Nc > 0 && !f8) ? a->ckv : nullptr, (uint64_t)a->B * a->Nc, 512) &&
-             mk(&m_kv, a->Tkv > 0 ? a->kv : nullptr, (uint64_t)a->B * a->Tkv, 512) &&
-             mk(&m_rotc, a->Nc > 0 ? (const void*)P.rot_c : nullptr, rows_rotc, 64) &&
-             mk(&m_rotw, (a->Tkv > 0 && a->W > 0) ? (const void*)P.rot_w : nullptr, (uint64_t)a->B * a->Tkv, 64);
+  bool okm = mk(&m_q, a->q, (uint64_t)rows * 64, 512, 64) &&
+             mk(&m_ckv, (a->Nc > 0 && !f8) ? a->ckv : nullptr, (uint64_t)a->B * a->Nc, 512, box_c) &&
+             mk(&m_kv, a->Tkv > 0 ? a->kv : nullptr, (uint64_t)a->B * a->Tkv, 512, 64) &&
+             mk(&m_rotc, a->Nc > 0 ? (const void*)P.rot_c : nullptr, rows_rotc, 64, box_c) &&
+             mk(&m_rotw, (a->Tkv > 0 && a->W > 0) ? (const void*)P.rot_w : nullptr, (uint64_t)a->B * a->Tkv, 64,
+                64);
   if (!okm) return cudaErrorInvalidValue;
   const int grid = g.n_items < sm_count() ? g.n_items : sm_count();
   kern<<<grid, kAtThreads, kAtSmem, st>>>(P, g, m_q, m_ckv, m_kv, m_rotc, m_rotw);

@@ -250,6 +250,12 @@ lcsa_status lcsa_set_wait_limit_ns(uint64_t ns) {
 
 void lcsa_test_withhold_stage(int chunk) { gemm_withhold_next().store(chunk < 0 ? -1 : chunk); }
 
+lcsa_status lcsa_set_attn_gather(int mode) {
+  if (mode != 0 && mode != 1) return LCSA_ERR_INVALID_ARG;
+  attn_gather_mode().store(mode);
+  return LCSA_OK;
+}
+
 lcsa_status lcsa_csa_compress(const void* kv, const void* gate, int gate_per_channel, int B, int T, int D, int m,
                               lcsa_dtype dtype, const float* rms_weight, float rms_eps, void* out,
                               lcsa_dtype out_dtype, void* stream) {

@@ -222,3 +222,11 @@ def test_fp8_cache_calls_check_arguments(lcsa):
     if not torch.cuda.is_available():
         ws = ctypes.c_void_p(0x100000)
         assert L.lcsa_hca_dense_attn_fp8(ctypes.byref(a), ctypes.byref(e), ws, 1 << 30, None) == 4   # no CPU path
+
+
+def test_attn_gather_mode_argument(lcsa):
+    """The CSA row-staging switch takes 0 (cp.async) or 1 (TMA gather) only."""
+    L = lcsa.lib
+    assert L.lcsa_set_attn_gather(2) == 1 and L.lcsa_set_attn_gather(-1) == 1
+    assert L.lcsa_set_attn_gather(1) == 0
+    assert L.lcsa_set_attn_gather(0) == 0
