@@ -454,11 +454,20 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
 #pragma unroll
     for (int w = 1; w < kTk2Warps; ++w) { lo = fminf(lo, s_lo[w]); hi = fmaxf(hi, s_hi[w]); }
     // one bucket for everything when the sampled range is empty or not finite
-    const float scale = (hi > lo && hi - lo < INFINITY) ? (float)kTk2Bins / (hi - lo) : 0.f;
+    const float s0 = (hi > lo && hi - lo < INFINITY) ? (float)kTk2Bins / (hi - lo) : 0.f;
+    const float scale = fabsf(lo * s0) < 1e30f ? s0 : 0.f;   // the offset below stays finite
+    // bucket = (v - lo) * scale - 1/2 rounded to an integer and clamped to
+    // [0, kTk2Bins - 1], taken from the low mantissa bits of a float in
+    // [2^23, 2^23 + kTk2Bins - 1] (where one ulp is 1): one FMA, two clamps
+    // and a mask.  A correctly rounded FMA of a function increasing in v is
+    // non-decreasing in v, and so is the clamp: the bucket order never
+    // contradicts the score order.  NaN-free rows (an infinite score clamps
+    // to an end bucket).
+    constexpr float kTwo23 = 8388608.f;
+    const float c0 = scale == 0.f ? kTwo23 : kTwo23 - lo * scale - 0.5f;
     auto bucket = [&](float v) -> uint32_t {
-      if (scale == 0.f) return 0u;
-      const float x = (v - lo) * scale;                 // monotone in v; NaN-free rows
-      return x <= 0.f ? 0u : (x >= (float)(kTk2Bins - 1) ? (uint32_t)(kTk2Bins - 1) : (uint32_t)x);
+      const float y = fminf(fmaxf(fmaf(v, scale, c0), kTwo23), kTwo23 + (float)(kTk2Bins - 1));
+      return __float_as_uint(y) & 0x7FFFFFu;
     };
     // contiguous warp segments [seg_lo, seg_hi), lengths multiples of 256:
     // lane L owns elements 8L .. 8L+7 of each 256-element step
