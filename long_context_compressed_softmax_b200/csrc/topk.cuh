@@ -331,6 +331,15 @@ constexpr int kTk2Bins = 2048;
 constexpr int kTk2List = 1024;
 constexpr uint16_t kTk2Sel = 2048;                  // code of a selected score of the pivot bucket
 
+// Two 16-bit codes per 32-bit word (codes <= 2048 < 2^15): adding
+// 0x7FFF - b to each half sets the half's bit 15 exactly when its code is
+// above b, with no carry between the halves; 0x8000 - b sets it when the code
+// is at least b.  Flags of a word land at bits 15 and 31.
+constexpr uint32_t kTk2Hi = 0x80008000u;
+__device__ __forceinline__ uint32_t half_add(uint32_t b0) { return b0 | (b0 << 16); }
+// flags (bits 15, 31) of the two codes of w -> bits 0, 1
+__device__ __forceinline__ uint32_t pair_bits(uint32_t t) { return ((t >> 15) | (t >> 30)) & 3u; }
+
 // Block-wide k-th largest key (ranks counted from 1) among cnt keys given by
 // get(c, &key) -> valid; refines *st over three digit levels so that on
 // return st->prefix is the exact key and st->kr the number of its copies to
@@ -548,22 +557,28 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     // (unordered: ranks use the column as the tie break)
     {
       uint32_t a = 0;
+      const uint32_t gt2 = half_add(0x7FFFu - bpiv), ge2 = half_add(0x8000u - bpiv);
       for (int base = seg_lo; base < seg_hi; base += 256) {
         const int i0 = base + 8 * lane;
-        uint32_t cq[8];
+        uint32_t f = 0;
         if (i0 + 7 < seg_hi) {
+          // eight codes at once: the count above bpiv and the flags of bpiv
           const uint4 c = *reinterpret_cast<const uint4*>(s_code + i0);
-          cq[0] = c.x & 0xFFFFu; cq[1] = c.x >> 16; cq[2] = c.y & 0xFFFFu; cq[3] = c.y >> 16;
-          cq[4] = c.z & 0xFFFFu; cq[5] = c.z >> 16; cq[6] = c.w & 0xFFFFu; cq[7] = c.w >> 16;
+          const uint32_t g0 = (c.x + gt2) & kTk2Hi, g1 = (c.y + gt2) & kTk2Hi;
+          const uint32_t g2 = (c.z + gt2) & kTk2Hi, g3 = (c.w + gt2) & kTk2Hi;
+          a += (uint32_t)__popc(g0 | (g1 >> 1) | (g2 >> 2) | (g3 >> 3));
+          if (fits) {
+            const uint32_t e0 = (c.x + ge2) & ~g0 & kTk2Hi, e1 = (c.y + ge2) & ~g1 & kTk2Hi;
+            const uint32_t e2 = (c.z + ge2) & ~g2 & kTk2Hi, e3 = (c.w + ge2) & ~g3 & kTk2Hi;
+            f = pair_bits(e0) | (pair_bits(e1) << 2) | (pair_bits(e2) << 4) | (pair_bits(e3) << 6);
+          }
         } else {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) cq[q] = i0 + q < seg_hi ? s_code[i0 + q] : 0u;
-        }
-        uint32_t f = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          a += (i0 + q < seg_hi && cq[q] > bpiv) ? 1u : 0u;
-          f |= (uint32_t)(fits && i0 + q < seg_hi && cq[q] == bpiv) << q;
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t cq = i0 + q < seg_hi ? s_code[i0 + q] : 0u;
+            a += (i0 + q < seg_hi && cq > bpiv) ? 1u : 0u;
+            f |= (uint32_t)(fits && i0 + q < seg_hi && cq == bpiv) << q;
+          }
         }
         if (!__any_sync(0xffffffffu, f != 0u)) continue;
         const uint32_t mine = (uint32_t)__popc(f);
@@ -682,6 +697,7 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
     if (has_next) smp_next = sample(src2, n2);         // next row's sample, in flight during the emission
     // ---- emission: the selection is {code > bpiv}, written in index order
     {
+      const uint32_t gt2 = half_add(0x7FFFu - bpiv);
       uint32_t pos = 0;
       for (int w = 0; w < warp; ++w) pos += s_wa[w];
       for (int base = seg_lo; base < seg_hi; base += 256) {
@@ -689,10 +705,8 @@ topk_smem_kernel(const float* __restrict__ scores, long long ld, int n_cols, con
         uint32_t f = 0;
         if (i0 + 7 < seg_hi) {
           const uint4 c = *reinterpret_cast<const uint4*>(s_code + i0);
-          f = (uint32_t)((c.x & 0xFFFFu) > bpiv) | ((uint32_t)((c.x >> 16) > bpiv) << 1) |
-              ((uint32_t)((c.y & 0xFFFFu) > bpiv) << 2) | ((uint32_t)((c.y >> 16) > bpiv) << 3) |
-              ((uint32_t)((c.z & 0xFFFFu) > bpiv) << 4) | ((uint32_t)((c.z >> 16) > bpiv) << 5) |
-              ((uint32_t)((c.w & 0xFFFFu) > bpiv) << 6) | ((uint32_t)((c.w >> 16) > bpiv) << 7);
+          f = pair_bits((c.x + gt2) & kTk2Hi) | (pair_bits((c.y + gt2) & kTk2Hi) << 2) |
+              (pair_bits((c.z + gt2) & kTk2Hi) << 4) | (pair_bits((c.w + gt2) & kTk2Hi) << 6);
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q) f |= (uint32_t)(i0 + q < seg_hi && s_code[i0 + q] > bpiv) << q;
