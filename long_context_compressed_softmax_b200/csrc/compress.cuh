@@ -282,6 +282,61 @@ __device__ __forceinline__ void fold4(Soft2& st, const float* kvs, const float* 
   fold_rows<float>(st, kvs, gs, D, r, 4);
 }
 
+// CSA with m = 4 on BF16 rows: the packed state of one block of 4 rows
+// (both channels), with the block maximum kept as -m log2e, the reference
+// its weights were taken against.
+struct Blk2 {
+  f2x nml2, s2, a2;
+  __device__ __forceinline__ void reset() {       // empty: m = -inf, s = a = 0
+    nml2 = pk2(INFINITY, INFINITY);
+    s2 = a2 = 0ull;
+  }
+};
+__device__ __forceinline__ void block4_packed(Blk2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D,
+                                              int r) {
+  uint32_t x[4], g[4], mw;
+  load4_bf16(kvs, gs, D, r, x, g, &mw);
+  constexpr float kL2e = 1.4426950408889634f;
+  st.nml2 = mul2(pk2(bf_lo(mw), bf_hi(mw)), pk2(-kL2e, -kL2e));
+  st.s2 = st.a2 = 0ull;
+  fold4_core(x, g, st.nml2, st.s2, st.a2);
+}
+// Fold the 8 rows of a stage into a running packed state (HCA blocks of a
+// multiple of 8 rows): one packed BF16 max tree over the 8 gate rows, one
+// rescale of the state to the new maximum (0 while the state is empty), then
+// the weights of the 8 rows against it.
+__device__ __forceinline__ void fold8_packed(Blk2& st, const __nv_bfloat16* kvs, const __nv_bfloat16* gs, int D) {
+  uint32_t x[8], g[8], mlo, mhi;
+  load4_bf16(kvs, gs, D, 0, x, g, &mlo);
+  load4_bf16(kvs, gs, D, 4, x + 4, g + 4, &mhi);
+  const __nv_bfloat162 m2 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&mlo),
+                                    *reinterpret_cast<const __nv_bfloat162*>(&mhi));
+  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m2);
+  constexpr float kL2e = 1.4426950408889634f;
+  const float2 cn = upk2(mul2(pk2(bf_lo(mw), bf_hi(mw)), pk2(-kL2e, -kL2e)));
+  const float2 on = upk2(st.nml2);
+  const f2x nml = pk2(fminf(on.x, cn.x), fminf(on.y, cn.y));   // the larger maximum
+  const float2 df = upk2(fma2(st.nml2, pk2(-1.f, -1.f), nml));   // (m_old - m_new) log2e <= 0
+  const f2x al2 = pk2(ex2(df.x), ex2(df.y));
+  st.s2 = mul2(st.s2, al2);
+  st.a2 = mul2(st.a2, al2);
+  st.nml2 = nml;
+  fold4_core(x, g, nml, st.s2, st.a2);
+  fold4_core(x + 4, g + 4, nml, st.s2, st.a2);
+}
+
+// CSA entry of blocks (prev, cur) per channel: the block with the larger
+// maximum weighs 1, the other exp2(-|dm| log2e) (0 when prev is empty).
+__device__ __forceinline__ float2 csa_merge_packed(const Blk2& p, const Blk2& c) {
+  const float2 d = upk2(fma2(p.nml2, pk2(-1.f, -1.f), c.nml2));     // (m_prev - m_cur) log2e
+  const float f0 = ex2(-fabsf(d.x)), f1 = ex2(-fabsf(d.y));
+  const bool p0 = d.x > 0.f, p1 = d.y > 0.f;
+  const f2x fa = pk2(p0 ? 1.f : f0, p1 ? 1.f : f1), fb = pk2(p0 ? f0 : 1.f, p1 ? f1 : 1.f);
+  const float2 num = upk2(fma2(p.a2, fa, mul2(c.a2, fb)));
+  const float2 den = upk2(fma2(p.s2, fa, mul2(c.s2, fb)));
+  return make_float2(__fdividef(num.x, den.x), __fdividef(num.y, den.y));
+}
+
 // Two output channels in one store.
 __device__ __forceinline__ void st_pair(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
 __device__ __forceinline__ void st_pair(__nv_bfloat16* p, float a, float b) {
@@ -350,6 +405,68 @@ compress_bulk_kernel(const Tin* __restrict__ kv, const Tin* __restrict__ gate, T
   // ------------------------------------------------------------------ folding
   const int c = 2 * tid;                                              // this thread's channels c, c+1
   const bool has = c < D;
+  if constexpr (kCSA && sizeof(Tin) == 2 && kCmpRows == 8) {
+    if (m == 4) {
+      // Blocks of 4 rows, two per stage (streaming starts on a block
+      // boundary): each block folds into one of two states that take turns
+      // as the current and the previous block, so an entry is one merge.
+      const __nv_bfloat16* kvb16 = reinterpret_cast<const __nv_bfloat16*>(smem) + c;
+      Blk2 s0, s1;
+      s1.reset();                                                     // the block before `first`: empty
+      const int nblk = je - first;
+      for (int k = 0; k < K; ++k) {
+        const int slot = k % kCmpStages;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(full + slot, (k / kCmpStages) & 1))) break;
+        const __nv_bfloat16* kvs = kvb16 + slot * 2 * tile_bytes / 2;
+        const __nv_bfloat16* gs = kvs + tile_bytes / 2;
+        const int q0 = 2 * k;                                         // block index within the range
+        if (has) {
+          block4_packed(s0, kvs, gs, D, 0);
+          if (first + q0 >= jb) {
+            const float2 o = csa_merge_packed(s1, s0);
+            st_pair(out + ((long long)b * Nc + first + q0) * D + c, o.x, o.y);
+          }
+          if (q0 + 1 < nblk) {
+            block4_packed(s1, kvs, gs, D, 4);
+            const float2 o = csa_merge_packed(s0, s1);               // block first + q0 + 1 >= jb
+            st_pair(out + ((long long)b * Nc + first + q0 + 1) * D + c, o.x, o.y);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty + slot);                 // this warp is done with the slot
+      }
+      return;
+    }
+  }
+  if constexpr (!kCSA && sizeof(Tin) == 2 && kCmpRows == 8) {
+    if (m % kCmpRows == 0) {
+      // HCA blocks of a multiple of 8 rows start on stage boundaries: one
+      // fold per stage, an entry every m / 8 stages.
+      const __nv_bfloat16* kvb16 = reinterpret_cast<const __nv_bfloat16*>(smem) + c;
+      const int spb = m / kCmpRows;                                   // stages per block
+      Blk2 st;
+      st.reset();
+      int blk = jb, in_blk = 0;
+      for (int k = 0; k < K; ++k) {
+        const int slot = k % kCmpStages;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(full + slot, (k / kCmpStages) & 1))) break;
+        const __nv_bfloat16* kvs = kvb16 + slot * 2 * tile_bytes / 2;
+        if (has) fold8_packed(st, kvs, kvs + tile_bytes / 2, D);
+        if (++in_blk == spb) {
+          if (has) {
+            const float2 a = upk2(st.a2), sm = upk2(st.s2);
+            st_pair(out + ((long long)b * Nc + blk) * D + c, __fdividef(a.x, sm.x), __fdividef(a.y, sm.y));
+          }
+          st.reset();
+          in_blk = 0;
+          ++blk;
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty + slot);                 // this warp is done with the slot
+      }
+      return;
+    }
+  }
   Soft2 st, prev;
   st.reset();
   prev.reset();
