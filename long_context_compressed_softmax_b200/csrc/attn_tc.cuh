@@ -828,8 +828,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
               const uint32_t pb = tc::smem_u32(s_p + sb * kAtPBytes);
               const uint32_t kb = tc::smem_u32(s_k + st * kAtKBytes);
               const int h_end = first && pv_half == 0 ? 1 : 2;   // a first PV goes one half at a time
-#pragma unroll 1
-              for (int half = pv_half; half < h_end; ++half) {
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                if (half < pv_half || half >= h_end) continue;  // unrolled: the issuing thread's hot loop
 #pragma unroll
                 for (int kstep = 0; kstep < kAtKT / 16; ++kstep) {
                   const uint64_t ad = tc::sdesc_sw128(pb + kstep * 32, 16, 1024);
