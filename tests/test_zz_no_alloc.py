@@ -142,7 +142,17 @@ r_other = run_in_current_context()
 ok(cu.cuCtxSetCurrent(primary), "cuCtxSetCurrent")                   # back to the first one
 r_back = run_in_current_context()
 ok(cu.cuCtxDestroy_v2(other), "cuCtxDestroy")
-if not (np.array_equal(r_primary, r_other) and np.array_equal(r_primary, r_back)):
+# a reset of this process's primary context (what cudaDeviceReset does): the
+# module is loaded again and the scratch array gets a new address
+ok(cu.cuCtxSetCurrent(None), "cuCtxSetCurrent")
+ok(cu.cuDevicePrimaryCtxRelease_v2(dev), "cuDevicePrimaryCtxRelease")
+ok(cu.cuDevicePrimaryCtxReset_v2(dev), "cuDevicePrimaryCtxReset")
+fresh = c_void_p()
+ok(cu.cuDevicePrimaryCtxRetain(byref(fresh), dev), "cuDevicePrimaryCtxRetain")
+ok(cu.cuCtxSetCurrent(fresh), "cuCtxSetCurrent")
+r_reset = run_in_current_context()
+if not (np.array_equal(r_primary, r_other) and np.array_equal(r_primary, r_back)
+        and np.array_equal(r_primary, r_reset)):
     raise SystemExit("results differ between contexts")
 print("contexts ok")
 '''
@@ -150,8 +160,9 @@ print("contexts ok")
 
 def test_noalloc_in_two_contexts(lcsa, tmp_path):
     """The scratch array's device address belongs to a context.  A caller that
-    switches between the primary context and a context of its own (driver API)
-    gets correct results in both, each call matching the workspace call.  Runs
+    switches between the primary context and a context of its own (driver API),
+    and then resets the primary context (as cudaDeviceReset does), gets correct
+    results each time, every call matching the workspace call.  Runs
     in a child process that uses only the driver API, so this process's
     contexts are not touched."""
     import os
