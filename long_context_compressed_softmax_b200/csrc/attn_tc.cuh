@@ -115,6 +115,12 @@ static bool attn_tc_supported(const lcsa_attn_args* a) {
   return a->dtype == LCSA_BF16 && a->H == 64 && a->D == 512 && a->R == 64;
 }
 
+// A row of zeros that the gather copies in place of an absent row or a bad
+// index (the tile's row mask already keeps such a key out of the softmax; a
+// zero row makes its value row harmless too), so that no copy needs a
+// zero-fill size or a null check.
+__device__ __align__(128) uint8_t g_zero_row[1024] = {};
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -447,7 +453,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       tc::prefetch_tmap(&tm_rotc);
       tc::prefetch_tmap(&tm_rotw);
     }
-    const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.cs);
+    const uint8_t* zero_row = g_zero_row;
     // Entry tiles that every producer fills (gathered rows, FP8 expansion)
     // make the producers leave only together, at named barrier 1.
     const bool coll = (g.sparse && !kG4) || kFp8;
@@ -690,9 +696,10 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
         const uint8_t** tab = s_tab + st * kAtKT * 2;
         if (tid < kAtKT) {
           const int kk = tid;
-          const uint8_t* rm = nullptr;
-          const uint8_t* rr = nullptr;
+          const uint8_t* rm = zero_row;
+          const uint8_t* rr = zero_row;
           float scl = 0.f;
+          bool valid = false;
           const int sl = gt * kAtKT + kk;
           if (sl < x.ks.n_c) {
             const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
@@ -701,6 +708,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
               rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
               rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
               if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
+              valid = true;
             } else {
               report(LCSA_DEV_BAD_INDEX);
             }
@@ -709,7 +717,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           tab[2 * kk + 1] = rr;
           s_scl[st * kAtKT + kk] = scl;
           // keys whose row is read: a bad index is skipped, not a zero key
-          const uint32_t vm = __ballot_sync(0xffffffffu, rm != nullptr);
+          const uint32_t vm = __ballot_sync(0xffffffffu, valid);
           if ((kk & 31) == 0) s_km[st * 2 + (kk >> 5)] = vm;
         }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
@@ -723,36 +731,40 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           for (int u = 0; u < kCodePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
-            const uint8_t* base = tab[2 * kk];
-            cp_async16(sb + kAtCodeStage + q * 16, base ? base + p * 16 : dummy, base ? 16u : 0u);
+            cp_async16(sb + kAtCodeStage + q * 16, tab[2 * kk] + p * 16, 16u);
           }
 #pragma unroll
           for (int u = 0; u < kRopePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q >> 3, c16 = q & 7;
-            const uint8_t* base = tab[2 * kk + 1];
-            cp_async16(sb + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4), base ? base + c16 * 16 : dummy,
-                       base ? 16u : 0u);
+            cp_async16(sb + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4), tab[2 * kk + 1] + c16 * 16, 16u);
           }
           cp_async_commit();
           if (pend >= 0 && !expand_pending(true)) { bad = true; break; }
           pend = st;
           continue;
         }
-        // 16-byte piece q = tid + u * kAtProdThreads of the 64 x 1 KB tile:
-        // key q / 64, piece q % 64 of its row (region = 64-dim block).
-        const uint32_t sbase = tc::smem_u32(stage);
-#pragma unroll 4
-        for (int u = 0; u < (kAtKT * 64 + kAtProdThreads - 1) / kAtProdThreads; ++u) {
-          const int q = tid + u * kAtProdThreads;
-          if (q >= kAtKT * 64) break;
-          const int kk = q >> 6, piece = q & 63;
+        // 16-byte piece `piece` (fixed per thread) of keys kk0 + 4u, u < 16:
+        // a warp copies 512 contiguous bytes of one row per instruction.  The
+        // 128B swizzle XORs bits 4-6 of the address with the key's row mod 8,
+        // which is kk0 for even u and kk0 + 4 for odd u, so every
+        // destination is one of two bases plus 1 KB per step of two keys.
+        static_assert(kAtKT * 64 == 16 * kAtProdThreads, "16 pieces per producer thread");
+        {
+          const uint32_t sbase = tc::smem_u32(stage);
+          const int piece = tid & 63, kk0 = tid >> 6;                 // kk0 < 4
           const int region = piece >> 3, c16 = piece & 7;
-          const uint32_t kb = sbase + region * kAtRegion + (c16 << 4);
+          const int sel = region == 7 ? 1 : 0;                        // rotated slice or entry row
           const int off = region == 7 ? c16 * 16 : piece * 16;
-          const uint8_t* base = tab[2 * kk + (region == 7 ? 1 : 0)];
-          const uint32_t dst = (kb + kk * 128) ^ ((uint32_t)(kk & 7) << 4);
-          cp_async16(dst, base ? base + off : dummy, base ? 16u : 0u);
+          const uint32_t kb = sbase + region * kAtRegion + (c16 << 4);
+          const uint32_t d_even = (kb ^ ((uint32_t)kk0 << 4)) + kk0 * 128;
+          const uint32_t d_odd = (kb ^ ((uint32_t)(kk0 + 4) << 4)) + (kk0 + 4) * 128;
+          const uint8_t* const* trow = tab + 2 * kk0 + sel;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            cp_async16(d_even + 1024 * j, trow[16 * j] + off, 16u);    // key kk0 + 8j
+            cp_async16(d_odd + 1024 * j, trow[16 * j + 8] + off, 16u); // key kk0 + 4 + 8j
+          }
         }
         cp_async_arrive_noinc(kv_full + st);
       }
