@@ -612,7 +612,42 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
 #pragma unroll
           for (int j = 0; j < 4; ++j) ev[j] = sl0 + j < x.ks.n_c ? __ldg(idx_row + sl0 + j) : -1;
         }
+        // Tiles copied through the row table (cp.async-gathered rows, FP8
+        // entry rows): the 64 table threads write the stage's row pointers
+        // and scales before the stage is free (only the producers read
+        // them, in this tile's copies), so the fill is off the path from
+        // the stage's release to its copies.  The row mask is read by the
+        // softmax of the stage's previous tile: it is written after the wait.
+        const bool tabt = coll && gt < x.ks.tiles_c;
+        uint32_t vm = 0;
+        if (tabt && tid < kAtKT) {
+          const uint8_t** tab = s_tab + st * kAtKT * 2;
+          const int kk = tid;
+          const uint8_t* rm = zero_row;
+          const uint8_t* rr = zero_row;
+          float scl = 0.f;
+          bool valid = false;
+          const int sl = gt * kAtKT + kk;
+          if (sl < x.ks.n_c) {
+            const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
+            if (j >= 0 && j < g.Nc) {
+              const long long e = (long long)x.b * g.Nc + j;
+              rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
+              rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
+              if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
+              valid = true;
+            } else {
+              report(LCSA_DEV_BAD_INDEX);
+            }
+          }
+          tab[2 * kk] = rm;
+          tab[2 * kk + 1] = rr;
+          if (kFp8) s_scl[st * kAtKT + kk] = scl;
+          // keys whose row is read: a bad index is skipped, not a zero key
+          vm = __ballot_sync(0xffffffffu, valid);
+        }
         if (slot >= kAtStages && waits && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
+        if (tabt && tid < kAtKT && (tid & 31) == 0) s_km[st * 2 + (tid >> 5)] = vm;
         if (*abort_flag) bad = true;
         if (gw) bad = __any_sync(0xffffffffu, bad);
         uint8_t* stage = s_k + st * kAtKBytes;
@@ -692,34 +727,9 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           }
           continue;
         }
-        // ---- gathered rows (CSA) or FP8 entry rows: per-tile row table first
-        const uint8_t** tab = s_tab + st * kAtKT * 2;
-        if (tid < kAtKT) {
-          const int kk = tid;
-          const uint8_t* rm = zero_row;
-          const uint8_t* rr = zero_row;
-          float scl = 0.f;
-          bool valid = false;
-          const int sl = gt * kAtKT + kk;
-          if (sl < x.ks.n_c) {
-            const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
-            if (j >= 0 && j < g.Nc) {
-              const long long e = (long long)x.b * g.Nc + j;
-              rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
-              rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
-              if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
-              valid = true;
-            } else {
-              report(LCSA_DEV_BAD_INDEX);
-            }
-          }
-          tab[2 * kk] = rm;
-          tab[2 * kk + 1] = rr;
-          s_scl[st * kAtKT + kk] = scl;
-          // keys whose row is read: a bad index is skipped, not a zero key
-          const uint32_t vm = __ballot_sync(0xffffffffu, valid);
-          if ((kk & 31) == 0) s_km[st * 2 + (kk >> 5)] = vm;
-        }
+        // ---- gathered rows (CSA) or FP8 entry rows: the row table (filled
+        // above) is published to every producer by named barrier 1
+        const uint8_t* const* tab = s_tab + st * kAtKT * 2;
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
         if (kFp8) {
           // FP8 entry rows: the 448 code bytes of each row land by 16-byte
