@@ -284,13 +284,15 @@ __device__ __forceinline__ void store16_v8_bits(__nv_bfloat16* p, const uint32_t
 // Epilogue of one item, executed by the 128 transition threads.  Row
 // statistics come from the softmax warps through shared memory; O -> sink,
 // normalisation, -t rotation of the rotary block -> output (or split
-// partials) straight from registers.  Piece k covers dims 32k .. 32k+31:
-// thread (h % 16) takes dims 32k .. +15 and thread (h % 16) + 16 dims
-// 32k+16 .. +31 (16x32bx2 with a 16-column offset), so each warp store
-// instruction writes 16 rows x 2 adjacent 32-byte pieces (BF16).  The TMEM
-// read of piece k+1 is in flight while piece k is scaled and stored;
-// o_free[0] (dims 0-255, the first PV half of the next item) is arrived on
-// after piece 7's read, o_free[1] after piece 15's.
+// partials) straight from registers.  Piece k covers dims 64k .. 64k+63:
+// thread (h % 16) takes dims 64k .. +31 and thread (h % 16) + 16 dims
+// 64k+32 .. +63 (16x32bx2 with a 32-column offset), so each warp store
+// instruction writes 16 rows x 2 32-byte pieces (BF16).  A wait covers
+// every TMEM load the thread has in flight, and two 32-register pieces do not
+// fit next to the rest of the kernel's registers, so the pieces are large and
+// read one at a time: eight round trips for the 512 columns.  o_free[0]
+// (dims 0-255, the first PV half of the next item) is arrived on after piece
+// 3's read, o_free[1] after piece 7's.
 __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done, uint64_t* o_free /*[2]*/,
                             uint64_t* stats_full, const float2* stats, int item, const float2* cs, long long row,
                             int split, int last, uint32_t tmem, uint32_t lane_base, int h, int half, int xt, bool ok) {
@@ -323,27 +325,30 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
                              : (g.out_bf16 ? nullptr : reinterpret_cast<float*>(P.out) + orow * 512);
   __nv_bfloat16* obf = (g.splits == 1 && g.out_bf16) ? reinterpret_cast<__nv_bfloat16*>(P.out) + orow * 512 : nullptr;
   const uint32_t taddr = tmem + lane_base + kTmO;
-  // piece k (0..15) = O columns 32k .. 32k+31: thread (h % 16) dims 32k .. +15,
-  // thread (h % 16) + 16 dims 32k+16 .. +31 (16x32bx2 with a 16-column offset)
-  uint32_t buf[2][16];
-  tc::tmem_ld_16x32bx2_x16<16>(taddr, buf[0]);
-#pragma unroll 2
-  for (int k = 0; k < 16; ++k) {
-    uint32_t* v = buf[k & 1];
-    tc::tmem_wait_ld_regs16(v);
-    if (k + 1 < 16) tc::tmem_ld_16x32bx2_x16<16>(taddr + (k + 1) * 32, buf[(k + 1) & 1]);
-    if (k == 7 || k == 15) {
+  // piece k (0..7) = O columns 64k .. 64k+63: thread (h % 16) dims 64k .. +31,
+  // thread (h % 16) + 16 dims 64k+32 .. +63
+  uint32_t v[32];
+  const f2x sc2 = pk2(scale_out, scale_out);
+#pragma unroll 1
+  for (int k = 0; k < 8; ++k) {
+    tc::tmem_ld_16x32bx2_x32<32>(taddr + k * 64, v);
+    tc::tmem_wait_ld_regs32(v);
+    if (k == 3 || k == 7) {
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(o_free + (k == 15 ? 1 : 0));  // that half of O may be overwritten
+      if (lane == 0) tc::mbar_arrive(o_free + (k == 7 ? 1 : 0));   // that half of O may be overwritten
     }
-    const int d0 = k * 32 + half * 16;                 // first output dim of this thread's piece
-    // scaled in place (FP32 bit patterns in v)
+    const int d0 = k * 64 + half * 32;                 // first output dim of this thread's piece
+    // scaled in place, two values per packed multiply (FP32 bit patterns in v)
 #pragma unroll
-    for (int q2 = 0; q2 < 16; ++q2) v[q2] = __float_as_uint(__uint_as_float(v[q2]) * scale_out);
-    if (k >= 14 && g.splits == 1) {
+    for (int q2 = 0; q2 < 32; q2 += 2) {
+      const float2 r = upk2(mul2(pk2(__uint_as_float(v[q2]), __uint_as_float(v[q2 + 1])), sc2));
+      v[q2] = __float_as_uint(r.x);
+      v[q2 + 1] = __float_as_uint(r.y);
+    }
+    if (k == 7 && g.splits == 1) {                     // dims 448 .. 511: the rotary block
 #pragma unroll
-      for (int q2 = 0; q2 < 16; q2 += 2) {
+      for (int q2 = 0; q2 < 32; q2 += 2) {
         const float2 e = cs[(d0 - 448 + q2) >> 1];      // rotate by -t: (cos, -sin)
         const float a0 = __uint_as_float(v[q2]), a1 = __uint_as_float(v[q2 + 1]);
         v[q2] = __float_as_uint(a0 * e.x + a1 * e.y);
@@ -351,11 +356,16 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
       }
     }
     if (g.out_v8) {
-      if (obf) store16_v8_bits(obf + d0, v);
-      else store16_v8_bits(of32 + d0, v);
+      if (obf) {
+        store16_v8_bits(obf + d0, v);
+        store16_v8_bits(obf + d0 + 16, v + 16);
+      } else {
+        store16_v8_bits(of32 + d0, v);
+        store16_v8_bits(of32 + d0 + 16, v + 16);
+      }
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; j += 8) {
+      for (int j = 0; j < 32; j += 8) {
         float o[8];
 #pragma unroll
         for (int q2 = 0; q2 < 8; ++q2) o[q2] = __uint_as_float(v[j + q2]);

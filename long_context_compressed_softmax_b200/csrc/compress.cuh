@@ -179,34 +179,6 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Packed FP32 pairs (the two channels of a thread): sm_100 executes add,
-// mul and fma on two FP32 lanes of a 64-bit register in one instruction.
-typedef unsigned long long f2x;
-__device__ __forceinline__ f2x pk2(float a, float b) {
-  f2x r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ float2 upk2(f2x r) {
-  float2 f;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
-  return f;
-}
-__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
-  f2x r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ f2x add2(f2x a, f2x b) {
-  f2x r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
-  f2x r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 // a BF16 pair (channel c in the low half) as a packed FP32 pair
 __device__ __forceinline__ f2x bf2f2(uint32_t w) { return pk2(bf_lo(w), bf_hi(w)); }
 
