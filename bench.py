@@ -58,7 +58,7 @@ NCU_TRAFFIC = {
     # 131.5 KB per query (Q in, BF16 output out; entry rows hit L2), scaled to
     # the stack's CSA launch of 2 x 131072 queries.
     "csa_sparse_attn": {"bytes_per_launch": 34.47e9, "file": "long_context_compressed_softmax_b200/csrc/attn_tc.cuh",
-                        "src": "c3ad10da29bfb051"},
+                        "src": "7437b5a4ca631463"},
 }
 
 def _src_hash(rel):

@@ -115,12 +115,6 @@ static bool attn_tc_supported(const lcsa_attn_args* a) {
   return a->dtype == LCSA_BF16 && a->H == 64 && a->D == 512 && a->R == 64;
 }
 
-// A row of zeros that the gather copies in place of an absent row or a bad
-// index (the tile's row mask already keeps such a key out of the softmax; a
-// zero row makes its value row harmless too), so that no copy needs a
-// zero-fill size or a null check.
-__device__ __align__(128) uint8_t g_zero_row[1024] = {};
-
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -284,15 +278,13 @@ __device__ __forceinline__ void store16_v8_bits(__nv_bfloat16* p, const uint32_t
 // Epilogue of one item, executed by the 128 transition threads.  Row
 // statistics come from the softmax warps through shared memory; O -> sink,
 // normalisation, -t rotation of the rotary block -> output (or split
-// partials) straight from registers.  Piece k covers dims 64k .. 64k+63:
-// thread (h % 16) takes dims 64k .. +31 and thread (h % 16) + 16 dims
-// 64k+32 .. +63 (16x32bx2 with a 32-column offset), so each warp store
-// instruction writes 16 rows x 2 32-byte pieces (BF16).  A wait covers
-// every TMEM load the thread has in flight, and two 32-register pieces do not
-// fit next to the rest of the kernel's registers, so the pieces are large and
-// read one at a time: eight round trips for the 512 columns.  o_free[0]
-// (dims 0-255, the first PV half of the next item) is arrived on after piece
-// 3's read, o_free[1] after piece 7's.
+// partials) straight from registers.  Piece k covers dims 32k .. 32k+31:
+// thread (h % 16) takes dims 32k .. +15 and thread (h % 16) + 16 dims
+// 32k+16 .. +31 (16x32bx2 with a 16-column offset), so each warp store
+// instruction writes 16 rows x 2 adjacent 32-byte pieces (BF16).  The TMEM
+// read of piece k+1 is in flight while piece k is scaled and stored;
+// o_free[0] (dims 0-255, the first PV half of the next item) is arrived on
+// after piece 7's read, o_free[1] after piece 15's.
 __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done, uint64_t* o_free /*[2]*/,
                             uint64_t* stats_full, const float2* stats, int item, const float2* cs, long long row,
                             int split, int last, uint32_t tmem, uint32_t lane_base, int h, int half, int xt, bool ok) {
@@ -325,30 +317,27 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
                              : (g.out_bf16 ? nullptr : reinterpret_cast<float*>(P.out) + orow * 512);
   __nv_bfloat16* obf = (g.splits == 1 && g.out_bf16) ? reinterpret_cast<__nv_bfloat16*>(P.out) + orow * 512 : nullptr;
   const uint32_t taddr = tmem + lane_base + kTmO;
-  // piece k (0..7) = O columns 64k .. 64k+63: thread (h % 16) dims 64k .. +31,
-  // thread (h % 16) + 16 dims 64k+32 .. +63
-  uint32_t v[32];
-  const f2x sc2 = pk2(scale_out, scale_out);
-#pragma unroll 1
-  for (int k = 0; k < 8; ++k) {
-    tc::tmem_ld_16x32bx2_x32<32>(taddr + k * 64, v);
-    tc::tmem_wait_ld_regs32(v);
-    if (k == 3 || k == 7) {
+  // piece k (0..15) = O columns 32k .. 32k+31: thread (h % 16) dims 32k .. +15,
+  // thread (h % 16) + 16 dims 32k+16 .. +31 (16x32bx2 with a 16-column offset)
+  uint32_t buf[2][16];
+  tc::tmem_ld_16x32bx2_x16<16>(taddr, buf[0]);
+#pragma unroll 2
+  for (int k = 0; k < 16; ++k) {
+    uint32_t* v = buf[k & 1];
+    tc::tmem_wait_ld_regs16(v);
+    if (k + 1 < 16) tc::tmem_ld_16x32bx2_x16<16>(taddr + (k + 1) * 32, buf[(k + 1) & 1]);
+    if (k == 7 || k == 15) {
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(o_free + (k == 7 ? 1 : 0));   // that half of O may be overwritten
+      if (lane == 0) tc::mbar_arrive(o_free + (k == 15 ? 1 : 0));  // that half of O may be overwritten
     }
-    const int d0 = k * 64 + half * 32;                 // first output dim of this thread's piece
-    // scaled in place, two values per packed multiply (FP32 bit patterns in v)
+    const int d0 = k * 32 + half * 16;                 // first output dim of this thread's piece
+    // scaled in place (FP32 bit patterns in v)
 #pragma unroll
-    for (int q2 = 0; q2 < 32; q2 += 2) {
-      const float2 r = upk2(mul2(pk2(__uint_as_float(v[q2]), __uint_as_float(v[q2 + 1])), sc2));
-      v[q2] = __float_as_uint(r.x);
-      v[q2 + 1] = __float_as_uint(r.y);
-    }
-    if (k == 7 && g.splits == 1) {                     // dims 448 .. 511: the rotary block
+    for (int q2 = 0; q2 < 16; ++q2) v[q2] = __float_as_uint(__uint_as_float(v[q2]) * scale_out);
+    if (k >= 14 && g.splits == 1) {
 #pragma unroll
-      for (int q2 = 0; q2 < 32; q2 += 2) {
+      for (int q2 = 0; q2 < 16; q2 += 2) {
         const float2 e = cs[(d0 - 448 + q2) >> 1];      // rotate by -t: (cos, -sin)
         const float a0 = __uint_as_float(v[q2]), a1 = __uint_as_float(v[q2 + 1]);
         v[q2] = __float_as_uint(a0 * e.x + a1 * e.y);
@@ -356,16 +345,11 @@ __device__ bool at_epilogue(const AtGeom& g, const AtPtrs& P, uint64_t* pv_done,
       }
     }
     if (g.out_v8) {
-      if (obf) {
-        store16_v8_bits(obf + d0, v);
-        store16_v8_bits(obf + d0 + 16, v + 16);
-      } else {
-        store16_v8_bits(of32 + d0, v);
-        store16_v8_bits(of32 + d0 + 16, v + 16);
-      }
+      if (obf) store16_v8_bits(obf + d0, v);
+      else store16_v8_bits(of32 + d0, v);
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
+      for (int j = 0; j < 16; j += 8) {
         float o[8];
 #pragma unroll
         for (int q2 = 0; q2 < 8; ++q2) o[q2] = __uint_as_float(v[j + q2]);
@@ -463,7 +447,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
       tc::prefetch_tmap(&tm_rotc);
       tc::prefetch_tmap(&tm_rotw);
     }
-    const uint8_t* zero_row = g_zero_row;
+    const uint8_t* dummy = reinterpret_cast<const uint8_t*>(P.cs);
     // Entry tiles that every producer fills (gathered rows, FP8 expansion)
     // make the producers leave only together, at named barrier 1.
     const bool coll = (g.sparse && !kG4) || kFp8;
@@ -622,42 +606,7 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
 #pragma unroll
           for (int j = 0; j < 4; ++j) ev[j] = sl0 + j < x.ks.n_c ? __ldg(idx_row + sl0 + j) : -1;
         }
-        // Tiles copied through the row table (cp.async-gathered rows, FP8
-        // entry rows): the 64 table threads write the stage's row pointers
-        // and scales before the stage is free (only the producers read
-        // them, in this tile's copies), so the fill is off the path from
-        // the stage's release to its copies.  The row mask is read by the
-        // softmax of the stage's previous tile: it is written after the wait.
-        const bool tabt = coll && gt < x.ks.tiles_c;
-        uint32_t vm = 0;
-        if (tabt && tid < kAtKT) {
-          const uint8_t** tab = s_tab + st * kAtKT * 2;
-          const int kk = tid;
-          const uint8_t* rm = zero_row;
-          const uint8_t* rr = zero_row;
-          float scl = 0.f;
-          bool valid = false;
-          const int sl = gt * kAtKT + kk;
-          if (sl < x.ks.n_c) {
-            const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
-            if (j >= 0 && j < g.Nc) {
-              const long long e = (long long)x.b * g.Nc + j;
-              rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
-              rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
-              if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
-              valid = true;
-            } else {
-              report(LCSA_DEV_BAD_INDEX);
-            }
-          }
-          tab[2 * kk] = rm;
-          tab[2 * kk + 1] = rr;
-          if (kFp8) s_scl[st * kAtKT + kk] = scl;
-          // keys whose row is read: a bad index is skipped, not a zero key
-          vm = __ballot_sync(0xffffffffu, valid);
-        }
         if (slot >= kAtStages && waits && !tc::mbar_wait(kv_empty + st, ((slot / kAtStages) - 1) & 1)) bad = true;
-        if (tabt && tid < kAtKT && (tid & 31) == 0) s_km[st * 2 + (tid >> 5)] = vm;
         if (*abort_flag) bad = true;
         if (gw) bad = __any_sync(0xffffffffu, bad);
         uint8_t* stage = s_k + st * kAtKBytes;
@@ -737,9 +686,32 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           }
           continue;
         }
-        // ---- gathered rows (CSA) or FP8 entry rows: the row table (filled
-        // above) is published to every producer by named barrier 1
-        const uint8_t* const* tab = s_tab + st * kAtKT * 2;
+        // ---- gathered rows (CSA) or FP8 entry rows: per-tile row table first
+        const uint8_t** tab = s_tab + st * kAtKT * 2;
+        if (tid < kAtKT) {
+          const int kk = tid;
+          const uint8_t* rm = nullptr;
+          const uint8_t* rr = nullptr;
+          float scl = 0.f;
+          const int sl = gt * kAtKT + kk;
+          if (sl < x.ks.n_c) {
+            const int j = g.sparse ? s_idx[sl - slot0] : sl;      // dense: slot sl holds entry sl
+            if (j >= 0 && j < g.Nc) {
+              const long long e = (long long)x.b * g.Nc + j;
+              rm = kFp8 ? P.c8 + e * kAtCodeBytes : reinterpret_cast<const uint8_t*>(P.ckv + e * 512);
+              rr = reinterpret_cast<const uint8_t*>(P.rot_c + (g.rot_slot ? (x.row * g.k + sl) : e) * 64);
+              if (kFp8) scl = ldexpf(1.f, (int)__ldg(P.c8s + e) - 127);
+            } else {
+              report(LCSA_DEV_BAD_INDEX);
+            }
+          }
+          tab[2 * kk] = rm;
+          tab[2 * kk + 1] = rr;
+          s_scl[st * kAtKT + kk] = scl;
+          // keys whose row is read: a bad index is skipped, not a zero key
+          const uint32_t vm = __ballot_sync(0xffffffffu, rm != nullptr);
+          if ((kk & 31) == 0) s_km[st * 2 + (kk >> 5)] = vm;
+        }
         if (!tc::bar_and(1, kAtProdThreads, !bad)) { bad = true; break; }
         if (kFp8) {
           // FP8 entry rows: the 448 code bytes of each row land by 16-byte
@@ -751,40 +723,36 @@ attn_tc_kernel(AtPtrs P, AtGeom g, const __grid_constant__ CUtensorMap tm_q, con
           for (int u = 0; u < kCodePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q / (kAtCodeBytes / 16), p = q - kk * (kAtCodeBytes / 16);
-            cp_async16(sb + kAtCodeStage + q * 16, tab[2 * kk] + p * 16, 16u);
+            const uint8_t* base = tab[2 * kk];
+            cp_async16(sb + kAtCodeStage + q * 16, base ? base + p * 16 : dummy, base ? 16u : 0u);
           }
 #pragma unroll
           for (int u = 0; u < kRopePer; ++u) {
             const int q = tid + u * kAtProdThreads;
             const int kk = q >> 3, c16 = q & 7;
-            cp_async16(sb + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4), tab[2 * kk + 1] + c16 * 16, 16u);
+            const uint8_t* base = tab[2 * kk + 1];
+            cp_async16(sb + 7 * kAtRegion + kk * 128 + ((c16 ^ (kk & 7)) << 4), base ? base + c16 * 16 : dummy,
+                       base ? 16u : 0u);
           }
           cp_async_commit();
           if (pend >= 0 && !expand_pending(true)) { bad = true; break; }
           pend = st;
           continue;
         }
-        // 16-byte piece `piece` (fixed per thread) of keys kk0 + 4u, u < 16:
-        // a warp copies 512 contiguous bytes of one row per instruction.  The
-        // 128B swizzle XORs bits 4-6 of the address with the key's row mod 8,
-        // which is kk0 for even u and kk0 + 4 for odd u, so every
-        // destination is one of two bases plus 1 KB per step of two keys.
-        static_assert(kAtKT * 64 == 16 * kAtProdThreads, "16 pieces per producer thread");
-        {
-          const uint32_t sbase = tc::smem_u32(stage);
-          const int piece = tid & 63, kk0 = tid >> 6;                 // kk0 < 4
+        // 16-byte piece q = tid + u * kAtProdThreads of the 64 x 1 KB tile:
+        // key q / 64, piece q % 64 of its row (region = 64-dim block).
+        const uint32_t sbase = tc::smem_u32(stage);
+#pragma unroll 4
+        for (int u = 0; u < (kAtKT * 64 + kAtProdThreads - 1) / kAtProdThreads; ++u) {
+          const int q = tid + u * kAtProdThreads;
+          if (q >= kAtKT * 64) break;
+          const int kk = q >> 6, piece = q & 63;
           const int region = piece >> 3, c16 = piece & 7;
-          const int sel = region == 7 ? 1 : 0;                        // rotated slice or entry row
-          const int off = region == 7 ? c16 * 16 : piece * 16;
           const uint32_t kb = sbase + region * kAtRegion + (c16 << 4);
-          const uint32_t d_even = (kb ^ ((uint32_t)kk0 << 4)) + kk0 * 128;
-          const uint32_t d_odd = (kb ^ ((uint32_t)(kk0 + 4) << 4)) + (kk0 + 4) * 128;
-          const uint8_t* const* trow = tab + 2 * kk0 + sel;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            cp_async16(d_even + 1024 * j, trow[16 * j] + off, 16u);    // key kk0 + 8j
-            cp_async16(d_odd + 1024 * j, trow[16 * j + 8] + off, 16u); // key kk0 + 4 + 8j
-          }
+          const int off = region == 7 ? c16 * 16 : piece * 16;
+          const uint8_t* base = tab[2 * kk + (region == 7 ? 1 : 0)];
+          const uint32_t dst = (kb + kk * 128) ^ ((uint32_t)(kk & 7) << 4);
+          cp_async16(dst, base ? base + off : dummy, base ? 16u : 0u);
         }
         cp_async_arrive_noinc(kv_full + st);
       }

@@ -176,22 +176,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_consta
       for (int qq = 0; qq < 2; ++qq) {
         const int q = 2 * half + qq;
         if (q < rows && j < g.Nc) {
-          // w_h relu(x_h) summed over the 64 heads: packed pairs of heads in
-          // four independent accumulators (a short dependency chain), the
-          // weights four at a time from shared memory
-          const float4* wq4 = reinterpret_cast<const float4*>(s_w + q * 64);
-          f2x acc[4] = {0ull, 0ull, 0ull, 0ull};
+          const float* wq = s_w + q * 64;
+          float s = 0.f;
 #pragma unroll
-          for (int h4 = 0; h4 < 16; ++h4) {
-            const float4 wv = wq4[h4];
-            const uint32_t* x = v[qq] + 4 * h4;
-            const f2x r01 = pk2(fmaxf(__uint_as_float(x[0]), 0.f), fmaxf(__uint_as_float(x[1]), 0.f));
-            const f2x r23 = pk2(fmaxf(__uint_as_float(x[2]), 0.f), fmaxf(__uint_as_float(x[3]), 0.f));
-            acc[(2 * h4) & 3] = fma2(pk2(wv.x, wv.y), r01, acc[(2 * h4) & 3]);
-            acc[(2 * h4 + 1) & 3] = fma2(pk2(wv.z, wv.w), r23, acc[(2 * h4 + 1) & 3]);
-          }
-          const float2 s01 = upk2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])));
-          const float s = s01.x + s01.y;
+          for (int h = 0; h < 64; ++h) s = fmaf(wq[h], fmaxf(__uint_as_float(v[qq][h]), 0.f), s);
           const long long srow = (long long)bl * g.ni + (i_first - g.i0) + q;
           scores[srow * g.Nc + j] = s;
         }
