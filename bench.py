@@ -54,10 +54,10 @@ SPEC_HBM_GBS = 7700.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # kernel source it was taken on; a changed source reports null.
 NCU_TRAFFIC = {
-    # csa_prefill_8k capture (8192 queries): 584.8 MB read + 492.4 MB written =
-    # 131.5 KB per query (Q in, BF16 output out; entry rows hit L2), scaled to
+    # csa_prefill_8k capture (8192 queries): 585.1 MB read + 493.5 MB written =
+    # 131.7 KB per query (Q in, BF16 output out; entry rows hit L2), scaled to
     # the stack's CSA launch of 2 x 131072 queries.
-    "csa_sparse_attn": {"bytes_per_launch": 34.47e9, "file": "long_context_compressed_softmax_b200/csrc/attn_tc.cuh",
+    "csa_sparse_attn": {"bytes_per_launch": 34.51e9, "file": "long_context_compressed_softmax_b200/csrc/attn_tc.cuh",
                         "src": "7437b5a4ca631463"},
 }
 
