@@ -103,6 +103,17 @@ void lcsa_test_withhold_stage(int chunk);
  * after it.  Any other value: LCSA_ERR_INVALID_ARG. */
 lcsa_status lcsa_set_attn_gather(int mode);
 
+/* How lcsa_indexer_topk_mxfp4 feeds its MXFP4 keys to the tensor cores
+ * (the pages give the FP4 QK path, [p2] "FP4 Quantization-Aware Training",
+ * not its kernel): mode 1 (default) hands query groups of one or two rows
+ * (decode) to a block-scaled MMA that reads the E2M1 codes and their UE8M0
+ * block scales as they are; mode 0 stages every key as FP8 E4M3 relative to
+ * its largest block scale first.  Scores agree to FP32 rounding order (and
+ * mode 1 stays exact where mode 0 rounds a block more than 2^13 below its
+ * entry's largest).  Process-wide; applies to calls issued after it.  Any
+ * other value: LCSA_ERR_INVALID_ARG. */
+lcsa_status lcsa_set_fp4_mma(int mode);
+
 /* ------------------------------------------------------------------------
  * KV compression ([p2] CSA Step 1: m consecutive tokens merged into one entry
  * with learned softmax weights; [p2] HCA: m' = 128 tokens per entry; [p3]
@@ -244,10 +255,14 @@ lcsa_status lcsa_quantize_mxfp4(const void* x, int64_t rows, int cols, lcsa_dtyp
  * MXFP4 values: the keys come quantised (the indexer-key cache in MXFP4,
  * e.g. written by lcsa_quantize_mxfp4 with cols = D_I), the BF16 queries are
  * quantised per (row, head) inside the call.  The products of the
- * dequantised values are exact and accumulate in FP32 (the kernel stages
- * each key entry and query head as FP8 E4M3 relative to its largest block
- * scale, exact while the entry's block scales lie within 2^13 of it; a block
- * further below rounds to the E4M3 grid).
+ * dequantised values are exact and accumulate in FP32.  Each query head is
+ * staged as FP8 E4M3 relative to its largest block scale, exact while its
+ * block scales lie within 2^13 of it (a block further below rounds to the
+ * E4M3 grid).  Keys: with one or two query rows per sequence (decode) the
+ * tensor cores read the E2M1 codes with their block scales (exact for any
+ * scales; see lcsa_set_fp4_mma); with more rows they are staged like the
+ * queries.  The block-scaled path needs k_codes 32-byte aligned (any
+ * allocation from the CUDA allocators is); 16-byte aligned codes are staged.
  *
  *   q_idx     [B,Tq,64,128] BF16, 16-byte aligned; finite values
  *   w         [B,Tq,64] FP32

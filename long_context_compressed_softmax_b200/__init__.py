@@ -35,7 +35,7 @@ EXPORTED = [
     "lcsa_grouped_out_proj_workspace", "lcsa_grouped_out_proj",
     "lcsa_attn_workspace", "lcsa_csa_sparse_attn", "lcsa_hca_dense_attn", "lcsa_attn_uses_tensor_cores",
     "lcsa_quantize_entries_fp8", "lcsa_csa_sparse_attn_fp8", "lcsa_hca_dense_attn_fp8",
-    "lcsa_set_wait_limit_ns", "lcsa_test_withhold_stage", "lcsa_set_attn_gather",
+    "lcsa_set_wait_limit_ns", "lcsa_test_withhold_stage", "lcsa_set_attn_gather", "lcsa_set_fp4_mma",
 ]
 
 
@@ -117,6 +117,7 @@ _sig = {
     "lcsa_set_wait_limit_ns": (_i, [ctypes.c_uint64]),
     "lcsa_test_withhold_stage": (None, [_i]),
     "lcsa_set_attn_gather": (_i, [_i]),
+    "lcsa_set_fp4_mma": (_i, [_i]),
     "lcsa_csa_sparse_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
     "lcsa_hca_dense_attn_fp8": (_i, [ctypes.POINTER(AttnArgs), ctypes.POINTER(Fp8Entries), _vp, _sz, _vp]),
 }
@@ -176,6 +177,11 @@ def set_wait_limit_ns(ns: int) -> None:
 def set_attn_gather(mode: int) -> None:
     """CSA row staging on BF16 entries: 0 = cp.async (default), 1 = TMA tile::gather4."""
     _check(_lib.lcsa_set_attn_gather(int(mode)), "set_attn_gather")
+
+
+def set_fp4_mma(mode: int) -> None:
+    """MXFP4 indexer keys: 1 = block-scaled MMA on the codes for 1-2 row groups (default), 0 = E4M3 staging."""
+    _check(_lib.lcsa_set_fp4_mma(int(mode)), "set_fp4_mma")
 
 
 def get_device_status() -> int:

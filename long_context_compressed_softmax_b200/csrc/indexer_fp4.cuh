@@ -340,14 +340,311 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
   }
 }
 
+// ---------------------------------------------------------------------------
+// Block-scaled variant for query groups of one or two rows (decode): the
+// codes go to the tensor cores as they are.  Per 128-entry tile:
+//   TMA        64-byte code rows -> 128-byte swizzled lines, each run of 16
+//              codes padded to 16 bytes (the 4-bit operand layout of
+//              tcgen05), 12-deep ring; 8 KB of HBM per tile
+//   scales     8 warps (two per TMEM lane quarter, alternate tiles) write
+//              each entry's four UE8M0 block scales to TMEM; each loads the
+//              scale words of its next 8 tiles ahead (16 tiles of
+//              lookahead: the words come from DRAM, whose latency under
+//              this load is several tiles long)
+//   MMA        tcgen05 kind::mxf8f6f4 with block scaling: A = E2M1 keys with
+//              their scales, B = E4M3 queries with scale 1, K = 32 per
+//              instruction (one scale per row), FP32 accumulate, so every
+//              product E2M1 x 2^(X_b - 127) x E4M3 is exact whatever the
+//              spread of an entry's block scales
+//   epilogue   8 warps, the two halves take alternate tiles (as the E4M3 path
+//              with 1-2 rows), no entry factor
+// TMEM: accumulators in columns [0, 384) (six of 64 or three of 128), the B
+// scales in [384, 400), seven A-scale buffers of 16 columns from 400.  A
+// scale buffer holds one group of 4 columns per K-step; the MMA reads the
+// scale of row m at lane m, column (group + m / 32), so each lane writes its
+// own entry's scale of block k in every column of group k, in every byte.
+// Warp roles (576 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
+// 2-9 epilogue, 10-17 scale writers.  Waits are bounded as in the E4M3 path.
+// 1: one- and two-row rectangles take the block-scaled kernel (default);
+// 0: every rectangle takes the E4M3 staging kernel (for comparison).
+inline std::atomic<int>& fp4_mma_mode_ref() {
+  static std::atomic<int> mode{1};
+  return mode;
+}
+inline int fp4_mma_mode() { return fp4_mma_mode_ref().load(std::memory_order_relaxed); }
+
+constexpr int kMxStages = 12;
+constexpr int kMxSf = 7;                       // A-scale buffers in TMEM
+constexpr int kMxScaleWarp0 = 10;
+constexpr int kMxThreads = (kMxScaleWarp0 + 8) * 32;          // 576
+constexpr int kMxSfAhead = 8;                  // scale words in flight per writer warp (its own tiles)
+constexpr uint32_t kMxQBytes = 128 * 128;      // up to 2 query rows x 64 heads x 128 E4M3
+constexpr uint32_t kMxCBytes = kIxTileE * 128; // one unpacked code tile in shared memory
+constexpr uint32_t kMxCTx = kIxTileE * 64;     // bytes the copy of a tile credits (packed)
+constexpr uint32_t kMxAccCols = 384;
+constexpr uint32_t kMxSfB = 384;               // B scales (all 1)
+constexpr uint32_t kMxSfA = 400;               // A-scale buffers
+static_assert(kMxSfA + 16 * kMxSf <= 512, "TMEM columns of the block-scaled indexer");
+constexpr int kMxBars = 1 + 2 * kMxStages + 2 * kMxSf + 2 * 6;
+constexpr size_t kMxSmem = 1024 + kMxQBytes + kMxStages * kMxCBytes + kIxRows * 64 * 4 + kMxBars * 8;
+static_assert(kMxSmem + 64 <= 232448, "shared memory of the block-scaled indexer kernel");
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A E2M1 (5),
+// B E4M3 (0), both K-major, UE8M0 scales (bit 23), M = 128.  Bits 4-5 (the
+// B scale-factor byte) are 1: the B scales are 1 in every byte.
+__host__ __device__ __forceinline__ uint32_t idesc_mx_e2m1_e4m3(int N) {
+  uint32_t d = 0;
+  d |= 1u << 4;
+  d |= 5u << 7;
+  d |= (uint32_t)((N >> 3) & 0x3F) << 17;
+  d |= 1u << 23;
+  d |= (uint32_t)(128 >> 4) << 24;
+  return d;
+}
+__device__ __forceinline__ void mma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kMxThreads, 1)
+indexer_mx_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap c_map,
+                  const uint32_t* __restrict__ k_scales, const float* __restrict__ w8, float* __restrict__ scores,
+                  IxGeom g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_q = smem;
+  uint8_t* s_c = s_q + kMxQBytes;
+  float* s_w = reinterpret_cast<float*>(s_c + kMxStages * kMxCBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + kIxRows * 64);
+  uint64_t* q_full = bars;
+  uint64_t* c_full = bars + 1;
+  uint64_t* c_empty = c_full + kMxStages;
+  uint64_t* sf_full = c_empty + kMxStages;
+  uint64_t* sf_empty = sf_full + kMxSf;
+  uint64_t* acc_full = sf_empty + kMxSf;
+  uint64_t* acc_empty = acc_full + 6;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work unit (as the E4M3 path; one group per sequence, 1-2 rows)
+  const int n_groups = g.nb * g.gps;
+  const int grp = n_groups - 1 - (int)blockIdx.x;
+  const int split = blockIdx.y;
+  const int bl = grp / g.gps;
+  const int b = g.b0 + bl;
+  const int gi = grp - bl * g.gps;
+  const int i_first = g.i0 + gi * kIxRows;
+  int rows = g.i0 + g.ni - i_first;
+  rows = rows < 2 ? rows : 2;
+  long long nv = (g.q_pos0 + i_first + rows - 1) / g.m;
+  if (nv > g.Nc) nv = g.Nc;
+  const int tiles_all = (int)((nv + kIxTileE - 1) / kIxTileE);
+  const int per_split = (tiles_all + g.splits - 1) / g.splits;
+  const int t_begin = split * per_split;
+  int t_end = t_begin + per_split;
+  t_end = t_end < tiles_all ? t_end : tiles_all;
+  const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
+  if (n_tiles == 0) return;
+  const long long rect_row = (long long)bl * g.ni + (i_first - g.i0);
+  const int n_acc = rows == 1 ? 6 : 3;
+  const uint32_t acc_cols = 64u * (uint32_t)rows;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int s = 0; s < kMxStages; ++s) { tc::mbar_init(c_full + s, 1); tc::mbar_init(c_empty + s, 1); }
+    for (int s = 0; s < kMxSf; ++s) { tc::mbar_init(sf_full + s, 4); tc::mbar_init(sf_empty + s, 1); }
+    for (int a = 0; a < 6; ++a) { tc::mbar_init(acc_full + a, 1); tc::mbar_init(acc_empty + a, 4); }
+    tc::fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 1) { tc::tmem_alloc(&s_tmem, 512); tc::tmem_relinquish(); }
+  for (int e = threadIdx.x; e < kIxRows * 64; e += kMxThreads) {
+    const int q = e >> 6;
+    s_w[e] = q < rows ? w8[(rect_row + q) * 64 + (e & 63)] : 0.f;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+  const long long ent0 = (long long)b * g.Nc;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&q_map);
+      tc::prefetch_tmap(&c_map);
+      tc::mbar_arrive_expect_tx(q_full, kMxQBytes);
+      tc::tma_load_2d(s_q, &q_map, q_full, 0, (int)(rect_row * 64));
+      int issued = 0;
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % kMxStages, r = n / kMxStages;
+        if (r > 0 && !tc::mbar_wait(c_empty + s, (r - 1) & 1)) { *abort_flag = 1; break; }
+        if (*abort_flag) break;
+        tc::mbar_arrive_expect_tx(c_full + s, kMxCTx);
+        tc::tma_load_2d(s_c + s * kMxCBytes, &c_map, c_full + s, 0,
+                        (int)(ent0 + (long long)(t_begin + n) * kIxTileE));
+        ++issued;
+      }
+      for (int n = issued - kMxStages > 0 ? issued - kMxStages : 0; n < issued; ++n)
+        tc::mbar_wait(c_full + n % kMxStages, (n / kMxStages) & 1);
+      tc::mbar_wait(q_full, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      const uint32_t idesc = idesc_mx_e2m1_e4m3(64 * rows);
+      bool ok = tc::mbar_wait(q_full, 0);
+      const uint32_t b_base = tc::smem_u32(s_q);
+      for (int n = 0; ok && n < n_tiles; ++n) {
+        const int s = n % kMxStages, rs = n / kMxStages;
+        const int f = n % kMxSf, rf = n / kMxSf;
+        const int a = n % n_acc, ra = n / n_acc;
+        if (*abort_flag) break;
+        if (!tc::mbar_wait_spin(c_full + s, rs & 1)) { ok = false; break; }
+        if (!tc::mbar_wait_spin(sf_full + f, rf & 1)) { ok = false; break; }
+        if (ra > 0 && !tc::mbar_wait_spin(acc_empty + a, (ra - 1) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t a_base = tc::smem_u32(s_c + s * kMxCBytes);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = tc::sdesc_sw128(a_base + ks * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(b_base + ks * 32, 16, 1024);
+          mma_mx_ss(tmem + (uint32_t)a * acc_cols, ad, bd, idesc, tmem + kMxSfA + 16u * (uint32_t)f + 4u * ks,
+                    tmem + kMxSfB, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(c_empty + s);
+        tc::mma_commit(sf_empty + f);
+        tc::mma_commit(acc_full + a);
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp < kMxScaleWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;                 // 0..7
+    const int quarter = warp & 3;           // TMEM lanes [32*quarter, 32*quarter+32)
+    const int half = e >> 2;                // takes the tiles n with n % 2 == half
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    for (int n = half; n < n_tiles; n += 2) {
+      const int a = n % n_acc, ra = n / n_acc;
+      const long long j = (long long)(t_begin + n) * kIxTileE + quarter * 32 + lane;
+      bool ok = !*abort_flag && tc::mbar_wait(acc_full + a, ra & 1);
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      tc::tc_fence_after();
+      float sc[2] = {0.f, 0.f};
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        if (qq < rows) {
+          const uint32_t col = tmem + lane_addr + (uint32_t)a * acc_cols + (uint32_t)(qq * 64);
+          const uint32_t wq = tc::smem_u32(s_w + qq * 64);
+          // w relu(x) = (w/2) x + (w/2) |x| (the prepared weights carry the 1/2)
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int hb = 0; hb < 64; hb += 32) {
+            uint32_t v[32];
+            tc::tmem_ld32(col + hb, v);
+            tc::tmem_wait_ld();
+            if (qq == rows - 1 && hb == 32) {      // accumulator read out: hand it back to the MMA warp
+              tc::tc_fence_before();
+              __syncwarp();
+              if (lane == 0) tc::mbar_arrive(acc_empty + a);
+            }
+#pragma unroll
+            for (int h = 0; h < 32; h += 4) {
+              const float4 w4 = tc::lds128f(wq + (hb + h) * 4);
+              const float x0 = __uint_as_float(v[h]), x1 = __uint_as_float(v[h + 1]);
+              const float x2 = __uint_as_float(v[h + 2]), x3 = __uint_as_float(v[h + 3]);
+              acc[0] = fmaf(w4.x, x0, acc[0]); acc[4] = fmaf(w4.x, fabsf(x0), acc[4]);
+              acc[1] = fmaf(w4.y, x1, acc[1]); acc[5] = fmaf(w4.y, fabsf(x1), acc[5]);
+              acc[2] = fmaf(w4.z, x2, acc[2]); acc[6] = fmaf(w4.z, fabsf(x2), acc[6]);
+              acc[3] = fmaf(w4.w, x3, acc[3]); acc[7] = fmaf(w4.w, fabsf(x3), acc[7]);
+            }
+          }
+          sc[qq] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
+        }
+      }
+      if (j < g.Nc) {
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq)
+          if (qq < rows) scores[(rect_row + qq) * g.Nc + j] = sc[qq];
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ scale writers
+    // lane l of this warp owns TMEM lane 32 * quarter + l = entry row of the
+    // tiles n with n % 2 == half
+    const int quarter = warp & 3;
+    const int half = (warp - kMxScaleWarp0) >> 2;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    auto scale_word = [&](int n) -> uint32_t {
+      const long long j = (long long)(t_begin + n) * kIxTileE + quarter * 32 + lane;
+      return n < n_tiles && j < g.Nc ? __ldg(k_scales + ent0 + j) : 0x7F7F7F7Fu;
+    };
+    uint32_t r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = 0x7F7F7F7Fu;
+    if (half == 0) tc::tmem_st16(tmem + lane_addr + kMxSfB, r);   // B scales: 1 (UE8M0 127) in every byte
+    // words of this warp's next kMxSfAhead tiles (a ring of registers, static
+    // indices: the loop below is unrolled by its length)
+    uint32_t ring[kMxSfAhead];
+#pragma unroll
+    for (int u = 0; u < kMxSfAhead; ++u) ring[u] = scale_word(half + 2 * u);
+    bool live = true;
+    for (int n0 = half; live && n0 < n_tiles; n0 += 2 * kMxSfAhead) {
+#pragma unroll
+    for (int u = 0; u < kMxSfAhead; ++u) {
+      const int n = n0 + 2 * u;
+      if (n >= n_tiles) { live = false; break; }
+      const int f = n % kMxSf, rf = n / kMxSf;
+      const uint32_t sw = ring[u];
+      ring[u] = scale_word(n + 2 * kMxSfAhead);
+      bool ok = !*abort_flag && (rf == 0 || tc::mbar_wait(sf_empty + f, (rf - 1) & 1));
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; live = false; break; }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t x = ((sw >> (8 * k)) & 0xFFu) * 0x01010101u;
+        r[4 * k] = x; r[4 * k + 1] = x; r[4 * k + 2] = x; r[4 * k + 3] = x;
+      }
+      tc::tmem_st16(tmem + lane_addr + kMxSfA + 16u * (uint32_t)f, r);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(sf_full + f);
+    }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
 // Scores of the chunk rectangle (sequences [b0, b0+nb), rows [i0, i0+ni)),
 // rows laid out [nb][ni][Nc].  q8 / w8: the prepared queries of the rectangle.
+// Calls of one or two rows per sequence (few_rows) take the block-scaled
+// kernel when the codes are 32-byte aligned, others the E4M3 staging kernel.
 static cudaError_t launch_indexer_fp4_rect(const uint8_t* k_codes, const uint8_t* k_scales, int B, int Nc,
                                            long long q_pos0, int m, const uint8_t* q8, const float* w8,
-                                           float* scores, int b0, int nb, int i0, int ni, cudaStream_t st) {
+                                           float* scores, int b0, int nb, int i0, int ni, bool few_rows,
+                                           cudaStream_t st) {
   CUtensorMap qm, cm;
-  if (!make_tmap_2d(&qm, q8, 1, (uint64_t)nb * ni * 64, 128, 128, 128, 256)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&cm, k_codes, 1, (uint64_t)B * Nc, 64, 64, 64, kIxTileE, false)) return cudaErrorInvalidValue;
+  const bool mx = few_rows && ni <= 2 && fp4_mma_mode() == 1 &&
+                  make_tmap_u4x128_2d(&cm, k_codes, (uint64_t)B * Nc, kIxTileE);
+  if (mx) {
+    if (!make_tmap_2d(&qm, q8, 1, (uint64_t)nb * ni * 64, 128, 128, 128, 128)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_2d(&qm, q8, 1, (uint64_t)nb * ni * 64, 128, 128, 128, 256)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&cm, k_codes, 1, (uint64_t)B * Nc, 64, 64, 64, kIxTileE, false)) return cudaErrorInvalidValue;
+  }
   IxGeom g;
   g.Tq = 0; g.Nc = Nc; g.H = 64;
   g.b0 = b0; g.nb = nb; g.i0 = i0; g.ni = ni;
@@ -359,11 +656,18 @@ static cudaError_t launch_indexer_fp4_rect(const uint8_t* k_codes, const uint8_t
   const int tiles = (int)((nv + kIxTileE - 1) / kIxTileE);
   const int splits = indexer_splits(n_groups, tiles);
   g.splits = splits;
-  cudaError_t e = cudaFuncSetAttribute(indexer_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem);
-  if (e != cudaSuccess) return e;
   dim3 grid(n_groups, splits);
-  indexer_fp4_kernel<<<grid, kI4Threads, kI4Smem, st>>>(qm, cm, reinterpret_cast<const uint32_t*>(k_scales), w8,
-                                                         scores, g);
+  if (mx) {
+    cudaError_t e = cudaFuncSetAttribute(indexer_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMxSmem);
+    if (e != cudaSuccess) return e;
+    indexer_mx_kernel<<<grid, kMxThreads, kMxSmem, st>>>(qm, cm, reinterpret_cast<const uint32_t*>(k_scales), w8,
+                                                          scores, g);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(indexer_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem);
+    if (e != cudaSuccess) return e;
+    indexer_fp4_kernel<<<grid, kI4Threads, kI4Smem, st>>>(qm, cm, reinterpret_cast<const uint32_t*>(k_scales), w8,
+                                                           scores, g);
+  }
   count_launch();
   return cudaGetLastError();
 }

@@ -256,6 +256,12 @@ lcsa_status lcsa_set_attn_gather(int mode) {
   return LCSA_OK;
 }
 
+lcsa_status lcsa_set_fp4_mma(int mode) {
+  if (mode != 0 && mode != 1) return LCSA_ERR_INVALID_ARG;
+  fp4_mma_mode_ref().store(mode);
+  return LCSA_OK;
+}
+
 lcsa_status lcsa_csa_compress(const void* kv, const void* gate, int gate_per_channel, int B, int T, int D, int m,
                               lcsa_dtype dtype, const float* rms_weight, float rms_eps, void* out,
                               lcsa_dtype out_dtype, void* stream) {
@@ -400,8 +406,10 @@ lcsa_status lcsa_indexer_topk_mxfp4(const lcsa_indexer_mxfp4_args* a, void* work
             (const __nv_bfloat16*)a->q_idx, a->w, a->Tq, b0, nb, i0, ni, q8, w8);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+        // the kernel follows the call's row count, not the chunking, so a
+        // smaller workspace gives the same scores
         return launch_indexer_fp4_rect(a->k_codes, a->k_scales, a->B, a->Nc, a->q_pos0, a->m, q8, w8, sc, b0, nb,
-                                       i0, ni, st);
+                                       i0, ni, a->Tq <= 2, st);
       });
 }
 

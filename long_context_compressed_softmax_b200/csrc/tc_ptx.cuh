@@ -405,5 +405,23 @@ static bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, u
                               uint32_t box_cols, uint32_t box_rows) {
   return make_tmap_2d(m, base, 2, rows, cols, ld, box_cols, box_rows);
 }
+// 2D tensor map over rows of 128 packed 4-bit values (64 bytes a row) that
+// land unpacked: each run of 16 values (8 bytes) takes 16 bytes of shared
+// memory (the upper 8 left as padding), so a row fills one 128-byte swizzled
+// line, the layout tcgen05 reads 4-bit operands from.  Box: 128 values x
+// box_rows rows.  The copy credits the packed bytes (64 per row) to its
+// mbarrier.  Fails (false) unless base is 32-byte aligned.
+static bool make_tmap_u4x128_2d(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 31u) != 0) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {64};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 }  // namespace lcsa

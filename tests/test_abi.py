@@ -230,3 +230,11 @@ def test_attn_gather_mode_argument(lcsa):
     assert L.lcsa_set_attn_gather(2) == 1 and L.lcsa_set_attn_gather(-1) == 1
     assert L.lcsa_set_attn_gather(1) == 0
     assert L.lcsa_set_attn_gather(0) == 0
+
+
+def test_fp4_mma_mode_argument(lcsa):
+    """The MXFP4 key path switch takes 0 (E4M3 staging) or 1 (block-scaled MMA) only."""
+    L = lcsa.lib
+    assert L.lcsa_set_fp4_mma(2) == 1 and L.lcsa_set_fp4_mma(-1) == 1
+    assert L.lcsa_set_fp4_mma(0) == 0
+    assert L.lcsa_set_fp4_mma(1) == 0

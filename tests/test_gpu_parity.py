@@ -328,6 +328,83 @@ def test_indexer_mxfp4_wide_block_scales(lcsa):
     np.testing.assert_array_equal(idx[0].cpu().numpy(), O.topk_from_scores(np64(sc[0]), nv, k))
 
 
+def _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k):
+    """Scores and selection with the block-scaled MMA (default) and with the E4M3 staging path."""
+    try:
+        lcsa.set_fp4_mma(0)
+        staged = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    finally:
+        lcsa.set_fp4_mma(1)
+    direct = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    assert lcsa.get_device_status() == 0
+    return direct, staged
+
+
+@pytest.mark.parametrize("B,Tq,Nc,q_pos0,k", [
+    (2, 1, 3000, 12000, 512),       # decode: entry-range splits, ragged last tile
+    (3, 2, 1030, 4100, 256),        # two rows per sequence, ragged tail
+    (1, 1, 100, 400, 64),           # less than one tile
+    (2, 1, 20000, 80000, 2048),     # long rows: the code and scale rings wrap many times
+    (1, 2, 64, 40, 64),             # the second row sees one more entry than the first
+])
+def test_indexer_mxfp4_block_scaled_mma(lcsa, B, Tq, Nc, q_pos0, k):
+    # one- and two-row calls read the E2M1 codes and their block scales on the
+    # tensor cores: same scores as the oracle and as the E4M3 staging path
+    m = 4
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=47, device=DEV)
+    kc, ks = lcsa.quantize_mxfp4(x["k_idx"])
+    assert kc.data_ptr() % 32 == 0
+    (idx1, sc1), (idx0, sc0) = _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k)
+    for b in range(B):
+        rkc, rks = O.quantize_mxfp4(np64(x["k_idx"][b]))
+        _, ref_s = O.indexer_topk_mxfp4(np64(x["q_idx"][b]), np64(x["w"][b]), rkc, rks, q_pos0, m, k)
+        nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+        _score_err_ok(np64(sc1[b]), ref_s, nv)
+        np.testing.assert_array_equal(idx1[b].cpu().numpy(), O.topk_from_scores(np64(sc1[b]), nv, k))
+        for i in range(Tq):
+            n = nv[i]
+            r, d = ref_s[i, :n], np64(sc1[b])[i, :n] - np64(sc0[b])[i, :n]
+            # the same exact products summed in FP32 in another order
+            assert (np.abs(d) <= 1e-5 * np.maximum(np.abs(r), np.sqrt(np.mean(r * r)))).all()
+
+
+def test_indexer_mxfp4_block_scaled_wide_block_scales(lcsa):
+    # blocks 2^-13, 2^6 and 2^-20 away from the others: the block-scaled path
+    # keeps every product exact, the 2^-20 block included
+    B, Tq, Nc, m, k, q_pos0 = 1, 2, 300, 4, 64, 1400
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=44, device=DEV)
+    kf = x["k_idx"].float()
+    kf[0, :, 32:64] *= 2.0 ** -13
+    kf[0, :, 64:96] *= 2.0 ** 6
+    kf[0, 7, 96:128] *= 2.0 ** -20
+    k_idx = kf.to(torch.bfloat16)
+    kc, ks = lcsa.quantize_mxfp4(k_idx)
+    idx, sc = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    rkc, rks = O.quantize_mxfp4(np64(k_idx[0]))
+    _, ref_s = O.indexer_topk_mxfp4(np64(x["q_idx"][0]), np64(x["w"][0]), rkc, rks, q_pos0, m, k)
+    nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
+    for i in range(Tq):
+        r, g_ = ref_s[i, :nv[i]], np64(sc[0])[i, :nv[i]]
+        assert (np.abs(g_ - r) <= 1e-5 * np.maximum(np.abs(r), np.sqrt(np.mean(r * r)))).all()
+    np.testing.assert_array_equal(idx[0].cpu().numpy(), O.topk_from_scores(np64(sc[0]), nv, k))
+
+
+def test_indexer_mxfp4_codes_16_byte_aligned_take_staging(lcsa):
+    # codes 16 but not 32 bytes aligned: the call falls back to the staging
+    # path and gives its results bit for bit
+    B, Tq, Nc, m, k, q_pos0 = 2, 1, 900, 4, 128, 3600
+    x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=48, device=DEV)
+    kc, ks = lcsa.quantize_mxfp4(x["k_idx"])
+    buf = torch.empty(B * Nc * 64 + 16, dtype=torch.uint8, device=DEV)
+    kc16 = buf[16:].view(B, Nc, 64)
+    kc16.copy_(kc)
+    assert kc16.data_ptr() % 32 == 16
+    got = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc16, ks, q_pos0, m, k, return_scores=True)
+    (_, _), (idx0, sc0) = _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k)
+    nv = O.n_visible(q_pos0, m, Nc)
+    assert torch.equal(got[0], idx0) and torch.equal(got[1][..., :nv], sc0[..., :nv])
+
+
 def test_indexer_mxfp4_small_workspace_chunks(lcsa):
     B, Tq, Nc, m, k, q_pos0 = 2, 40, 900, 4, 128, 3600
     x = gen.make_indexer_inputs(B, Tq, Nc, 64, 128, "bf16", seed=45, device=DEV)
