@@ -105,13 +105,14 @@ lcsa_status lcsa_set_attn_gather(int mode);
 
 /* How lcsa_indexer_topk_mxfp4 feeds its MXFP4 keys to the tensor cores
  * (the pages give the FP4 QK path, [p2] "FP4 Quantization-Aware Training",
- * not its kernel): mode 1 (default) hands query groups of one or two rows
- * (decode) to a block-scaled MMA that reads the E2M1 codes and their UE8M0
- * block scales as they are; mode 0 stages every key as FP8 E4M3 relative to
- * its largest block scale first.  Scores agree to FP32 rounding order (and
- * mode 1 stays exact where mode 0 rounds a block more than 2^13 below its
- * entry's largest).  Process-wide; applies to calls issued after it.  Any
- * other value: LCSA_ERR_INVALID_ARG. */
+ * not its kernel): mode 0 (default) stages every key as FP8 E4M3 relative
+ * to its largest block scale before an E4M3 MMA; mode 1 hands calls of one
+ * or two query rows per sequence (decode) to a block-scaled MMA that reads
+ * the E2M1 codes and their UE8M0 block scales as they are.  Scores agree to
+ * FP32 rounding order, and mode 1 stays exact where mode 0 rounds a block
+ * more than 2^13 below its entry's largest; mode 0 is the faster on B200.
+ * Process-wide; applies to calls issued after it.  Any other value:
+ * LCSA_ERR_INVALID_ARG. */
 lcsa_status lcsa_set_fp4_mma(int mode);
 
 /* ------------------------------------------------------------------------
@@ -258,11 +259,11 @@ lcsa_status lcsa_quantize_mxfp4(const void* x, int64_t rows, int cols, lcsa_dtyp
  * dequantised values are exact and accumulate in FP32.  Each query head is
  * staged as FP8 E4M3 relative to its largest block scale, exact while its
  * block scales lie within 2^13 of it (a block further below rounds to the
- * E4M3 grid).  Keys: with one or two query rows per sequence (decode) the
- * tensor cores read the E2M1 codes with their block scales (exact for any
- * scales; see lcsa_set_fp4_mma); with more rows they are staged like the
- * queries.  The block-scaled path needs k_codes 32-byte aligned (any
- * allocation from the CUDA allocators is); 16-byte aligned codes are staged.
+ * E4M3 grid).  Keys are staged the same way, or, with lcsa_set_fp4_mma(1)
+ * and one or two query rows per sequence (decode), read by the tensor cores
+ * as E2M1 codes with their block scales (exact for any scales).  That path
+ * needs k_codes 32-byte aligned (any allocation from the CUDA allocators
+ * is); 16-byte aligned codes are staged.
  *
  *   q_idx     [B,Tq,64,128] BF16, 16-byte aligned; finite values
  *   w         [B,Tq,64] FP32

@@ -180,7 +180,7 @@ def set_attn_gather(mode: int) -> None:
 
 
 def set_fp4_mma(mode: int) -> None:
-    """MXFP4 indexer keys: 1 = block-scaled MMA on the codes for 1-2 row groups (default), 0 = E4M3 staging."""
+    """MXFP4 indexer keys: 0 = E4M3 staging (default), 1 = block-scaled MMA on the codes for 1-2 row calls."""
     _check(_lib.lcsa_set_fp4_mma(int(mode)), "set_fp4_mma")
 
 

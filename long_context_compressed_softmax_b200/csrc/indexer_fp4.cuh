@@ -341,8 +341,13 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Block-scaled variant for query groups of one or two rows (decode): the
-// codes go to the tensor cores as they are.  Per 128-entry tile:
+// Block-scaled variant for query groups of one or two rows (decode), taken
+// when lcsa_set_fp4_mma(1) asks for it: the codes go to the tensor cores as
+// they are, exact for any spread of block scales.  On B200 it is not the
+// faster one: 67.7 us against 65.5 us for the staging kernel on 8 sequences
+// x 262144 entries (ALU pipe 15 % busy instead of 55 %, tensor pipe 12 %,
+// DRAM 27 %), so the per-tile chain of one CTA per SM, not the
+// dequantisation, bounds both.  Per 128-entry tile:
 //   TMA        64-byte code rows -> 128-byte swizzled lines, each run of 16
 //              codes padded to 16 bytes (the 4-bit operand layout of
 //              tcgen05), 12-deep ring; 8 KB of HBM per tile
@@ -365,10 +370,11 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 // own entry's scale of block k in every column of group k, in every byte.
 // Warp roles (576 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
 // 2-9 epilogue, 10-17 scale writers.  Waits are bounded as in the E4M3 path.
-// 1: one- and two-row rectangles take the block-scaled kernel (default);
-// 0: every rectangle takes the E4M3 staging kernel (for comparison).
+// 0: every rectangle takes the E4M3 staging kernel (default: measured the
+// faster on B200, 544 against 564 us for 64 decode queries over 262144
+// entries); 1: calls of one or two rows take the block-scaled kernel.
 inline std::atomic<int>& fp4_mma_mode_ref() {
-  static std::atomic<int> mode{1};
+  static std::atomic<int> mode{0};
   return mode;
 }
 inline int fp4_mma_mode() { return fp4_mma_mode_ref().load(std::memory_order_relaxed); }

@@ -328,14 +328,19 @@ def test_indexer_mxfp4_wide_block_scales(lcsa):
     np.testing.assert_array_equal(idx[0].cpu().numpy(), O.topk_from_scores(np64(sc[0]), nv, k))
 
 
-def _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k):
-    """Scores and selection with the block-scaled MMA (default) and with the E4M3 staging path."""
+def _mxfp4_direct(lcsa, *args, **kw):
+    """The call with the block-scaled MMA on the E2M1 keys (mode 1), then back to the default."""
     try:
-        lcsa.set_fp4_mma(0)
-        staged = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
-    finally:
         lcsa.set_fp4_mma(1)
-    direct = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+        return lcsa.indexer_topk_mxfp4(*args, **kw)
+    finally:
+        lcsa.set_fp4_mma(0)
+
+
+def _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k):
+    """Scores and selection with the block-scaled MMA and with the E4M3 staging path (default)."""
+    direct = _mxfp4_direct(lcsa, x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    staged = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
     assert lcsa.get_device_status() == 0
     return direct, staged
 
@@ -379,7 +384,7 @@ def test_indexer_mxfp4_block_scaled_wide_block_scales(lcsa):
     kf[0, 7, 96:128] *= 2.0 ** -20
     k_idx = kf.to(torch.bfloat16)
     kc, ks = lcsa.quantize_mxfp4(k_idx)
-    idx, sc = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
+    idx, sc = _mxfp4_direct(lcsa, x["q_idx"], x["w"], kc, ks, q_pos0, m, k, return_scores=True)
     rkc, rks = O.quantize_mxfp4(np64(k_idx[0]))
     _, ref_s = O.indexer_topk_mxfp4(np64(x["q_idx"][0]), np64(x["w"][0]), rkc, rks, q_pos0, m, k)
     nv = [O.n_visible(q_pos0 + i, m, Nc) for i in range(Tq)]
@@ -399,7 +404,7 @@ def test_indexer_mxfp4_codes_16_byte_aligned_take_staging(lcsa):
     kc16 = buf[16:].view(B, Nc, 64)
     kc16.copy_(kc)
     assert kc16.data_ptr() % 32 == 16
-    got = lcsa.indexer_topk_mxfp4(x["q_idx"], x["w"], kc16, ks, q_pos0, m, k, return_scores=True)
+    got = _mxfp4_direct(lcsa, x["q_idx"], x["w"], kc16, ks, q_pos0, m, k, return_scores=True)
     (_, _), (idx0, sc0) = _mxfp4_both_paths(lcsa, x, kc, ks, q_pos0, m, k)
     nv = O.n_visible(q_pos0, m, Nc)
     assert torch.equal(got[0], idx0) and torch.equal(got[1][..., :nv], sc0[..., :nv])
