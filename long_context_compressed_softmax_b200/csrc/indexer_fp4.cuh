@@ -353,9 +353,7 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 //              tcgen05), 12-deep ring; 8 KB of HBM per tile
 //   scales     8 warps (two per TMEM lane quarter, alternate tiles) write
 //              each entry's four UE8M0 block scales to TMEM; each loads the
-//              scale words of its next 8 tiles ahead (16 tiles of
-//              lookahead: the words come from DRAM, whose latency under
-//              this load is several tiles long)
+//              scale words of its next 8 tiles ahead
 //   MMA        tcgen05 kind::mxf8f6f4 with block scaling: A = E2M1 keys with
 //              their scales, B = E4M3 queries with scale 1, K = 32 per
 //              instruction (one scale per row), FP32 accumulate, so every
@@ -370,9 +368,11 @@ indexer_fp4_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_const
 // own entry's scale of block k in every column of group k, in every byte.
 // Warp roles (576 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
 // 2-9 epilogue, 10-17 scale writers.  Waits are bounded as in the E4M3 path.
-// 0: every rectangle takes the E4M3 staging kernel (default: measured the
-// faster on B200, 544 against 564 us for 64 decode queries over 262144
-// entries); 1: calls of one or two rows take the block-scaled kernel.
+
+// Key path of the FP4 indexer call.  0: every rectangle takes the E4M3
+// staging kernel (default: measured the faster on B200, 544 against 564 us
+// for 64 decode queries over 262144 entries); 1: calls of one or two rows
+// take the block-scaled kernel.
 inline std::atomic<int>& fp4_mma_mode_ref() {
   static std::atomic<int> mode{0};
   return mode;
@@ -390,7 +390,8 @@ constexpr uint32_t kMxCTx = kIxTileE * 64;     // bytes the copy of a tile credi
 constexpr uint32_t kMxAccCols = 384;
 constexpr uint32_t kMxSfB = 384;               // B scales (all 1)
 constexpr uint32_t kMxSfA = 400;               // A-scale buffers
-static_assert(kMxSfA + 16 * kMxSf <= 512, "TMEM columns of the block-scaled indexer");
+static_assert(kMxAccCols <= kMxSfB && kMxSfB + 16 <= kMxSfA && kMxSfA + 16 * kMxSf <= 512,
+              "TMEM columns of the block-scaled indexer");
 constexpr int kMxBars = 1 + 2 * kMxStages + 2 * kMxSf + 2 * 6;
 constexpr size_t kMxSmem = 1024 + kMxQBytes + kMxStages * kMxCBytes + kIxRows * 64 * 4 + kMxBars * 8;
 static_assert(kMxSmem + 64 <= 232448, "shared memory of the block-scaled indexer kernel");
@@ -459,8 +460,8 @@ indexer_mx_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_consta
   const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
   if (n_tiles == 0) return;
   const long long rect_row = (long long)bl * g.ni + (i_first - g.i0);
-  const int n_acc = rows == 1 ? 6 : 3;
   const uint32_t acc_cols = 64u * (uint32_t)rows;
+  const int n_acc = (int)(kMxAccCols / acc_cols);     // 6 or 3 accumulators
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
